@@ -1,0 +1,17 @@
+"""Block-sparse self-attention for video DiTs with hybrid top-k + top-p block masks, on B200.
+
+The compute path is the C-ABI library ``libbsa.so`` (hand-written sm_100a CUDA kernels).  The
+Python functions re-exported here are argument marshalling around that library; importing them
+loads it and fails loudly if it has not been built.  ``workloads`` (seeded inputs) does not need
+the library.
+"""
+_API = ("pool_blocks", "select_mask_topk_topp", "select_from_logits", "block_sparse_attn_fwd",
+        "dense_attn_fwd", "sparse_attention", "SAError", "lib")
+
+
+def __getattr__(name):
+    if name in _API:
+        from . import sparse_attn
+
+        return getattr(sparse_attn, name)
+    raise AttributeError(name)

@@ -1,0 +1,188 @@
+"""fp64 CPU oracle for block-sparse attention with hybrid top-k + top-p block masks.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, the package smoke check and the benchmark's
+CPU-baseline leg may import this module.  The CUDA path never imports it, and it never imports
+the CUDA path: the two share nothing but the seeded input generator.
+
+The arithmetic lives in ``oracle.c`` (plain fp64 loops, OpenMP over rows).  This module only
+compiles it, loads it with ctypes and marshals numpy arrays.  Each function cites the passage it
+follows in its C definition.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so (plain -O2, no fast-math, portable ISA)."""
+    if (not force and os.path.exists(_LIB)
+            and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC)):
+        return _LIB
+    tmp = _LIB + ".tmp%d" % os.getpid()
+    cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", _SRC, "-o", tmp, "-lm"]
+    subprocess.check_call(cmd)
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    build()
+    lib = ctypes.CDLL(_LIB)
+    P = ctypes.c_void_p
+    I = ctypes.c_int64
+    D = ctypes.c_double
+    lib.or_num_threads.restype = ctypes.c_int
+    lib.or_pool_blocks.argtypes = [P, I, I, I, I, P]
+    lib.or_block_probs.argtypes = [P, P, I, I, I, I, D, P]
+    lib.or_softmax_rows.argtypes = [P, I, I, P]
+    lib.or_select_rows.argtypes = [P, I, I, I, D, P, P, P, P, P, P, P, P]
+    lib.or_masked_attention.argtypes = [P, P, P, I, I, I, P, D, P, P, I, P]
+    lib.or_dense_attention.argtypes = [P, P, P, I, I, D, P, P, I, P]
+    for f in (lib.or_pool_blocks, lib.or_block_probs, lib.or_softmax_rows, lib.or_select_rows,
+              lib.or_masked_attention, lib.or_dense_attention):
+        f.restype = None
+    _lib = lib
+    return lib
+
+
+def _ptr(a: np.ndarray):
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def _bits(x: np.ndarray) -> np.ndarray:
+    """bf16 tensors travel as their uint16 bit patterns."""
+    x = np.ascontiguousarray(x)
+    if x.dtype != np.uint16:
+        raise TypeError("bf16 inputs must be given as uint16 bit patterns, got %s" % x.dtype)
+    return x
+
+
+def num_threads() -> int:
+    return int(_load().or_num_threads())
+
+
+def pool_blocks(x_bits: np.ndarray, bs: int) -> np.ndarray:
+    """Mean of each block of bs tokens (tail block: mean of its valid tokens).
+
+    x_bits: [..., N, d] uint16 (bf16 bits).  Returns [..., nb, d] float64.
+    """
+    x = _bits(x_bits)
+    *lead, N, d = x.shape
+    BH = int(np.prod(lead)) if lead else 1
+    nb = (N + bs - 1) // bs
+    out = np.empty((BH, nb, d), np.float64)
+    _load().or_pool_blocks(_ptr(x), BH, N, d, bs, _ptr(out))
+    return out.reshape(*lead, nb, d)
+
+
+def block_probs(qp: np.ndarray, kp: np.ndarray, scale: float) -> np.ndarray:
+    """Row softmax of the pooled block scores Qp Kp^T * scale.  qp: [..., nbq, d]."""
+    qp = np.ascontiguousarray(qp, np.float64)
+    kp = np.ascontiguousarray(kp, np.float64)
+    *lead, nbq, d = qp.shape
+    nbk = kp.shape[-2]
+    BH = int(np.prod(lead)) if lead else 1
+    out = np.empty((BH, nbq, nbk), np.float64)
+    _load().or_block_probs(_ptr(qp), _ptr(kp), BH, nbq, nbk, d, float(scale), _ptr(out))
+    return out.reshape(*lead, nbq, nbk)
+
+
+def softmax_rows(logits: np.ndarray) -> np.ndarray:
+    x = np.ascontiguousarray(logits, np.float64)
+    n = x.shape[-1]
+    rows = x.size // n if n else 0
+    out = np.empty_like(x)
+    _load().or_softmax_rows(_ptr(x), rows, n, _ptr(out))
+    return out
+
+
+class Selection:
+    """Per-row result of the hybrid selection, with the diagnostics the parity rule needs."""
+
+    def __init__(self, mask, cnt, tau_k, tau_p, m_p, cum_lo, cum_hi, rank, prob, topk, topp):
+        self.mask, self.cnt = mask, cnt
+        self.tau_k, self.tau_p, self.m_p = tau_k, tau_p, m_p
+        self.cum_lo, self.cum_hi, self.rank = cum_lo, cum_hi, rank
+        self.prob, self.topk, self.topp = prob, topk, topp
+
+
+def select_from_probs(prob: np.ndarray, topk: int, topp: float) -> Selection:
+    """Hybrid top-k union top-p selection applied row by row to block probabilities."""
+    P = np.ascontiguousarray(prob, np.float64)
+    *lead, nb = P.shape
+    rows = int(np.prod(lead)) if lead else 1
+    mask = np.empty((rows, nb), np.uint8)
+    cnt = np.empty(rows, np.int32)
+    tau_k = np.empty(rows, np.float64)
+    tau_p = np.empty(rows, np.float64)
+    m_p = np.empty(rows, np.int32)
+    lo = np.empty(rows, np.float64)
+    hi = np.empty(rows, np.float64)
+    rank = np.empty((rows, nb), np.int32)
+    _load().or_select_rows(_ptr(P), rows, nb, int(topk), float(topp), _ptr(mask), _ptr(cnt),
+                           _ptr(tau_k), _ptr(tau_p), _ptr(m_p), _ptr(lo), _ptr(hi), _ptr(rank))
+    shp = tuple(lead)
+    return Selection(mask.reshape(*shp, nb), cnt.reshape(shp), tau_k.reshape(shp),
+                     tau_p.reshape(shp), m_p.reshape(shp), lo.reshape(shp), hi.reshape(shp),
+                     rank.reshape(*shp, nb), P, topk, topp)
+
+
+def select_from_logits(logits: np.ndarray, topk: int, topp: float) -> Selection:
+    return select_from_probs(softmax_rows(logits), topk, topp)
+
+
+def select(qp: np.ndarray, kp: np.ndarray, topk: int, topp: float, scale: float) -> Selection:
+    """Block scores, row softmax and hybrid selection from pooled Q and K."""
+    return select_from_probs(block_probs(qp, kp, scale), topk, topp)
+
+
+def masked_attention(q_bits, k_bits, v_bits, mask, bs: int, scale: float, sel=None):
+    """Attention restricted to the kept key blocks of each query block.
+
+    q/k/v_bits: [BH, N, d] uint16; mask: [BH, nb, nb] 0/1.
+    sel: optional list of (bh, i) query blocks; default all.  Returns [nsel, bs, d] float64
+    (rows at or beyond N are zero) and the selection arrays.
+    """
+    q, k, v = _bits(q_bits), _bits(k_bits), _bits(v_bits)
+    BH, N, d = q.shape
+    nb = (N + bs - 1) // bs
+    m = np.ascontiguousarray(mask, np.uint8).reshape(BH, nb, nb)
+    if sel is None:
+        sel = [(bh, i) for bh in range(BH) for i in range(nb)]
+    sel = np.asarray(sel, np.int64).reshape(-1, 2)
+    sb = np.ascontiguousarray(sel[:, 0])
+    si = np.ascontiguousarray(sel[:, 1])
+    out = np.zeros((len(sel), bs, d), np.float64)
+    _load().or_masked_attention(_ptr(q), _ptr(k), _ptr(v), N, d, bs, _ptr(m), float(scale),
+                                _ptr(sb), _ptr(si), len(sel), _ptr(out))
+    return out
+
+
+def dense_attention(q_bits, k_bits, v_bits, scale: float, rows=None):
+    """Full softmax attention.  rows: optional list of (bh, t); default every row.
+
+    Returns [nrows, d] float64.
+    """
+    q, k, v = _bits(q_bits), _bits(k_bits), _bits(v_bits)
+    BH, N, d = q.shape
+    if rows is None:
+        rows = [(bh, t) for bh in range(BH) for t in range(N)]
+    rows = np.asarray(rows, np.int64).reshape(-1, 2)
+    sb = np.ascontiguousarray(rows[:, 0])
+    st = np.ascontiguousarray(rows[:, 1])
+    out = np.zeros((len(rows), d), np.float64)
+    _load().or_dense_attention(_ptr(q), _ptr(k), _ptr(v), N, d, float(scale), _ptr(sb), _ptr(st),
+                               len(rows), _ptr(out))
+    return out

@@ -1,0 +1,323 @@
+/*
+ * Reference oracle for block-sparse attention with hybrid top-k + top-p block masks.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is a plain, slow, fp64 CPU statement of what the
+ * block-sparse attention path computes.  Only the test suite, the package's smoke check and
+ * the benchmark's CPU-baseline leg may load it.  It shares no code, header, table or helper
+ * with the CUDA path, and it never reads anything the CUDA path produced.
+ *
+ * Sources (page title, section):
+ *   [SA2]  "SpargeAttention2とは？Top-k+Top-pハイブリッドマスキングでビデオ生成を16.2倍高速化",
+ *          section "Top-kとTop-pの限界を解剖する" (top-k keeps the k largest probabilities; top-p
+ *          takes blocks from the top until the cumulative probability passes p) and section
+ *          "ハイブリッドマスキングと蒸留微調整" (the hybrid mask is the union of both sets).
+ *   [SVG2] "Sparse VideoGen2: Accelerate Video Generation with Sparse Attention via
+ *          Semantic-Aware Permutation", section 1 (block representatives by mean pooling) and
+ *          section 2.B (scores between representatives, sorted, cumulative top-p that reaches p).
+ *   The block size, mean pooling, the 1/sqrt(d) score scale and the bf16 [B,H,N,d] layout are
+ *   fixed by the problem statement this library implements; the pages leave them open.
+ *
+ * Readings where the pages are silent (each one is listed in the design notes):
+ *   - pooling is the mean over the valid tokens of a block (a tail block has fewer than bs);
+ *   - block probabilities are softmax_j(Qp_i . Kp_j * scale) over all key blocks of the row;
+ *   - ranking is by probability descending, ties broken by the lower block index;
+ *   - top-p keeps the shortest ranked prefix whose cumulative probability is >= p
+ *     ("reaches", [SVG2] 2.B); p <= 0 keeps nothing, p >= 1 keeps every block;
+ *   - keys at or beyond N never enter attention; a query block with no kept key block
+ *     produces zeros.
+ *
+ * Parity pins: every function here is pinned in tests/test_oracle_pins.py against closed forms,
+ * brute force and independent library routines (numpy, scipy, torch), not against itself.
+ *
+ * Everything is fp64.  bf16 inputs arrive as their raw 16-bit patterns and are widened exactly.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* exact widening of a bf16 bit pattern: it is the top half of an IEEE binary32 */
+static double bf16_to_double(uint16_t bits) {
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+int or_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* ---------------------------------------------------------------------------------------------
+ * Block representatives: xp[bh, i, c] = mean over tokens t of block i (t < N) of x[bh, t, c].
+ * [SVG2] section 1 names mean pooling of contiguous token blocks as the representative.
+ * x: [BH, N, d] bf16 bits.  xp: [BH, nb, d] fp64, nb = ceil(N / bs).
+ * ------------------------------------------------------------------------------------------- */
+void or_pool_blocks(const uint16_t *x, int64_t BH, int64_t N, int64_t d, int64_t bs, double *xp) {
+    int64_t nb = (N + bs - 1) / bs;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t bh = 0; bh < BH; ++bh) {
+        for (int64_t i = 0; i < nb; ++i) {
+            int64_t t0 = i * bs;
+            int64_t t1 = t0 + bs < N ? t0 + bs : N;
+            double n = (double)(t1 - t0);
+            for (int64_t c = 0; c < d; ++c) {
+                double s = 0.0;
+                for (int64_t t = t0; t < t1; ++t) s += bf16_to_double(x[(bh * N + t) * d + c]);
+                xp[(bh * nb + i) * d + c] = s / n;
+            }
+        }
+    }
+}
+
+/* ---------------------------------------------------------------------------------------------
+ * Block scores and their row softmax ([SVG2] 2.B: scores between representatives stand in
+ * for the full attention map; the problem statement fixes softmax(Qp Kp^T * scale)).
+ * qp: [BH, nbq, d], kp: [BH, nbk, d] fp64.  prob: [BH, nbq, nbk] fp64.
+ * ------------------------------------------------------------------------------------------- */
+void or_block_probs(const double *qp, const double *kp, int64_t BH, int64_t nbq, int64_t nbk,
+                    int64_t d, double scale, double *prob) {
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t bh = 0; bh < BH; ++bh) {
+        for (int64_t i = 0; i < nbq; ++i) {
+            const double *q = qp + (bh * nbq + i) * d;
+            double *row = prob + (bh * nbq + i) * nbk;
+            double mx = -INFINITY;
+            for (int64_t j = 0; j < nbk; ++j) {
+                const double *k = kp + (bh * nbk + j) * d;
+                double s = 0.0;
+                for (int64_t c = 0; c < d; ++c) s += q[c] * k[c];
+                row[j] = s * scale;
+                if (row[j] > mx) mx = row[j];
+            }
+            double z = 0.0;
+            for (int64_t j = 0; j < nbk; ++j) {
+                row[j] = exp(row[j] - mx);
+                z += row[j];
+            }
+            for (int64_t j = 0; j < nbk; ++j) row[j] /= z;
+        }
+    }
+}
+
+/* softmax of given logits, row by row (used to feed hand-made rows into the selection) */
+void or_softmax_rows(const double *logits, int64_t rows, int64_t n, double *prob) {
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        const double *x = logits + r * n;
+        double *y = prob + r * n;
+        double mx = -INFINITY;
+        for (int64_t j = 0; j < n; ++j) if (x[j] > mx) mx = x[j];
+        double z = 0.0;
+        for (int64_t j = 0; j < n; ++j) { y[j] = exp(x[j] - mx); z += y[j]; }
+        for (int64_t j = 0; j < n; ++j) y[j] /= z;
+    }
+}
+
+/* ---------------------------------------------------------------------------------------------
+ * Hybrid selection, one row at a time ([SA2] "Top-kとTop-pの限界を解剖する" and
+ * "ハイブリッドマスキングと蒸留微調整"; [SVG2] 2.B for the sort-then-accumulate top-p).
+ *
+ *   order  : block ids sorted by probability descending, lower id first on equal probability
+ *   S_k    : the first min(k, nb) blocks of the order
+ *   S_p    : the first m blocks, m the least count with sum of their probabilities >= p
+ *            (p <= 0: m = 0; p >= 1: m = nb)
+ *   keep   : S_k union S_p
+ *
+ * Outputs per row: mask[nb] (0/1), cnt (|keep|), and diagnostics used by the parity rule:
+ *   tau_k  : probability of the last block of S_k (NaN if S_k is empty)
+ *   tau_p  : probability of the last block of S_p (NaN if S_p is empty)
+ *   m_p    : |S_p|
+ *   cum_lo : sum of the first m-1 ranked probabilities (the mass just before the cut)
+ *   cum_hi : sum of the first m ranked probabilities (the mass at the cut)
+ *   rank   : rank[j] = position of block j in the order
+ * ------------------------------------------------------------------------------------------- */
+typedef struct {
+    double p;
+    int32_t j;
+} ranked_t;
+
+static int ranked_cmp(const void *a, const void *b) {
+    const ranked_t *x = (const ranked_t *)a, *y = (const ranked_t *)b;
+    if (x->p > y->p) return -1;
+    if (x->p < y->p) return 1;
+    return (x->j > y->j) - (x->j < y->j);
+}
+
+void or_select_rows(const double *prob, int64_t rows, int64_t nb, int64_t topk, double topp,
+                    uint8_t *mask, int32_t *cnt, double *tau_k, double *tau_p, int32_t *m_p,
+                    double *cum_lo, double *cum_hi, int32_t *rank) {
+#pragma omp parallel
+    {
+        ranked_t *ord = (ranked_t *)malloc(sizeof(ranked_t) * (size_t)(nb > 0 ? nb : 1));
+        uint8_t *in_k = (uint8_t *)malloc((size_t)(nb > 0 ? nb : 1));
+        uint8_t *in_p = (uint8_t *)malloc((size_t)(nb > 0 ? nb : 1));
+#pragma omp for schedule(static)
+        for (int64_t r = 0; r < rows; ++r) {
+            const double *P = prob + r * nb;
+            for (int64_t j = 0; j < nb; ++j) { ord[j].p = P[j]; ord[j].j = (int32_t)j; }
+            qsort(ord, (size_t)nb, sizeof(ranked_t), ranked_cmp);
+            if (rank) for (int64_t q = 0; q < nb; ++q) rank[r * nb + ord[q].j] = (int32_t)q;
+
+            /* top-k: the k largest probabilities */
+            int64_t kk = topk < nb ? topk : nb;
+            if (kk < 0) kk = 0;
+            memset(in_k, 0, (size_t)nb);
+            for (int64_t q = 0; q < kk; ++q) in_k[ord[q].j] = 1;
+
+            /* top-p: shortest ranked prefix whose cumulative probability reaches p */
+            int64_t m;
+            double lo = 0.0, hi = 0.0;
+            if (topp <= 0.0) {
+                m = 0;
+            } else if (topp >= 1.0) {
+                m = nb;
+                for (int64_t q = 0; q < nb; ++q) { lo = hi; hi += ord[q].p; }
+            } else {
+                double cum = 0.0;
+                m = nb;
+                for (int64_t q = 0; q < nb; ++q) {
+                    lo = cum;
+                    cum += ord[q].p;
+                    hi = cum;
+                    if (cum >= topp) { m = q + 1; break; }
+                }
+            }
+            memset(in_p, 0, (size_t)nb);
+            for (int64_t q = 0; q < m; ++q) in_p[ord[q].j] = 1;
+
+            /* hybrid: union of the two sets */
+            int32_t c = 0;
+            for (int64_t j = 0; j < nb; ++j) {
+                uint8_t keep = (uint8_t)(in_k[j] | in_p[j]);
+                mask[r * nb + j] = keep;
+                c += keep;
+            }
+            cnt[r] = c;
+            if (tau_k) tau_k[r] = kk > 0 ? ord[kk - 1].p : NAN;
+            if (tau_p) tau_p[r] = m > 0 ? ord[m - 1].p : NAN;
+            if (m_p) m_p[r] = (int32_t)m;
+            if (cum_lo) cum_lo[r] = lo;
+            if (cum_hi) cum_hi[r] = hi;
+        }
+        free(ord);
+        free(in_k);
+        free(in_p);
+    }
+}
+
+/* ---------------------------------------------------------------------------------------------
+ * Masked attention: for every query token t of query block i (t < N),
+ *   O[t] = sum_{s in kept blocks of i, s < N} softmax_s(scale * Q[t].K[s]) V[s]
+ * with the softmax normalised over the kept keys only; two passes (max, then sum) in fp64.
+ * A query block with no kept key block yields O = 0.
+ *
+ * q, k, v: [BH, N, d] bf16 bits.  mask: [BH, nbq, nbk] 0/1 with nbq = nbk = ceil(N / bs).
+ * The query blocks to evaluate are listed in (sel_bh[s], sel_i[s]) for s < nsel; their rows are
+ * written to out[s, r, :] for r < bs (rows at or beyond N are left at 0).  out: [nsel, bs, d].
+ * ------------------------------------------------------------------------------------------- */
+void or_masked_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t N,
+                         int64_t d, int64_t bs, const uint8_t *mask, double scale,
+                         const int64_t *sel_bh, const int64_t *sel_i, int64_t nsel, double *out) {
+    int64_t nb = (N + bs - 1) / bs;
+#pragma omp parallel
+    {
+        double *w = (double *)malloc(sizeof(double) * (size_t)N);
+        double *qr = (double *)malloc(sizeof(double) * (size_t)d);
+        double *acc = (double *)malloc(sizeof(double) * (size_t)d);
+#pragma omp for collapse(2) schedule(dynamic, 1)
+        for (int64_t s = 0; s < nsel; ++s) {
+            for (int64_t r = 0; r < bs; ++r) {
+                int64_t bh = sel_bh[s], i = sel_i[s];
+                int64_t t = i * bs + r;
+                double *o = out + (s * bs + r) * d;
+                for (int64_t c = 0; c < d; ++c) o[c] = 0.0;
+                if (t >= N) continue;
+                const uint8_t *mrow = mask + (bh * nb + i) * nb;
+                for (int64_t c = 0; c < d; ++c) qr[c] = bf16_to_double(q[(bh * N + t) * d + c]);
+                /* pass 1: logits of the kept keys and their maximum */
+                double mx = -INFINITY;
+                int any = 0;
+                for (int64_t j = 0; j < nb; ++j) {
+                    if (!mrow[j]) continue;
+                    int64_t s1 = (j + 1) * bs < N ? (j + 1) * bs : N;
+                    for (int64_t sk = j * bs; sk < s1; ++sk) {
+                        const uint16_t *kr = k + (bh * N + sk) * d;
+                        double x = 0.0;
+                        for (int64_t c = 0; c < d; ++c) x += qr[c] * bf16_to_double(kr[c]);
+                        x *= scale;
+                        w[sk] = x;
+                        if (x > mx) mx = x;
+                        any = 1;
+                    }
+                }
+                if (!any) continue;
+                /* pass 2: normaliser and weighted sum of values */
+                double z = 0.0;
+                for (int64_t c = 0; c < d; ++c) acc[c] = 0.0;
+                for (int64_t j = 0; j < nb; ++j) {
+                    if (!mrow[j]) continue;
+                    int64_t s1 = (j + 1) * bs < N ? (j + 1) * bs : N;
+                    for (int64_t sk = j * bs; sk < s1; ++sk) {
+                        double e = exp(w[sk] - mx);
+                        z += e;
+                        const uint16_t *vr = v + (bh * N + sk) * d;
+                        for (int64_t c = 0; c < d; ++c) acc[c] += e * bf16_to_double(vr[c]);
+                    }
+                }
+                for (int64_t c = 0; c < d; ++c) o[c] = acc[c] / z;
+            }
+        }
+        free(w);
+        free(qr);
+        free(acc);
+    }
+}
+
+/* ---------------------------------------------------------------------------------------------
+ * Dense attention, the 0 %-sparsity control: O[t] = sum_{s<N} softmax_s(scale Q[t].K[s]) V[s].
+ * Written without blocks so that it is an independent statement of the same softmax.
+ * Rows to evaluate: (sel_bh[s], sel_t[s]); out: [nsel, d].
+ * ------------------------------------------------------------------------------------------- */
+void or_dense_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t N,
+                        int64_t d, double scale, const int64_t *sel_bh, const int64_t *sel_t,
+                        int64_t nsel, double *out) {
+#pragma omp parallel
+    {
+        double *w = (double *)malloc(sizeof(double) * (size_t)N);
+        double *qr = (double *)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic, 8)
+        for (int64_t s = 0; s < nsel; ++s) {
+            int64_t bh = sel_bh[s], t = sel_t[s];
+            double *o = out + s * d;
+            for (int64_t c = 0; c < d; ++c) qr[c] = bf16_to_double(q[(bh * N + t) * d + c]);
+            double mx = -INFINITY;
+            for (int64_t sk = 0; sk < N; ++sk) {
+                const uint16_t *kr = k + (bh * N + sk) * d;
+                double x = 0.0;
+                for (int64_t c = 0; c < d; ++c) x += qr[c] * bf16_to_double(kr[c]);
+                w[sk] = x * scale;
+                if (w[sk] > mx) mx = w[sk];
+            }
+            double z = 0.0;
+            for (int64_t c = 0; c < d; ++c) o[c] = 0.0;
+            for (int64_t sk = 0; sk < N; ++sk) {
+                double e = exp(w[sk] - mx);
+                z += e;
+                const uint16_t *vr = v + (bh * N + sk) * d;
+                for (int64_t c = 0; c < d; ++c) o[c] += e * bf16_to_double(vr[c]);
+            }
+            for (int64_t c = 0; c < d; ++c) o[c] /= z;
+        }
+        free(w);
+        free(qr);
+    }
+}

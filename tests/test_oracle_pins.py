@@ -1,0 +1,303 @@
+"""Pins for the fp64 oracle against facts that do not come from the oracle itself.
+
+Each test checks one oracle function against a closed form, an invariant the pages state, a
+brute-force enumeration, or an independent library routine (numpy / scipy / torch in float64).
+The set is chosen so that a plausible slip in the oracle (a dropped term, a wrong sign or index,
+a transposed operand, an off-by-one at the top-p cut, the wrong tie order) fails at least one of
+them; tests/test_oracle_mutants.py compiles such slips into the C source and checks that they do.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+
+from block_sparse_attention_blocks_b200.workloads import f32_to_bf16_bits, bf16_bits_to_f32
+
+
+def bits(x):
+    return f32_to_bf16_bits(np.asarray(x, np.float32))
+
+
+def widen(b):
+    return bf16_bits_to_f32(b).astype(np.float64)
+
+
+# ------------------------------------------------------------------------------------------------
+# pooling: mean over the valid tokens of each block
+# ------------------------------------------------------------------------------------------------
+def test_pool_constant_blocks(orc):
+    bs, nb, d = 16, 5, 8
+    vals = np.array([1.5, -2.0, 0.25, 7.0, -0.125], np.float32)
+    x = np.repeat(vals, bs)[:, None] * np.ones((1, d), np.float32)
+    xp = orc.pool_blocks(bits(x)[None], bs)[0]
+    assert np.array_equal(xp, np.repeat(vals.astype(np.float64)[:, None], d, 1))
+
+
+def test_pool_ramp_midpoint_and_tail(orc):
+    # x_t = t within the block (exact in bf16); the mean of 0..n-1 is (n-1)/2, also for the tail
+    bs, N, d = 64, 64 * 3 + 10, 4
+    t = np.arange(N) % bs
+    x = np.repeat(t[:, None], d, 1).astype(np.float32)
+    xp = orc.pool_blocks(bits(x)[None], bs)[0]
+    want = np.array([31.5, 31.5, 31.5, 4.5])
+    assert np.array_equal(xp[:, 0], want)
+    assert xp.shape == (4, d)
+
+
+def test_pool_matches_numpy_mean(orc):
+    rng = np.random.default_rng(1)
+    BH, N, d, bs = 3, 300, 16, 64
+    xb = bits(rng.standard_normal((BH, N, d)))
+    xp = orc.pool_blocks(xb, bs)
+    xf = widen(xb)
+    for i in range(xp.shape[1]):
+        ref = xf[:, i * bs:min((i + 1) * bs, N)].mean(axis=1)
+        np.testing.assert_allclose(xp[:, i], ref, rtol=0, atol=1e-14)
+
+
+# ------------------------------------------------------------------------------------------------
+# block probabilities: softmax(Qp Kp^T * scale) per query-block row
+# ------------------------------------------------------------------------------------------------
+def test_block_probs_match_scipy(orc):
+    from scipy.special import softmax
+
+    rng = np.random.default_rng(2)
+    qp = rng.standard_normal((2, 7, 16))
+    kp = rng.standard_normal((2, 9, 16))
+    scale = 0.37
+    P = orc.block_probs(qp, kp, scale)
+    ref = softmax(np.einsum("bic,bjc->bij", qp, kp) * scale, axis=-1)
+    np.testing.assert_allclose(P, ref, rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(P.sum(-1), 1.0, rtol=0, atol=1e-12)
+
+
+def test_block_probs_uniform_and_two_blocks(orc):
+    P = orc.block_probs(np.zeros((1, 3, 4)), np.ones((1, 5, 4)), 1.0)
+    assert np.allclose(P, 0.2, rtol=0, atol=1e-15)
+    # two key blocks with logits a, b: P0 = 1 / (1 + exp(b - a))
+    qp = np.array([[[1.0, 0.0]]])
+    kp = np.array([[[2.0, 0.0], [-1.0, 5.0]]])
+    P = orc.block_probs(qp, kp, 0.5)[0, 0]
+    assert abs(P[0] - 1.0 / (1.0 + math.exp(-0.5 - 1.0))) < 1e-15
+    # the score uses Qp_i . Kp_j, not Kp_i . Qp_j: an asymmetric case tells them apart
+    qp2 = np.array([[[1.0, 0.0], [0.0, 1.0]]])
+    kp2 = np.array([[[3.0, 0.0], [0.0, 0.0]]])
+    P2 = orc.block_probs(qp2, kp2, 1.0)[0]
+    assert abs(P2[0, 0] - 1.0 / (1.0 + math.exp(-3.0))) < 1e-15
+    assert abs(P2[1, 0] - 0.5) < 1e-15
+
+
+# ------------------------------------------------------------------------------------------------
+# hybrid selection: top-k union top-p (SpargeAttention2), top-p reaching p (SVG2 2.B)
+# ------------------------------------------------------------------------------------------------
+def _set(mask_row):
+    return set(np.nonzero(mask_row)[0].tolist())
+
+
+def test_select_worked_example(orc):
+    # P = (0.5, 0.3, 0.15, 0.05), fed as probabilities (exact) and as logits ln P
+    P = np.array([[0.5, 0.3, 0.15, 0.05]])
+    s = orc.select_from_probs(P, 1, 0.7)
+    assert _set(s.mask[0]) == {0, 1}
+    s = orc.select_from_probs(P, 3, 0.7)
+    assert _set(s.mask[0]) == {0, 1, 2}
+    s = orc.select_from_probs(P, 0, 0.96)
+    assert _set(s.mask[0]) == {0, 1, 2, 3}
+    # cumulative mass equals p exactly: "reaches p" keeps one block
+    s = orc.select_from_probs(P, 0, 0.5)
+    assert _set(s.mask[0]) == {0} and s.m_p[0] == 1 and s.cum_hi[0] == 0.5
+    # via logits the cut at exactly p is decided by rounding: the oracle reports the masses
+    s = orc.select_from_logits(np.log(P), 0, 0.5)
+    assert s.m_p[0] in (1, 2) and abs(s.cum_hi[0] - 0.5) < 1e-12 or abs(s.cum_lo[0] - 0.5) < 1e-12
+
+
+def test_select_uniform_row_keeps_ceil_p_nb(orc):
+    # uniform row (SpargeAttention2 Fig. 2 situation): top-p keeps ceil(p * nb), top-k keeps k
+    nb = 16
+    L = np.zeros((1, nb))
+    s = orc.select_from_logits(L, 0, 0.6)
+    assert s.cnt[0] == 10 and _set(s.mask[0]) == set(range(10))
+    s = orc.select_from_logits(L, 12, 0.6)
+    assert s.cnt[0] == 12 and _set(s.mask[0]) == set(range(12))
+    for p in (0.05, 0.3, 0.55, 0.81, 0.99):
+        s = orc.select_from_logits(np.zeros((1, 40)), 2, p)
+        assert s.m_p[0] == math.ceil(p * 40 - 1e-9)
+
+
+def test_select_sink_row_top_k_rescues(orc):
+    # one sink block (SpargeAttention2 Fig. 3): top-p stops at the sink, top-k still keeps k
+    nb = 24
+    L = np.zeros((1, nb))
+    L[0, 9] = 20.0
+    s = orc.select_from_logits(L, 0, 0.9)
+    assert _set(s.mask[0]) == {9}
+    s = orc.select_from_logits(L, 4, 0.9)
+    # ties among the rest resolve to the lower block ids
+    assert _set(s.mask[0]) == {9, 0, 1, 2} and s.cnt[0] == 4
+
+
+def test_select_k_all_or_p_one_keeps_everything(orc):
+    rng = np.random.default_rng(3)
+    L = rng.standard_normal((5, 13)) * 3
+    for s in (orc.select_from_logits(L, 13, 0.1), orc.select_from_logits(L, 40, 0.0),
+              orc.select_from_logits(L, 0, 1.0)):
+        assert (s.mask == 1).all() and (s.cnt == 13).all()
+    s = orc.select_from_logits(L, 0, 0.0)
+    assert (s.mask == 0).all() and (s.cnt == 0).all()
+
+
+def _brute_min_count(P, p):
+    """Least |S| over all subsets S with sum_S P >= p (enumeration)."""
+    n = len(P)
+    for size in range(0, n + 1):
+        for S in itertools.combinations(range(n), size):
+            if P[list(S)].sum() >= p:
+                return size
+    return n
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_select_brute_force_small(orc, seed):
+    rng = np.random.default_rng(100 + seed)
+    nb = int(rng.integers(2, 11))
+    L = rng.standard_normal(nb) * rng.choice([0.3, 1.0, 3.0])
+    if seed % 3 == 0:
+        L[rng.integers(nb)] += 6.0  # sink-like row
+    P = orc.softmax_rows(L[None])[0]
+    k = int(rng.integers(0, nb + 1))
+    p = float(rng.choice([0.2, 0.5, 0.8, 0.9, 0.95]))
+    s = orc.select_from_probs(P[None], k, p)
+    kept = _set(s.mask[0])
+    # top-p part: minimum cardinality over ALL subsets, realised by the top-ranked blocks
+    m = _brute_min_count(P, p)
+    assert s.m_p[0] == m
+    order = sorted(range(nb), key=lambda j: (-P[j], j))
+    assert set(order[:m]) <= kept
+    # top-k part: the k largest probabilities
+    assert set(order[:min(k, nb)]) <= kept
+    # nothing else
+    assert kept == set(order[:min(k, nb)]) | set(order[:m])
+    # invariants: kept mass >= p; dropping the last top-p block goes below p
+    assert P[list(kept)].sum() >= p - 1e-15
+    if m > 0:
+        assert P[order[:m - 1]].sum() < p
+
+
+def test_select_random_rows_invariants(orc):
+    rng = np.random.default_rng(4)
+    rows, nb = 64, 97
+    L = rng.standard_normal((rows, nb)) * rng.uniform(0.1, 5.0, (rows, 1))
+    k, p = 7, 0.8
+    s = orc.select_from_logits(L, k, p)
+    P = orc.softmax_rows(L)
+    for r in range(rows):
+        order = np.lexsort((np.arange(nb), -P[r]))
+        kept = _set(s.mask[r])
+        assert set(order[:k].tolist()) <= kept
+        assert P[r, list(kept)].sum() >= p
+        m = s.m_p[r]
+        assert np.cumsum(P[r, order])[m - 1] >= p and (m == 1 or np.cumsum(P[r, order])[m - 2] < p)
+        assert s.cnt[r] == max(k, m) == len(kept)
+        assert s.tau_k[r] == P[r, order[k - 1]] and s.tau_p[r] == P[r, order[m - 1]]
+
+
+# ------------------------------------------------------------------------------------------------
+# attention: masked softmax attention and the dense control
+# ------------------------------------------------------------------------------------------------
+def _rand_qkv(rng, BH, N, d, sc=1.0):
+    return [bits(rng.standard_normal((BH, N, d)) * sc) for _ in range(3)]
+
+
+def test_dense_matches_torch_sdpa(orc):
+    import torch
+
+    rng = np.random.default_rng(5)
+    BH, N, d = 2, 150, 32
+    q, k, v = _rand_qkv(rng, BH, N, d, 1.5)
+    out = orc.dense_attention(q, k, v, 1 / math.sqrt(d)).reshape(BH, N, d)
+    Q, K, V = (torch.from_numpy(widen(x)) for x in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(Q, K, V).numpy()
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+
+
+def test_masked_all_ones_equals_dense(orc):
+    rng = np.random.default_rng(6)
+    BH, N, d, bs = 2, 200, 16, 64
+    q, k, v = _rand_qkv(rng, BH, N, d)
+    nb = (N + bs - 1) // bs
+    mask = np.ones((BH, nb, nb), np.uint8)
+    o = orc.masked_attention(q, k, v, mask, bs, 0.25)
+    dense = orc.dense_attention(q, k, v, 0.25).reshape(BH, N, d)
+    for bh in range(BH):
+        for i in range(nb):
+            rows = range(i * bs, min((i + 1) * bs, N))
+            np.testing.assert_allclose(o[bh * nb + i, :len(rows)], dense[bh, rows.start:rows.stop],
+                                       rtol=0, atol=1e-12)
+            assert (o[bh * nb + i, len(rows):] == 0).all()
+
+
+def test_masked_matches_torch_with_block_mask(orc):
+    import torch
+
+    rng = np.random.default_rng(7)
+    BH, N, d, bs = 1, 250, 16, 64
+    q, k, v = _rand_qkv(rng, BH, N, d)
+    nb = 4
+    mask = (rng.random((BH, nb, nb)) < 0.5).astype(np.uint8)
+    mask[:, :, 0] = 1
+    o = orc.masked_attention(q, k, v, mask, bs, 0.3)
+    tok = np.repeat(np.repeat(mask[0], bs, 0), bs, 1)[:N, :N].astype(bool)
+    Q, K, V = (torch.from_numpy(widen(x))[0] for x in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        Q[None], K[None], V[None], attn_mask=torch.from_numpy(tok)[None], scale=0.3)[0].numpy()
+    for i in range(nb):
+        r0, r1 = i * bs, min((i + 1) * bs, N)
+        np.testing.assert_allclose(o[i, :r1 - r0], ref[r0:r1], rtol=0, atol=1e-12)
+
+
+def test_masked_single_block_constant_v_and_tail_token(orc):
+    rng = np.random.default_rng(8)
+    N, d, bs = 129, 8, 128  # block 1 holds one token
+    q, k, _ = _rand_qkv(rng, 1, N, d, 2.0)
+    v = np.zeros((1, N, d), np.float32)
+    v[0, :128] = 3.25
+    v[0, 128] = np.arange(d) - 2.5
+    vb = bits(v)
+    mask = np.zeros((1, 2, 2), np.uint8)
+    mask[0, 0, 0] = 1  # block 0 sees only block 0 (constant V)
+    mask[0, 1, 1] = 1  # block 1 sees only the single tail token
+    o = orc.masked_attention(q, k, vb, mask, bs, 0.5)
+    assert np.allclose(o[0], 3.25, rtol=0, atol=1e-13)
+    assert np.array_equal(o[1, 0], np.arange(d) - 2.5) and (o[1, 1:] == 0).all()
+    # a block with nothing kept produces zeros
+    mask[0, 1, 1] = 0
+    o = orc.masked_attention(q, k, vb, mask, bs, 0.5)
+    assert (o[1] == 0).all()
+
+
+def test_masked_two_keys_closed_form(orc):
+    N, d, bs = 2, 2, 1  # each key its own block
+    q = bits([[[1.0, 2.0], [0.5, -1.0]]])
+    k = bits([[[1.0, 0.0], [0.0, 1.0]]])
+    v = bits([[[4.0, -2.0], [1.0, 8.0]]])
+    mask = np.ones((1, 2, 2), np.uint8)
+    o = orc.masked_attention(q, k, v, mask, bs, 1.0)
+    for t, (x1, x2) in enumerate([(1.0, 2.0), (0.5, -1.0)]):
+        w1 = 1.0 / (1.0 + math.exp(x2 - x1))
+        want = w1 * np.array([4.0, -2.0]) + (1 - w1) * np.array([1.0, 8.0])
+        np.testing.assert_allclose(o[t, 0], want, rtol=0, atol=1e-14)
+
+
+def test_masked_key_order_invariance(orc):
+    # permuting the tokens inside a kept key block leaves every output unchanged
+    rng = np.random.default_rng(9)
+    N, d, bs = 256, 16, 64
+    q, k, v = _rand_qkv(rng, 1, N, d)
+    mask = np.zeros((1, 4, 4), np.uint8)
+    mask[0, :, 1] = mask[0, :, 3] = 1
+    o1 = orc.masked_attention(q, k, v, mask, bs, 0.25)
+    perm = np.arange(N)
+    perm[64:128] = 64 + rng.permutation(64)
+    o2 = orc.masked_attention(q, k[:, perm], v[:, perm], mask, bs, 0.25)
+    np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-12)
