@@ -6,7 +6,8 @@ loads it and fails loudly if it has not been built.  ``workloads`` (seeded input
 the library.
 """
 _API = ("pool_blocks", "select_mask_topk_topp", "select_from_logits", "block_sparse_attn_fwd",
-        "dense_attn_fwd", "sparse_attention", "SAError", "lib")
+        "dense_attn_fwd", "sparse_attention", "num_blocks", "device_error", "set_wait_limit_ns",
+        "probe_bounded_wait", "SAError", "lib")
 
 
 def __getattr__(name):

@@ -1,0 +1,357 @@
+// Block-sparse attention forward over a compacted per-query-block key-block list, and the dense
+// control (every key block).
+//
+// For each query block i and each kept key block j, S = Q_i K_j^T is a dense 128 x BS x d
+// contraction and O_i += P V_j a dense 128 x d x BS one, so both run on the tcgen05 tensor cores
+// with fp32 accumulators in tensor memory; softmax is online (running max and sum, O rescaled
+// when the max grows by more than 2^8), as in FlashAttention.  The key-block walk is what Sparse
+// VideoGen2 (section 2.C) describes: dense compute on a contiguous query tile, sparse loads of
+// the kept key/value blocks.  Keys at or beyond N are masked; query rows at or beyond N (and,
+// for BS = 64, rows of the next query block inside the 128-row tile) are computed but not
+// stored.  A query block with an empty list writes zeros.
+//
+// CTA roles (256 threads, two CTAs per SM, persistent over query blocks):
+//   warp 0 lane 0  TMA producer: Q tile once per query block, then K_j and V_j per kept block
+//   warp 1 lane 0  MMA issuer:   S = Q K_j^T (SS form), O += P V_j (P read from tensor memory)
+//   warp 2         tensor-memory allocator (256 columns: S/P at 0, O at 128)
+//   warps 4..7     softmax: one thread per query row; reads S, writes P (bf16) over S, rescales
+//                  O, and runs the epilogue O / l -> bf16 -> global
+// Per CTA the chain S -> softmax -> PV is serial; the second CTA on the SM fills the tensor
+// pipe while this one is in softmax.
+#include "bsa_internal.h"
+
+namespace bsa {
+
+struct AttnParams {
+    const int32_t *kv_idx;  // [units, nbk] ascending key-block ids, or null for dense
+    const int32_t *kv_cnt;  // [units], or null for dense
+    __nv_bfloat16 *o;       // [BH, N, D]
+    int N, nbq, nbk;
+    long long units;        // BH * nbq
+    float scale_log2;       // softmax scale * log2(e)
+    unsigned long long wait_ns;
+};
+
+template <int D, int BS>
+struct AttnCfg {
+    static constexpr int QROWS = 128;
+    static constexpr int CHUNKS = D / 64;           // 64-column (128-byte) swizzle chunks
+    static constexpr int Q_CHUNK = QROWS * 128;     // bytes per Q chunk
+    static constexpr int KV_CHUNK = BS * 128;       // bytes per K or V chunk
+    static constexpr int Q_BYTES = CHUNKS * Q_CHUNK;
+    static constexpr int KV_BYTES = CHUNKS * KV_CHUNK;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + Q_BYTES;
+    static constexpr int OFF_V = OFF_K + KV_BYTES;
+    static constexpr int OFF_BAR = OFF_V + KV_BYTES;
+    static constexpr int SMEM = OFF_BAR + 128 + 1024;  // barriers + slack for 1024-byte alignment
+    static constexpr uint32_t TMEM_COLS = 256;
+    static constexpr uint32_t COL_S = 0, COL_O = 128;
+};
+
+enum { B_QF, B_QE, B_KF, B_KE, B_VF, B_VE, B_SF, B_PF, B_OD, B_ED, B_FIN, B_COUNT };
+
+__device__ __forceinline__ int clamp_block(int j, int nbk) {
+    if (j < 0 || j >= nbk) {
+        atomicOr(&g_bsa_device_error, BSA_DEVERR_BOUNDS);
+        j = j < 0 ? 0 : nbk - 1;
+    }
+    return j;
+}
+
+// Waits used while unwinding after an abort: they ignore the abort flag but stay bounded.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, unsigned long long ns) {
+    int never = 0;
+    mbar_wait(bar, parity, ns, (volatile int *)&never);
+}
+
+template <int D, int BS>
+__global__ void __launch_bounds__(256, 2)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const AttnParams prm) {
+    using C = AttnCfg<D, BS>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_BAR + 8 * B_COUNT);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_BAR + 8 * B_COUNT + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t sQ = smem_u32(smem + C::OFF_Q);
+    const uint32_t sK = smem_u32(smem + C::OFF_K);
+    const uint32_t sV = smem_u32(smem + C::OFF_V);
+    auto bar = [&](int b) { return smem_u32(&bars[b]); };
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(B_QF), 1);
+        mbar_init(bar(B_QE), 1);
+        mbar_init(bar(B_KF), 1);
+        mbar_init(bar(B_KE), 1);
+        mbar_init(bar(B_VF), 1);
+        mbar_init(bar(B_VE), 1);
+        mbar_init(bar(B_SF), 1);
+        mbar_init(bar(B_PF), 128);
+        mbar_init(bar(B_OD), 1);
+        mbar_init(bar(B_ED), 128);
+        mbar_init(bar(B_FIN), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+    }
+    if (warp == 2) {
+        tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_holder;
+    const uint32_t tS = tbase + C::COL_S;
+    const uint32_t tO = tbase + C::COL_O;
+    const unsigned long long wns = prm.wait_ns;
+    const bool dense = prm.kv_idx == nullptr;
+
+    if (warp == 0 && lane == 0) {
+        // ---------------------------------------------------------------- TMA producer
+        uint32_t nq = 0, nk = 0, nv = 0;
+        bool ok = true;
+        for (long long u = blockIdx.x; u < prm.units && ok; u += gridDim.x) {
+            const int cnt = dense ? prm.nbk : min(max(prm.kv_cnt[u], 0), prm.nbk);
+            if (cnt == 0) continue;
+            const int bh = (int)(u / prm.nbq);
+            const int i = (int)(u - (long long)bh * prm.nbq);
+            const int32_t *list = dense ? nullptr : prm.kv_idx + (size_t)u * prm.nbk;
+            if (nq > 0 && !(ok = mbar_wait(bar(B_QE), (nq - 1) & 1, wns, abort_flag))) break;
+            mbar_arrive_expect_tx(bar(B_QF), C::Q_BYTES);
+#pragma unroll
+            for (int c = 0; c < C::CHUNKS; ++c)
+                tma_load_3d(sQ + c * C::Q_CHUNK, &tmQ, bar(B_QF), c * 64, i * BS, bh);
+            ++nq;
+            for (int t = 0; t < cnt; ++t) {
+                const int j = dense ? t : clamp_block(list[t], prm.nbk);
+                if (nk > 0 && !(ok = mbar_wait(bar(B_KE), (nk - 1) & 1, wns, abort_flag))) break;
+                mbar_arrive_expect_tx(bar(B_KF), C::KV_BYTES);
+#pragma unroll
+                for (int c = 0; c < C::CHUNKS; ++c)
+                    tma_load_3d(sK + c * C::KV_CHUNK, &tmK, bar(B_KF), c * 64, j * BS, bh);
+                ++nk;
+                if (nv > 0 && !(ok = mbar_wait(bar(B_VE), (nv - 1) & 1, wns, abort_flag))) break;
+                mbar_arrive_expect_tx(bar(B_VF), C::KV_BYTES);
+#pragma unroll
+                for (int c = 0; c < C::CHUNKS; ++c)
+                    tma_load_3d(sV + c * C::KV_CHUNK, &tmV, bar(B_VF), c * 64, j * BS, bh);
+                ++nv;
+            }
+        }
+        if (!ok) {  // let every copy that was started land before the CTA leaves
+            if (nq) drain_wait(bar(B_QF), (nq - 1) & 1, wns);
+            if (nk) drain_wait(bar(B_KF), (nk - 1) & 1, wns);
+            if (nv) drain_wait(bar(B_VF), (nv - 1) & 1, wns);
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ---------------------------------------------------------------- MMA issuer
+        constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BS, 0, 0);
+        constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, 0, 1);
+        uint32_t nq = 0, nk = 0, nv = 0, np = 0, npv = 0, ned = 0, units_done = 0;
+        bool ok = true;
+        for (long long u = blockIdx.x; u < prm.units && ok; u += gridDim.x) {
+            const int cnt = dense ? prm.nbk : min(max(prm.kv_cnt[u], 0), prm.nbk);
+            if (cnt == 0) continue;
+            if (!(ok = mbar_wait(bar(B_QF), nq & 1, wns, abort_flag))) break;
+            ++nq;
+            for (int t = 0; t < cnt; ++t) {
+                if (!(ok = mbar_wait(bar(B_KF), nk & 1, wns, abort_flag))) break;
+                ++nk;
+                // S/P columns are reused: the previous P V must have finished reading P
+                if (npv > 0 && !(ok = mbar_wait(bar(B_OD), (npv - 1) & 1, wns, abort_flag))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk & 3) * 32;  // K step inside the 128-byte swizzled row
+                    const uint64_t a = smem_desc_sw128(sQ + (kk >> 2) * C::Q_CHUNK + off, 16, 1024);
+                    const uint64_t b = smem_desc_sw128(sK + (kk >> 2) * C::KV_CHUNK + off, 16, 1024);
+                    mma_ss(tS, a, b, IDESC_S, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(bar(B_SF));
+                mma_commit(bar(B_KE));
+                if (t == cnt - 1) mma_commit(bar(B_QE));
+                if (!(ok = mbar_wait(bar(B_PF), np & 1, wns, abort_flag))) break;
+                ++np;
+                if (t == 0 && units_done > 0) {
+                    // O is about to be overwritten: the previous epilogue must have read it
+                    if (!(ok = mbar_wait(bar(B_ED), ned & 1, wns, abort_flag))) break;
+                    ++ned;
+                }
+                if (!(ok = mbar_wait(bar(B_VF), nv & 1, wns, abort_flag))) break;
+                ++nv;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < BS / 16; ++kk) {
+                    const uint64_t b = smem_desc_sw128(sV + kk * 2048, C::KV_CHUNK, 1024);
+                    mma_ts(tO, tS + kk * 8, b, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(bar(B_VE));
+                mma_commit(bar(B_OD));
+                ++npv;
+            }
+            ++units_done;
+        }
+        // every MMA this thread issued must be complete before tensor memory is released
+        mma_commit(bar(B_FIN));
+        drain_wait(bar(B_FIN), 0, wns);
+    } else if (warp >= 4) {
+        // ---------------------------------------------------------------- softmax + epilogue
+        const int q4 = warp & 3;
+        const int r = q4 * 32 + lane;  // query row inside the tile == TMEM lane
+        const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+        const uint32_t tSr = tS + lane_off, tOr = tO + lane_off;
+        const float sl2 = prm.scale_log2;
+        uint32_t ns = 0, npv = 0;
+        bool ok = true;
+        for (long long u = blockIdx.x; u < prm.units && ok; u += gridDim.x) {
+            const int cnt = dense ? prm.nbk : min(max(prm.kv_cnt[u], 0), prm.nbk);
+            const int bh = (int)(u / prm.nbq);
+            const int i = (int)(u - (long long)bh * prm.nbq);
+            const int grow = i * BS + r;
+            const bool row_ok = r < BS && grow < prm.N;
+            __nv_bfloat16 *orow = prm.o + ((size_t)bh * prm.N + (row_ok ? grow : 0)) * D;
+            if (cnt == 0) {
+                if (row_ok) {
+                    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                    for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4 *>(orow)[c] = z;
+                }
+                continue;
+            }
+            const int32_t *list = dense ? nullptr : prm.kv_idx + (size_t)u * prm.nbk;
+            float m_ref = -INFINITY;  // running max, log2 domain
+            float l = 0.f;            // running sum
+            for (int t = 0; t < cnt; ++t) {
+                const int j = dense ? t : min(max(list[t], 0), prm.nbk - 1);
+                const int valid = min(BS, prm.N - j * BS);
+                if (!(ok = mbar_wait(bar(B_SF), ns & 1, wns, abort_flag))) break;
+                ++ns;
+                tc_fence_after();
+                uint32_t v[32];
+                float mx = -INFINITY;
+#pragma unroll 1
+                for (int c = 0; c < BS / 32; ++c) {
+                    tmem_ld32(tSr + c * 32, v);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (c * 32 + e < valid) mx = fmaxf(mx, __uint_as_float(v[e]));
+                }
+                const float mxs = mx * sl2;
+                if (mxs > m_ref + 8.f) {
+                    const float alpha = ex2(m_ref - mxs);  // 0 on the first block
+                    if (t > 0) {
+                        // the previous P V is complete: this S was issued after it finished
+#pragma unroll
+                        for (int c = 0; c < D / 32; ++c) {
+                            tmem_ld32(tOr + c * 32, v);
+#pragma unroll
+                            for (int e = 0; e < 32; ++e)
+                                v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+                            tmem_st32(tOr + c * 32, v);
+                        }
+                    }
+                    l *= alpha;
+                    m_ref = mxs;
+                }
+#pragma unroll 1
+                for (int c = 0; c < BS / 32; ++c) {
+                    tmem_ld32(tSr + c * 32, v);
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        const float p0 = (c * 32 + e < valid)
+                                             ? ex2(fmaf(__uint_as_float(v[e]), sl2, -m_ref)) : 0.f;
+                        const float p1 = (c * 32 + e + 1 < valid)
+                                             ? ex2(fmaf(__uint_as_float(v[e + 1]), sl2, -m_ref)) : 0.f;
+                        l += p0 + p1;
+                        pk[e >> 1] = pack_bf16(p0, p1);
+                    }
+                    tmem_st16(tSr + c * 16, pk);  // P (bf16 pairs) over the consumed S columns
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(B_PF));
+            }
+            if (!ok) break;
+            // epilogue: wait for the last P V of this query block
+            npv += cnt;
+            if (!(ok = mbar_wait(bar(B_OD), (npv - 1) & 1, wns, abort_flag))) break;
+            tc_fence_after();
+            const float inv_l = 1.f / l;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld32(tOr + c * 32, v);
+                if (row_ok) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2)
+                        pk[e >> 1] = pack_bf16(__uint_as_float(v[e]) * inv_l,
+                                               __uint_as_float(v[e + 1]) * inv_l);
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+#pragma unroll
+                    for (int w = 0; w < 4; ++w)
+                        dst[w] = make_uint4(pk[4 * w], pk[4 * w + 1], pk[4 * w + 2], pk[4 * w + 3]);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(bar(B_ED));
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 2) tmem_dealloc(tbase, C::TMEM_COLS);
+}
+
+// ------------------------------------------------------------------------------------------
+// host side
+// ------------------------------------------------------------------------------------------
+template <int D, int BS>
+static cudaError_t launch_attn_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                 const AttnParams &p, int num_sms, cudaStream_t st) {
+    using C = AttnCfg<D, BS>;
+    // at least 80 KB per CTA so that no more than two CTAs (2 x 256 TMEM columns) share an SM
+    const int smem = C::SMEM > 80 * 1024 ? C::SMEM : 80 * 1024;
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, BS>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    long long grid = 2LL * num_sms;
+    if (grid > p.units) grid = p.units;
+    if (grid <= 0) return cudaSuccess;
+    attn_fwd_kernel<D, BS><<<(unsigned)grid, 256, smem, st>>>(tq, tk, tv, p);
+    return cudaGetLastError();
+}
+
+cudaError_t attn_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                     const int32_t *kv_idx, const int32_t *kv_cnt, void *o, long long BH, int N,
+                     int d, int bs, float scale, unsigned long long wait_ns, int num_sms,
+                     cudaStream_t st) {
+    AttnParams p;
+    p.kv_idx = kv_idx;
+    p.kv_cnt = kv_cnt;
+    p.o = reinterpret_cast<__nv_bfloat16 *>(o);
+    p.N = N;
+    p.nbq = (N + bs - 1) / bs;
+    p.nbk = p.nbq;
+    p.units = BH * p.nbq;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.wait_ns = wait_ns;
+    if (d == 128 && bs == 128) return launch_attn_t<128, 128>(tq, tk, tv, p, num_sms, st);
+    if (d == 128 && bs == 64) return launch_attn_t<128, 64>(tq, tk, tv, p, num_sms, st);
+    if (d == 64 && bs == 128) return launch_attn_t<64, 128>(tq, tk, tv, p, num_sms, st);
+    if (d == 64 && bs == 64) return launch_attn_t<64, 64>(tq, tk, tv, p, num_sms, st);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace bsa

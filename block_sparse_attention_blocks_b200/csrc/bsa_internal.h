@@ -1,0 +1,28 @@
+// Declarations shared by the CUDA translation units of libbsa (not part of the public C ABI).
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ptx.cuh"
+
+namespace bsa {
+
+cudaError_t pool_blocks(const void *q, const void *k, float *qp, float *kp, long long BH, int N,
+                        int d, int bs, cudaStream_t st);
+
+cudaError_t block_scores(const float *qp, const float *kp, float *logits, long long BH, int nb,
+                         int d, float scale, cudaStream_t st);
+
+cudaError_t select_rows(const float *logits, long long rows, int nb, int topk, float topp,
+                        uint8_t *mask, int32_t *kv_idx, int32_t *kv_cnt, cudaStream_t st);
+
+cudaError_t attn_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                     const int32_t *kv_idx, const int32_t *kv_cnt, void *o, long long BH, int N,
+                     int d, int bs, float scale, unsigned long long wait_ns, int num_sms,
+                     cudaStream_t st);
+
+cudaError_t bounded_wait_probe(unsigned long long wait_ns, cudaStream_t st);
+
+}  // namespace bsa

@@ -1,0 +1,7 @@
+// Single translation unit of libbsa.so: the kernels share the device error word defined in
+// ptx.cuh, so they are compiled together.
+#include "pool.cu"
+#include "select.cu"
+#include "attn.cu"
+#include "probe.cu"
+#include "capi.cu"

@@ -1,0 +1,198 @@
+"""Python binding of libbsa (include/sparse_attn.h): argument marshalling only.
+
+Every step of the path runs in the library's sm_100a kernels; this module checks tensor
+properties, allocates outputs through PyTorch (which owns device memory and streams here) and
+passes raw pointers and the current CUDA stream through ctypes.  There is no fallback: if the
+library is missing, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libbsa.so")
+
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        "libbsa.so is not built; run `python -m block_sparse_attention_blocks_b200.build` "
+        "(nvcc for sm_100a) first")
+
+lib = ctypes.CDLL(_LIB_PATH)
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+
+lib.sa_pool_blocks.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]
+lib.sa_select_mask_topk_topp.argtypes = [_P, _P, _I, _I, _I, _I, _I, _F, _F, _P, _P, _P, _P]
+lib.sa_select_from_logits.argtypes = [_P, _I, _I, _I, _I, _F, _P, _P, _P, _P]
+lib.sa_block_sparse_attn_fwd.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]
+lib.sa_dense_attn_fwd.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P]
+lib.sa_get_error_string.argtypes = [_I]
+lib.sa_get_error_string.restype = ctypes.c_char_p
+lib.sa_get_device_error.argtypes = [_P]
+lib.sa_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+lib.sa_probe_bounded_wait.argtypes = [_P]
+lib.sa_num_blocks.argtypes = [_I, _I]
+for _f in (lib.sa_pool_blocks, lib.sa_select_mask_topk_topp, lib.sa_select_from_logits,
+           lib.sa_block_sparse_attn_fwd, lib.sa_dense_attn_fwd, lib.sa_get_device_error,
+           lib.sa_set_wait_limit_ns, lib.sa_probe_bounded_wait, lib.sa_num_blocks):
+    _f.restype = _I
+lib.sa_get_error_string.restype = ctypes.c_char_p
+
+SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_CUDA, SA_ERR_TIMEOUT = range(5)
+
+
+class SAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {lib.sa_get_error_string(status).decode()}")
+
+
+def _check(status: int, where: str):
+    if status != SA_OK:
+        raise SAError(status, where)
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _ptr(t: torch.Tensor) -> ctypes.c_void_p:
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t: torch.Tensor, name: str, dtype, ndim: int):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dim() != ndim or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {ndim}-d tensor, got shape {tuple(t.shape)}")
+
+
+def num_blocks(N: int, bs: int) -> int:
+    return (N + bs - 1) // bs
+
+
+def pool_blocks(q: torch.Tensor, k: torch.Tensor, bs: int, qp=None, kp=None):
+    """Mean of Q and K over each block of bs tokens -> (qp, kp) [B, H, nb, d] fp32."""
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k, "k", torch.bfloat16, 4)
+    if q.shape != k.shape:
+        raise ValueError("q and k must have the same shape")
+    B, H, N, d = q.shape
+    nb = num_blocks(N, bs)
+    qp = qp if qp is not None else torch.empty(B, H, nb, d, device=q.device, dtype=torch.float32)
+    kp = kp if kp is not None else torch.empty(B, H, nb, d, device=q.device, dtype=torch.float32)
+    _need(qp, "qp", torch.float32, 4)
+    _need(kp, "kp", torch.float32, 4)
+    _check(lib.sa_pool_blocks(_ptr(q), _ptr(k), _ptr(qp), _ptr(kp), B, H, N, d, bs,
+                              _stream(q.device)), "sa_pool_blocks")
+    return qp, kp
+
+
+def _sel_outputs(B, H, nb, device, mask, kv_idx, kv_cnt):
+    mask = mask if mask is not None else torch.empty(B, H, nb, nb, device=device, dtype=torch.uint8)
+    kv_idx = kv_idx if kv_idx is not None else torch.empty(B, H, nb, nb, device=device,
+                                                           dtype=torch.int32)
+    kv_cnt = kv_cnt if kv_cnt is not None else torch.empty(B, H, nb, device=device,
+                                                           dtype=torch.int32)
+    _need(mask, "mask", torch.uint8, 4)
+    _need(kv_idx, "kv_idx", torch.int32, 4)
+    _need(kv_cnt, "kv_cnt", torch.int32, 3)
+    return mask, kv_idx, kv_cnt
+
+
+def select_mask_topk_topp(qp, kp, topk: int, topp: float, scale: float | None = None, mask=None,
+                          kv_idx=None, kv_cnt=None):
+    """Hybrid top-k union top-p block selection -> (mask, kv_idx, kv_cnt)."""
+    _need(qp, "qp", torch.float32, 4)
+    _need(kp, "kp", torch.float32, 4)
+    B, H, nb, d = qp.shape
+    mask, kv_idx, kv_cnt = _sel_outputs(B, H, nb, qp.device, mask, kv_idx, kv_cnt)
+    _check(lib.sa_select_mask_topk_topp(_ptr(qp), _ptr(kp), B, H, nb, d, int(topk), float(topp),
+                                        float(scale or 0.0), _ptr(mask), _ptr(kv_idx),
+                                        _ptr(kv_cnt), _stream(qp.device)),
+           "sa_select_mask_topk_topp")
+    return mask, kv_idx, kv_cnt
+
+
+def select_from_logits(logits, topk: int, topp: float, mask=None, kv_idx=None, kv_cnt=None):
+    """Selection from given block scores [B, H, nb, nb] fp32 -> (mask, kv_idx, kv_cnt)."""
+    _need(logits, "logits", torch.float32, 4)
+    B, H, nb, _ = logits.shape
+    mask, kv_idx, kv_cnt = _sel_outputs(B, H, nb, logits.device, mask, kv_idx, kv_cnt)
+    _check(lib.sa_select_from_logits(_ptr(logits), B, H, nb, int(topk), float(topp), _ptr(mask),
+                                     _ptr(kv_idx), _ptr(kv_cnt), _stream(logits.device)),
+           "sa_select_from_logits")
+    return mask, kv_idx, kv_cnt
+
+
+def block_sparse_attn_fwd(q, k, v, kv_idx, kv_cnt, bs: int, scale: float | None = None, o=None):
+    """Attention over the kept key blocks listed in (kv_idx, kv_cnt) -> O [B, H, N, d] bf16."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, torch.bfloat16, 4)
+    _need(kv_idx, "kv_idx", torch.int32, 4)
+    _need(kv_cnt, "kv_cnt", torch.int32, 3)
+    B, H, N, d = q.shape
+    o = o if o is not None else torch.empty_like(q)
+    _need(o, "o", torch.bfloat16, 4)
+    _check(lib.sa_block_sparse_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_idx), _ptr(kv_cnt),
+                                        _ptr(o), B, H, N, d, bs, float(scale or 0.0),
+                                        _stream(q.device)), "sa_block_sparse_attn_fwd")
+    return o
+
+
+def dense_attn_fwd(q, k, v, scale: float | None = None, o=None):
+    """Dense softmax attention (the 0 %-sparsity control) -> O [B, H, N, d] bf16."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, torch.bfloat16, 4)
+    B, H, N, d = q.shape
+    o = o if o is not None else torch.empty_like(q)
+    _need(o, "o", torch.bfloat16, 4)
+    _check(lib.sa_dense_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d,
+                                 float(scale or 0.0), _stream(q.device)), "sa_dense_attn_fwd")
+    return o
+
+
+def sparse_attention(q, k, v, bs: int, topk: int, topp: float, scale: float | None = None,
+                     device=None, return_selection: bool = False):
+    """The whole path: pool -> select -> block-sparse attention.
+
+    q, k, v may live on the host (ideally pinned) or on a CUDA device.  Host inputs are copied
+    to `device` (default: the current CUDA device) on the current stream and O is copied back
+    to the host; device inputs return a device O.
+    """
+    on_host = not q.is_cuda
+    if on_host:
+        dev = torch.device(device) if device is not None else torch.device("cuda",
+                                                                           torch.cuda.current_device())
+        q, k, v = (t.to(dev, non_blocking=True) for t in (q, k, v))
+    qp, kp = pool_blocks(q, k, bs)
+    mask, kv_idx, kv_cnt = select_mask_topk_topp(qp, kp, topk, topp, scale)
+    o = block_sparse_attn_fwd(q, k, v, kv_idx, kv_cnt, bs, scale)
+    if on_host:
+        o = o.to("cpu")
+    if return_selection:
+        return o, (mask, kv_idx, kv_cnt)
+    return o
+
+
+def device_error(stream=None) -> int:
+    """Synchronise and read/clear the library's device error word (an sa_status code)."""
+    s = ctypes.c_void_p(stream) if stream is not None else _stream(None)
+    return int(lib.sa_get_device_error(s))
+
+
+def set_wait_limit_ns(ns: int):
+    _check(lib.sa_set_wait_limit_ns(int(ns)), "sa_set_wait_limit_ns")
+
+
+def probe_bounded_wait():
+    _check(lib.sa_probe_bounded_wait(_stream(None)), "sa_probe_bounded_wait")

@@ -1,0 +1,152 @@
+/*
+ * sparse_attn.h: C ABI of libbsa, block-sparse self-attention for video diffusion transformers
+ * with hybrid top-k + top-p block masks, for NVIDIA B200 (sm_100a).
+ *
+ * The path, one attention call (all steps asynchronous on one CUDA stream):
+ *
+ *   Q, K, V [B, H, N, d] bf16
+ *     sa_pool_blocks            -> Qp, Kp [B, H, nb, d] fp32    mean of each block of bs tokens
+ *     sa_select_mask_topk_topp  -> mask [B, H, nb, nb] uint8, kv_idx, kv_cnt
+ *                                  softmax(Qp Kp^T * scale) per query-block row; keep the union of
+ *                                  the top-k blocks and the shortest top-p prefix
+ *     sa_block_sparse_attn_fwd  -> O [B, H, N, d] bf16          softmax attention over the kept
+ *                                                               key blocks only
+ *   sa_dense_attn_fwd is the 0 %-sparsity control (every key block).
+ *
+ * Sources (page title, section):
+ *   SpargeAttention2 ("SpargeAttention2とは？Top-k+Top-pハイブリッドマスキングでビデオ生成を16.2倍高速化"):
+ *     section "Top-kとTop-pの限界を解剖する" defines top-k (keep the k largest probabilities) and
+ *     top-p (take from the top until the cumulative probability passes p); section
+ *     "ハイブリッドマスキングと蒸留微調整" makes the mask the union of the two.
+ *   Sparse VideoGen2 ("Sparse VideoGen2: Accelerate Video Generation with Sparse Attention via
+ *     Semantic-Aware Permutation"): section 1 (block representatives by mean pooling), section
+ *     2.B (scores between representatives, sorted, taken until the cumulative score reaches p),
+ *     section 2.C (sparse loads of the kept key/value blocks, dense compute on query tiles).
+ *   The block size, mean pooling, the score scale 1/sqrt(d) and the tensor layouts are fixed by
+ *   the problem statement this library implements; the pages leave them open.
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are DEVICE pointers owned by the caller.  The library allocates and frees
+ *     nothing; it never synchronises the stream except in sa_get_device_error.
+ *   - Tensors are dense and row-major with the last dimension contiguous.  bf16 tensors are
+ *     passed as void*; their base addresses must be 16-byte aligned, fp32 tensors too.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  The call
+ *     runs on the device that owns the output pointer.
+ *   - Supported shapes: d in {64, 128}, bs in {64, 128}, N >= 1 (any N; a tail block shorter
+ *     than bs is handled inside), B*H in [1, 65535], nb = ceil(N / bs) <= 1024.
+ *   - Argument errors are detected on the host and returned before anything is launched.
+ *     A failed launch returns SA_ERR_CUDA.  Device-side conditions (a bounded wait that ran
+ *     out, an out-of-range block id in kv_idx) are recorded in a device error word that
+ *     sa_get_device_error reads and clears.
+ */
+#ifndef SPARSE_ATTN_H
+#define SPARSE_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SA_OK = 0,
+    SA_ERR_INVALID_ARG = 1, /* null or misaligned pointer, bad size or parameter */
+    SA_ERR_UNSUPPORTED = 2, /* d, bs or nb outside the supported set */
+    SA_ERR_CUDA = 3,        /* a CUDA runtime or driver call failed */
+    SA_ERR_TIMEOUT = 4      /* a device-side bounded wait ran out (reported by sa_get_device_error) */
+} sa_status;
+
+/*
+ * Block representatives (Sparse VideoGen2, section 1: mean pooling of contiguous blocks).
+ *   qp[b,h,i,:] = mean over t in [i*bs, min((i+1)*bs, N)) of q[b,h,t,:], likewise kp from k.
+ * q, k   : [B, H, N, d] bf16, read only.
+ * qp, kp : [B, H, nb, d] fp32, written; nb = ceil(N / bs).  Accumulation is fp32.
+ */
+sa_status sa_pool_blocks(const void *q, const void *k, float *qp, float *kp, int B, int H, int N,
+                         int d, int bs, void *stream);
+
+/*
+ * Hybrid block selection (SpargeAttention2, "Top-kとTop-pの限界を解剖する" and
+ * "ハイブリッドマスキングと蒸留微調整"; Sparse VideoGen2 section 2.B).
+ *   P[i,:]  = softmax_j(qp_i . kp_j * scale) over the nb key blocks of row i (fp32)
+ *   order   = key blocks by P descending, the lower block id first on equal P
+ *   S_k     = first min(topk, nb) blocks of the order
+ *   S_p     = first m blocks, m the least count whose cumulative P is >= topp
+ *             (topp <= 0: m = 0; topp >= 1: m = nb)
+ *   keep(i) = S_k union S_p      (both are prefixes of one order, so |keep| = max(min(k,nb), m))
+ * qp, kp  : [B, H, nb, d] fp32 (as written by sa_pool_blocks).
+ * topk    : >= 0 (values above nb act as nb).  topp : in [0, 1].
+ * scale   : score scale; <= 0 selects 1/sqrt(d).
+ * mask    : [B, H, nb, nb] uint8, written with 0/1.
+ * kv_idx  : [B, H, nb, nb] int32.  Row (b,h,i) receives the kept key-block ids in ascending
+ *           order in its first kv_cnt[b,h,i] entries; the remaining entries are scratch and
+ *           undefined on return (the buffer also stages the fp32 block scores).
+ * kv_cnt  : [B, H, nb] int32, written.
+ */
+sa_status sa_select_mask_topk_topp(const float *qp, const float *kp, int B, int H, int nb, int d,
+                                   int topk, float topp, float scale, uint8_t *mask,
+                                   int32_t *kv_idx, int32_t *kv_cnt, void *stream);
+
+/*
+ * Selection from caller-provided block scores (the second half of sa_select_mask_topk_topp,
+ * exposed for tests that feed hand-made rows).  logits: [B, H, nb, nb] fp32 scores already
+ * scaled; the row softmax, ranking, top-k union top-p and outputs are as above.  logits may be
+ * the same buffer as kv_idx.
+ */
+sa_status sa_select_from_logits(const float *logits, int B, int H, int nb, int topk, float topp,
+                                uint8_t *mask, int32_t *kv_idx, int32_t *kv_cnt, void *stream);
+
+/*
+ * Block-sparse attention forward (online softmax over the kept key blocks only).
+ *   O[b,h,t,:] = sum over kept blocks j of query block i = t / bs, keys s in block j with s < N,
+ *                of softmax_s(scale * Q[t] . K[s]) V[s]; zero when the block keeps nothing.
+ * q, k, v : [B, H, N, d] bf16.       o : [B, H, N, d] bf16, written.
+ * kv_idx  : [B, H, nb, nb] int32, ascending ids < nb in the first kv_cnt entries of each row
+ *           (as written by sa_select_mask_topk_topp).  kv_cnt : [B, H, nb] int32 in [0, nb].
+ *           Ids outside [0, nb) are clamped and flagged in the device error word.
+ * bs      : block size of both query and key blocks.  scale : <= 0 selects 1/sqrt(d).
+ * Arithmetic: bf16 operands, fp32 accumulation on the tensor cores, P rounded to bf16.
+ */
+sa_status sa_block_sparse_attn_fwd(const void *q, const void *k, const void *v,
+                                   const int32_t *kv_idx, const int32_t *kv_cnt, void *o, int B,
+                                   int H, int N, int d, int bs, float scale, void *stream);
+
+/*
+ * Dense attention forward, the 0 %-sparsity control: O = softmax(scale Q K^T) V over all N keys.
+ * Same layouts and arithmetic as sa_block_sparse_attn_fwd (internally bs = 128).
+ */
+sa_status sa_dense_attn_fwd(const void *q, const void *k, const void *v, void *o, int B, int H,
+                            int N, int d, float scale, void *stream);
+
+/* Human-readable name of a status code (static storage). */
+const char *sa_get_error_string(sa_status status);
+
+/*
+ * Synchronise `stream`, then read and clear the device error word of the current device.
+ * Returns SA_ERR_TIMEOUT if a bounded wait ran out since the last call, SA_ERR_INVALID_ARG if
+ * a kernel met an out-of-range key-block id, SA_ERR_CUDA if the synchronisation failed.
+ */
+sa_status sa_get_device_error(void *stream);
+
+/*
+ * Upper bound, in nanoseconds of device time, on every device-side wait of later launches
+ * (default 2e9).  After it a kernel records SA_ERR_TIMEOUT, unwinds and exits.  0 restores the
+ * default.
+ */
+sa_status sa_set_wait_limit_ns(uint64_t ns);
+
+/*
+ * Failure-detection check: launches one CTA that waits on a barrier nothing ever arrives at,
+ * bounded by the current wait limit.  A subsequent sa_get_device_error returns SA_ERR_TIMEOUT.
+ */
+sa_status sa_probe_bounded_wait(void *stream);
+
+/* Number of key-block ids per row of kv_idx for a given N and bs, i.e. nb = ceil(N / bs). */
+int sa_num_blocks(int N, int bs);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSE_ATTN_H */

@@ -1,0 +1,126 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every entry point
+declared in include/*.h, and rejects bad arguments before launching anything."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from block_sparse_attention_blocks_b200 import build
+
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names |= set(re.findall(r"\b(sa_[a-z0-9_]+)\s*\(", src))
+    return sorted(names)
+
+
+def test_header_declares_the_path():
+    names = _declared()
+    for required in ("sa_pool_blocks", "sa_select_mask_topk_topp", "sa_block_sparse_attn_fwd",
+                     "sa_dense_attn_fwd", "sa_get_error_string", "sa_get_device_error",
+                     "sa_select_from_logits"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in _declared():
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+
+
+def test_error_strings(lib):
+    lib.sa_get_error_string.restype = ctypes.c_char_p
+    lib.sa_get_error_string.argtypes = [ctypes.c_int]
+    assert lib.sa_get_error_string(0) == b"SA_OK"
+    assert b"TIMEOUT" in lib.sa_get_error_string(4)
+    assert b"unknown" in lib.sa_get_error_string(99)
+
+
+def test_num_blocks(lib):
+    lib.sa_num_blocks.argtypes = [ctypes.c_int, ctypes.c_int]
+    assert lib.sa_num_blocks(32760, 128) == 256
+    assert lib.sa_num_blocks(75600, 128) == 591
+    assert lib.sa_num_blocks(118800, 128) == 929
+    assert lib.sa_num_blocks(1024, 64) == 16
+    assert lib.sa_num_blocks(0, 128) == 0
+
+
+# Fake, 16-byte aligned, non-null addresses: every call below must be rejected by the host-side
+# checks before the library touches CUDA.
+A = ctypes.c_void_p(0x10000)
+A2 = ctypes.c_void_p(0x20000)
+MIS = ctypes.c_void_p(0x10008)
+NUL = ctypes.c_void_p(0)
+S = ctypes.c_void_p(0)
+
+
+def test_pool_argument_checks(lib):
+    f = lib.sa_pool_blocks
+    f.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 5 + [ctypes.c_void_p]
+    assert f(NUL, A, A, A, 1, 1, 128, 128, 128, S) == 1
+    assert f(A, A, A, A, 0, 1, 128, 128, 128, S) == 1
+    assert f(A, A, A, A, 1, 1, 0, 128, 128, S) == 1
+    assert f(A, A, A, A, 300, 300, 128, 128, 128, S) == 1  # B*H > 65535
+    assert f(A, A, A, A, 1, 1, 128, 96, 128, S) == 2
+    assert f(A, A, A, A, 1, 1, 128, 128, 32, S) == 2
+    assert f(MIS, A, A, A, 1, 1, 128, 128, 128, S) == 1
+
+
+def test_select_argument_checks(lib):
+    f = lib.sa_select_mask_topk_topp
+    f.argtypes = [ctypes.c_void_p] * 2 + [ctypes.c_int] * 5 + [ctypes.c_float] * 2 + \
+        [ctypes.c_void_p] * 4
+    ok = dict(B=1, H=1, nb=16, d=64, k=2, p=0.5, s=0.0)
+
+    def call(qp=A, mask=A2, idx=A, cnt=A2, **kw):
+        a = {**ok, **kw}
+        return f(qp, A, a["B"], a["H"], a["nb"], a["d"], a["k"], a["p"], a["s"], mask, idx, cnt, S)
+
+    assert call(qp=NUL) == 1
+    assert call(k=-1) == 1
+    assert call(p=1.5) == 1
+    assert call(p=-0.1) == 1
+    assert call(p=float("nan")) == 1
+    assert call(s=float("nan")) == 1
+    assert call(d=80) == 2
+    assert call(nb=1025) == 2
+    assert call(idx=MIS) == 1
+    g = lib.sa_select_from_logits
+    g.argtypes = [ctypes.c_void_p] + [ctypes.c_int] * 4 + [ctypes.c_float] + [ctypes.c_void_p] * 4
+    assert g(NUL, 1, 1, 16, 2, 0.5, A, A, A, S) == 1
+    assert g(A, 1, 1, 2000, 2, 0.5, A, A, A, S) == 2
+    assert g(A, 1, 1, 16, 2, 2.0, A, A, A, S) == 1
+
+
+def test_attention_argument_checks(lib):
+    f = lib.sa_block_sparse_attn_fwd
+    f.argtypes = [ctypes.c_void_p] * 6 + [ctypes.c_int] * 5 + [ctypes.c_float, ctypes.c_void_p]
+    assert f(A, A, A, NUL, A, A, 1, 1, 256, 128, 128, 0.0, S) == 1
+    assert f(A, A, A, A, A, A, 1, 1, 256, 256, 128, 0.0, S) == 2
+    assert f(A, A, A, A, A, A, 1, 1, 256, 128, 256, 0.0, S) == 2
+    assert f(A, A, A, A, A, A, 1, 1, 128 * 1025, 128, 128, 0.0, S) == 2
+    assert f(A, A, A, A, A, MIS, 1, 1, 256, 128, 128, 0.0, S) == 1
+    assert f(A, A, A, A, A, A, 1, 1, 256, 128, 128, float("nan"), S) == 1
+    g = lib.sa_dense_attn_fwd
+    g.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 4 + [ctypes.c_float, ctypes.c_void_p]
+    assert g(A, A, NUL, A, 1, 1, 256, 128, 0.0, S) == 1
+    assert g(A, A, A, A, 1, 1, 256, 32, 0.0, S) == 2
+
+
+def test_python_binding_imports():
+    import block_sparse_attention_blocks_b200 as pkg
+
+    assert callable(pkg.sparse_attention)
+    assert pkg.num_blocks(75600, 128) == 591

@@ -1,0 +1,244 @@
+"""GPU parity of each kernel against the fp64 oracle on small cases (several tiles, ragged tails,
+edge cases).  All calls go through the C ABI via the Python binding."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_blocks_b200.workloads import bf16_bits_to_f32, f32_to_bf16_bits
+from tests.parity import compare_attention, compare_masks, list_from_mask
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import block_sparse_attention_blocks_b200 as bsa  # noqa: E402  (loads libbsa.so, fails loudly)
+
+DEV = torch.device("cuda", 0)
+
+
+def to_dev_bf16(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits)).view(torch.bfloat16).to(DEV)
+
+
+def dev_bits(t):
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def rand_bits(rng, shape, scale=1.0):
+    return f32_to_bf16_bits(rng.standard_normal(shape).astype(np.float32) * np.float32(scale))
+
+
+# ------------------------------------------------------------------------------------------------
+# pooling
+# ------------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("d,bs,N", [(128, 128, 1000), (64, 128, 384), (128, 64, 777), (64, 64, 65)])
+def test_pool_parity(orc, d, bs, N):
+    rng = np.random.default_rng(d + bs + N)
+    B, H = 2, 3
+    q = rand_bits(rng, (B, H, N, d), 2.0)
+    k = rand_bits(rng, (B, H, N, d), 0.5)
+    qp, kp = bsa.pool_blocks(to_dev_bf16(q), to_dev_bf16(k), bs)
+    torch.cuda.synchronize()
+    for x, got in ((q, qp), (k, kp)):
+        ref = orc.pool_blocks(x.reshape(B * H, N, d), bs).reshape(B, H, -1, d)
+        g = got.cpu().numpy().astype(np.float64)
+        # fp32 accumulation of n terms: |err| <= n * 2^-24 * max|x| (plus the final division)
+        xf = bf16_bits_to_f32(x).astype(np.float64)
+        nb = ref.shape[2]
+        for i in range(nb):
+            blk = np.abs(xf[:, :, i * bs:(i + 1) * bs]).max()
+            n = min(bs, N - i * bs)
+            tol = (n + 1) * 2.0 ** -24 * blk
+            assert np.abs(g[:, :, i] - ref[:, :, i]).max() <= tol
+
+
+# ------------------------------------------------------------------------------------------------
+# selection
+# ------------------------------------------------------------------------------------------------
+def _gpu_select_logits(logits32, topk, topp):
+    t = torch.from_numpy(np.ascontiguousarray(logits32, np.float32)).to(DEV)
+    mask, idx, cnt = bsa.select_from_logits(t, topk, topp)
+    torch.cuda.synchronize()
+    return mask.cpu().numpy(), idx.cpu().numpy(), cnt.cpu().numpy()
+
+
+def test_select_handmade_rows(orc):
+    nb = 24
+    rows = []
+    rows.append(np.log(np.r_[[0.5, 0.3, 0.15, 0.05], np.full(nb - 4, 1e-30)]))  # worked example
+    rows.append(np.zeros(nb))  # uniform row
+    sink = np.zeros(nb)
+    sink[9] = 20.0
+    rows.append(sink)  # single sink
+    rows.append(np.arange(nb, dtype=np.float64) * -0.3)  # geometric
+    rows.append(np.r_[np.full(12, 2.0), np.zeros(12)])  # ties
+    L = np.array(rows, np.float32)[None, None]  # [1, 1, rows, nb] read as one head of 5 rows
+    L = np.concatenate([L, np.zeros((1, 1, nb - L.shape[2], nb), np.float32)], 2)
+    for k, p in [(1, 0.7), (3, 0.7), (0, 0.96), (4, 0.9), (0, 0.6), (12, 0.6), (2, 0.0),
+                 (0, 1.0), (30, 0.5)]:
+        m, idx, cnt = _gpu_select_logits(L, k, p)
+        sel = orc.select_from_logits(L.astype(np.float64), k, p)
+        compare_masks(m, idx, cnt, sel)
+    # the pages' two failure modes, asserted directly on the GPU result
+    m, idx, cnt = _gpu_select_logits(L, 0, 0.6)
+    assert cnt[0, 0, 1] == math.ceil(0.6 * nb)  # uniform row: top-p keeps ceil(p nb)
+    m, idx, cnt = _gpu_select_logits(L, 4, 0.9)
+    assert set(idx[0, 0, 2, :cnt[0, 0, 2]].tolist()) == {0, 1, 2, 9}  # sink row: top-k rescues
+
+
+@pytest.mark.parametrize("nb", [7, 32, 33, 100, 256, 591, 1024])
+def test_select_parity_random(orc, nb):
+    rng = np.random.default_rng(nb)
+    B, H, d = 1, 3, 64
+    qp = (rng.standard_normal((B, H, nb, d)) * rng.uniform(0.2, 1.5)).astype(np.float32)
+    kp = (rng.standard_normal((B, H, nb, d)) * 1.0).astype(np.float32)
+    scale = 1 / math.sqrt(d)
+    for k, p in [(max(1, nb // 20), 0.9), (0, 0.5), (nb, 0.1), (3, 0.99)]:
+        mask, idx, cnt = bsa.select_mask_topk_topp(torch.from_numpy(qp).to(DEV),
+                                                   torch.from_numpy(kp).to(DEV), k, p)
+        torch.cuda.synchronize()
+        sel = orc.select(qp.astype(np.float64), kp.astype(np.float64), k, p, scale)
+        st = compare_masks(mask.cpu().numpy(), idx.cpu().numpy(), cnt.cpu().numpy(), sel)
+        assert st["mismatch"] <= max(2, st["rows"] // 50), st
+
+
+# ------------------------------------------------------------------------------------------------
+# attention with an injected mask
+# ------------------------------------------------------------------------------------------------
+def _run_sparse(q, k, v, mask, bs, scale=0.0):
+    idx, cnt = list_from_mask(mask)
+    o = bsa.block_sparse_attn_fwd(to_dev_bf16(q), to_dev_bf16(k), to_dev_bf16(v),
+                                  torch.from_numpy(idx).to(DEV), torch.from_numpy(cnt).to(DEV),
+                                  bs, scale)
+    torch.cuda.synchronize()
+    assert bsa.device_error() == 0
+    return bf16_bits_to_f32(dev_bits(o))
+
+
+@pytest.mark.parametrize("d,bs,N", [(128, 128, 1000), (64, 128, 700), (128, 64, 515),
+                                    (64, 64, 1024), (128, 128, 128), (64, 128, 1)])
+def test_attention_parity_random_masks(orc, d, bs, N):
+    rng = np.random.default_rng(N * 7 + d)
+    B, H = 1, 2
+    q = rand_bits(rng, (B, H, N, d), 1.5)
+    k = rand_bits(rng, (B, H, N, d), 1.5)
+    v = rand_bits(rng, (B, H, N, d))
+    nb = (N + bs - 1) // bs
+    mask = (rng.random((B, H, nb, nb)) < 0.4).astype(np.uint8)
+    mask[0, 0, 0, :] = 1                       # a full row
+    if nb > 1:
+        mask[0, 1, 1, :] = 0                   # an empty row -> zeros
+        mask[0, 0, nb - 1, :] = 0
+        mask[0, 0, nb - 1, nb - 1] = 1         # only the ragged tail block
+    o = _run_sparse(q, k, v, mask, bs).reshape(B * H, N, d)
+    ref = orc.masked_attention(q.reshape(B * H, N, d), k.reshape(B * H, N, d),
+                               v.reshape(B * H, N, d), mask.reshape(B * H, nb, nb), bs,
+                               1 / math.sqrt(d))
+    got = np.zeros_like(ref)
+    for s in range(B * H * nb):
+        bh, i = divmod(s, nb)
+        r1 = min(bs, N - i * bs)
+        got[s, :r1] = o[bh, i * bs:i * bs + r1]
+    compare_attention(got, ref)
+    if nb > 1:
+        assert (o[1, bs:2 * bs] == 0).all()   # the empty row
+
+
+def test_attention_all_blocks_equals_dense_oracle(orc):
+    rng = np.random.default_rng(11)
+    B, H, N, d, bs = 1, 2, 900, 128, 128
+    q, k, v = (rand_bits(rng, (B, H, N, d), 1.2) for _ in range(3))
+    nb = (N + bs - 1) // bs
+    o_sparse = _run_sparse(q, k, v, np.ones((B, H, nb, nb), np.uint8), bs)
+    od = bsa.dense_attn_fwd(to_dev_bf16(q), to_dev_bf16(k), to_dev_bf16(v))
+    torch.cuda.synchronize()
+    o_dense = bf16_bits_to_f32(dev_bits(od))
+    rows = [(bh, t) for bh in range(B * H) for t in range(0, N, 7)]
+    ref = orc.dense_attention(q.reshape(B * H, N, d), k.reshape(B * H, N, d),
+                              v.reshape(B * H, N, d), 1 / math.sqrt(d), rows)
+    for o in (o_sparse, o_dense):
+        o = o.reshape(B * H, N, d)
+        compare_attention(np.stack([o[bh, t] for bh, t in rows]), ref)
+
+
+def test_attention_large_logits_and_constant_v(orc):
+    # sharp rows (logits of order 50) exercise the online max / lazy rescale; a constant-V block
+    # returns that constant up to the bf16 rounding of P (P V uses bf16 P, l sums fp32 P)
+    rng = np.random.default_rng(12)
+    B, H, N, d, bs = 1, 1, 512, 64, 128
+    q = rand_bits(rng, (B, H, N, d), 4.0)
+    k = rand_bits(rng, (B, H, N, d), 4.0)
+    v = rand_bits(rng, (B, H, N, d))
+    nb = 4
+    mask = np.ones((B, H, nb, nb), np.uint8)
+    o = _run_sparse(q, k, v, mask, bs).reshape(N, d)
+    ref = orc.masked_attention(q[0], k[0], v[0], mask[0], bs, 1 / 8.0).reshape(N, d)
+    compare_attention(o, ref)
+    vc = f32_to_bf16_bits(np.full((B, H, N, d), 1.75, np.float32))
+    mask2 = np.zeros_like(mask)
+    mask2[..., 2] = 1
+    o2 = _run_sparse(q, k, vc, mask2, bs)
+    assert np.abs(o2 - 1.75).max() <= 1.75 * 2.0 ** -8 + 2.0 ** -7
+
+
+def test_out_of_range_ids_are_clamped_and_flagged():
+    B, H, N, d, bs = 1, 1, 256, 64, 128
+    z = torch.zeros(B, H, N, d, device=DEV, dtype=torch.bfloat16)
+    idx = torch.tensor([[[[0, 5], [1, 0]]]], dtype=torch.int32, device=DEV)
+    cnt = torch.tensor([[[2, 1]]], dtype=torch.int32, device=DEV)
+    bsa.block_sparse_attn_fwd(z, z, z, idx, cnt, bs)
+    assert bsa.device_error() == bsa.sparse_attn.SA_ERR_INVALID_ARG
+    assert bsa.device_error() == 0  # cleared
+
+
+def test_bounded_wait_reports_timeout():
+    bsa.set_wait_limit_ns(2_000_000)  # 2 ms
+    try:
+        bsa.probe_bounded_wait()
+        assert bsa.device_error() == bsa.sparse_attn.SA_ERR_TIMEOUT
+    finally:
+        bsa.set_wait_limit_ns(0)
+    assert bsa.device_error() == 0
+    # the context is still usable
+    x = torch.ones(4, device=DEV)
+    assert float(x.sum()) == 4.0
+
+
+def test_full_path_small(orc):
+    rng = np.random.default_rng(13)
+    B, H, N, d, bs, topk, topp = 1, 2, 1500, 128, 128, 2, 0.8
+    q = rand_bits(rng, (B, H, N, d), 1.0)
+    k = rand_bits(rng, (B, H, N, d), 1.0)
+    v = rand_bits(rng, (B, H, N, d))
+    o, (mask, idx, cnt) = bsa.sparse_attention(to_dev_bf16(q), to_dev_bf16(k), to_dev_bf16(v),
+                                               bs, topk, topp, return_selection=True)
+    torch.cuda.synchronize()
+    qp = orc.pool_blocks(q.reshape(B * H, N, d), bs)
+    kp = orc.pool_blocks(k.reshape(B * H, N, d), bs)
+    sel = orc.select(qp, kp, topk, topp, 1 / math.sqrt(d))
+    compare_masks(mask.cpu().numpy(), idx.cpu().numpy(), cnt.cpu().numpy(), sel)
+    gm = mask.cpu().numpy().reshape(B * H, -1, sel.mask.shape[-1])
+    ref = orc.masked_attention(q.reshape(B * H, N, d), k.reshape(B * H, N, d),
+                               v.reshape(B * H, N, d), gm, bs, 1 / math.sqrt(d))
+    og = bf16_bits_to_f32(dev_bits(o)).reshape(B * H, N, d)
+    nb = gm.shape[1]
+    got = np.zeros_like(ref)
+    for s in range(B * H * nb):
+        bh, i = divmod(s, nb)
+        r1 = min(bs, N - i * bs)
+        got[s, :r1] = og[bh, i * bs:i * bs + r1]
+    compare_attention(got, ref)
+
+
+def test_host_inputs_roundtrip(orc):
+    rng = np.random.default_rng(14)
+    B, H, N, d, bs = 1, 1, 600, 64, 128
+    q, k, v = (rand_bits(rng, (B, H, N, d)) for _ in range(3))
+    qh, kh, vh = (torch.from_numpy(x).view(torch.bfloat16).pin_memory() for x in (q, k, v))
+    o = bsa.sparse_attention(qh, kh, vh, bs, 5, 1.0)
+    assert not o.is_cuda
+    ref = orc.dense_attention(q[0], k[0], v[0], 1 / 8.0).reshape(N, d)
+    compare_attention(bf16_bits_to_f32(o.view(torch.int16).numpy().view(np.uint16))[0, 0], ref)

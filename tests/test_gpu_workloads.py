@@ -1,0 +1,101 @@
+"""GPU parity on the five video-DiT-shaped workloads at their full sizes.
+
+Masks are compared in full (every row of every head) under the rule in tests/parity.py.  The
+attention kernel gets the oracle's mask injected and is compared with the fp64 oracle on a
+seeded sample of query blocks (always including the first block and the ragged last block of
+head 0), since the oracle evaluates attention one query block at a time.  The launch
+configuration is the one bench.py times.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_blocks_b200 import workloads as W
+from tests.parity import compare_attention, compare_masks, list_from_mask
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import block_sparse_attention_blocks_b200 as bsa  # noqa: E402
+
+DEV = torch.device("cuda", 0)
+NSAMPLE = 24
+
+
+def _dev(bits):
+    return torch.from_numpy(bits).view(torch.bfloat16).to(DEV)
+
+
+def _bits(t):
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def _sample_blocks(w, rng):
+    BH, nb = w.B * w.H, w.nb
+    picks = {(0, 0), (0, nb - 1), (BH - 1, nb - 1)}
+    while len(picks) < NSAMPLE:
+        picks.add((int(rng.integers(BH)), int(rng.integers(nb))))
+    return sorted(picks)
+
+
+def _check_attention(orc, w, qb, kb, vb, q, k, v, mask_bhnn, sel_blocks):
+    BH, N, d, nb, bs = w.B * w.H, w.N, w.d, w.nb, w.bs
+    idx, cnt = list_from_mask(mask_bhnn)
+    o = bsa.block_sparse_attn_fwd(q, k, v, torch.from_numpy(idx).to(DEV),
+                                  torch.from_numpy(cnt).to(DEV), bs)
+    torch.cuda.synchronize()
+    assert bsa.device_error() == 0
+    of = W.bf16_bits_to_f32(_bits(o)).reshape(BH, N, d)
+    ref = orc.masked_attention(qb.reshape(BH, N, d), kb.reshape(BH, N, d), vb.reshape(BH, N, d),
+                               mask_bhnn.reshape(BH, nb, nb), bs, w.scale, sel_blocks)
+    got = np.zeros_like(ref)
+    for s, (bh, i) in enumerate(sel_blocks):
+        r1 = min(bs, N - i * bs)
+        got[s, :r1] = of[bh, i * bs:i * bs + r1]
+    return compare_attention(got, ref)
+
+
+@pytest.mark.parametrize("name", list(W.WORKLOADS))
+def test_workload_parity(orc, name):
+    w = W.get(name)
+    qb, kb, vb = W.make_qkv(w)
+    BH, N, d, nb, bs = w.B * w.H, w.N, w.d, w.nb, w.bs
+    q, k, v = _dev(qb), _dev(kb), _dev(vb)
+
+    # pooling: fp32 on the GPU against fp64
+    qp, kp = bsa.pool_blocks(q, k, bs)
+    oq = orc.pool_blocks(qb.reshape(BH, N, d), bs)
+    ok_ = orc.pool_blocks(kb.reshape(BH, N, d), bs)
+    for got, ref, x in ((qp, oq, qb), (kp, ok_, kb)):
+        g = got.cpu().numpy().reshape(BH, nb, d).astype(np.float64)
+        amax = np.abs(W.bf16_bits_to_f32(x)).max()
+        assert np.abs(g - ref).max() <= (bs + 1) * 2.0 ** -24 * amax
+
+    # selection at the workload's (k, p) and at every sweep point
+    points = [(w.topk, w.topp)] + [pt for pt in w.sweep if pt != (w.topk, w.topp)]
+    if name == "stress_mixed":
+        points.append((nb, w.topp))  # dense control: k = all blocks
+    oracle_mask = None
+    for topk, topp in points:
+        mask, idx, cnt = bsa.select_mask_topk_topp(qp, kp, topk, topp)
+        torch.cuda.synchronize()
+        sel = orc.select(oq, ok_, topk, topp, w.scale)
+        st = compare_masks(mask.cpu().numpy(), idx.cpu().numpy(), cnt.cpu().numpy(), sel)
+        print(f"{name} k={topk} p={topp}: density {sel.cnt.mean() / nb:.4f} {st}")
+        if (topk, topp) == (w.topk, w.topp):
+            oracle_mask = sel.mask.reshape(w.B, w.H, nb, nb)
+        if topk >= nb:
+            assert (mask.cpu().numpy() == 1).all()
+
+    # attention with the oracle's mask injected, sampled query blocks
+    rng = np.random.default_rng(1234)
+    blocks = _sample_blocks(w, rng)
+    mx, mean = _check_attention(orc, w, qb, kb, vb, q, k, v, oracle_mask, blocks)
+    print(f"{name} attention: max abs {mx:.3e} mean abs {mean:.3e}")
+    if name == "stress_mixed":
+        ones = np.ones_like(oracle_mask)
+        _check_attention(orc, w, qb, kb, vb, q, k, v, ones, blocks[:8])
