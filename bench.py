@@ -1,0 +1,491 @@
+#!/usr/bin/env python3
+"""Benchmark of block-sparse attention with hybrid top-k + top-p block masks on B200.
+
+One step is one attention call through the whole path, on inputs resident in HBM:
+    pool Q,K per block -> block scores + hybrid selection -> block-sparse attention
+at the Wan2.1-14B-720p self-attention shape (B=1, H=40, N=75600, d=128, block 128) with k for
+95 % block sparsity (k=30) and p=0.9, on seeded synthetic Q/K/V of the video-DiT structure
+described in block_sparse_attention_blocks_b200/workloads.py.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {bsa,reference}]
+
+Prints one JSON line (rank 0).  `value` is effective TFLOPS over the executed block pairs
+(4*d*rows*cols per pair, valid tokens only) per whole call, summed over ranks; `ms_per_step` is
+ms per call.  Multi-GPU: one process per GPU (torchrun), every rank runs its own independent
+call (the (b, h) units of the path never exchange data), so the scaling is weak and there is no
+collective on the data path; the step time is the max over ranks.
+
+`--impl reference` times the fp64 CPU oracle (a deliberately slow, obviously correct program)
+on the host cores on a bounded sample of the same workload and prints the same line with
+"impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ms/call and effective TFLOPS (% BF16 peak) of block-sparse attn at 95% sparsity"
+WORKLOAD = "wan14b_720p"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 2**20
+
+
+# ----------------------------------------------------------------------------------------------
+# helpers
+# ----------------------------------------------------------------------------------------------
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+                power.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(smax)),
+                "power_w_max": float(max(power)), "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def executed_flops(kv_cnt, mask, N, d, bs):
+    """4*d*sum over executed (query block, key block) pairs of valid rows x valid columns."""
+    import torch
+
+    nb = kv_cnt.shape[-1]
+    rows = torch.full((nb,), float(bs), dtype=torch.float64, device=kv_cnt.device)
+    rows[-1] = float(N - (nb - 1) * bs)
+    cols_sum = kv_cnt.to(torch.float64) * bs - mask[..., -1].to(torch.float64) * (bs - rows[-1])
+    pairs = int(kv_cnt.sum().item())
+    flops = float((4.0 * d * (cols_sum * rows).sum()).item())
+    return flops, pairs
+
+
+def make_inputs(w, rank, world):
+    """Seeded inputs; rank 0 generates them once and shares them through /dev/shm."""
+    from block_sparse_attention_blocks_b200 import workloads as W
+
+    if world == 1:
+        return W.make_qkv(w)
+    import torch.distributed as dist
+
+    shm = f"/dev/shm/bsa_bench_{w.name}_{os.getpid() if rank == 0 else 0}"
+    names = None
+    if rank == 0:
+        q, k, v = W.make_qkv(w)
+        base = f"/dev/shm/bsa_bench_{w.name}_{os.getpid()}"
+        for nm, x in zip("qkv", (q, k, v)):
+            np.save(f"{base}_{nm}.npy", x)
+        names = [base]
+    obj = [names[0] if names else None]
+    dist.broadcast_object_list(obj, src=0)
+    base = obj[0]
+    if rank != 0:
+        q, k, v = (np.load(f"{base}_{nm}.npy", mmap_mode="r") for nm in "qkv")
+        q, k, v = (np.ascontiguousarray(x) for x in (q, k, v))
+    dist.barrier()
+    if rank == 0:
+        for nm in "qkv":
+            try:
+                os.remove(f"{base}_{nm}.npy")
+            except OSError:
+                pass
+    return q, k, v
+
+
+# ----------------------------------------------------------------------------------------------
+# CPU oracle timing (reference arm and cpu_baseline)
+# ----------------------------------------------------------------------------------------------
+def oracle_sample(w, q, k, v, heads, qblocks_per_head, seed=0):
+    """Time the oracle on a bounded sample: pool + select for `heads` heads in full, then masked
+    attention for `qblocks_per_head` seeded query blocks of each.  Returns a dict with the time
+    and the executed-pair FLOPs of the sampled attention."""
+    import oracle
+
+    BH, N, d, bs, nb = w.B * w.H, w.N, w.d, w.bs, w.nb
+    qf, kf, vf = (x.reshape(BH, N, d) for x in (q, k, v))
+    hs = list(heads)
+    t0 = time.perf_counter()
+    qp = oracle.pool_blocks(qf[hs], bs)
+    kp = oracle.pool_blocks(kf[hs], bs)
+    sel = oracle.select(qp, kp, w.topk, w.topp, w.scale)
+    t_ps = time.perf_counter() - t0
+    rng = np.random.default_rng(seed)
+    picks = [(hi, int(i)) for hi in range(len(hs))
+             for i in rng.choice(nb, size=min(qblocks_per_head, nb), replace=False)]
+    mask = sel.mask.reshape(len(hs), nb, nb)
+    t0 = time.perf_counter()
+    oracle.masked_attention(qf[hs], kf[hs], vf[hs], mask, bs, w.scale, picks)
+    t_att = time.perf_counter() - t0
+    flops = 0.0
+    last = N - (nb - 1) * bs
+    for hi, i in picks:
+        rows = bs if i < nb - 1 else last
+        cols = mask[hi, i].sum() * bs - (bs - last) * mask[hi, i, nb - 1]
+        flops += 4.0 * d * rows * cols
+    pairs_sel = mask.sum()
+    # the full call: pool+select of all heads scales with heads, attention with executed pairs
+    return {"t_pool_select": t_ps, "t_attn": t_att, "attn_flops": flops, "heads": len(hs),
+            "qblocks": len(picks), "pairs_heads": int(pairs_sel), "threads": oracle.num_threads()}
+
+
+def cpu_estimate(w, s, total_flops):
+    """Extrapolate a sample to the full call: pool+select by heads, attention by FLOPs."""
+    t_ps_full = s["t_pool_select"] * (w.B * w.H) / s["heads"]
+    t_att_full = s["t_attn"] * total_flops / max(s["attn_flops"], 1.0)
+    ms = (t_ps_full + t_att_full) * 1e3
+    return ms, total_flops / (ms * 1e-3) / 1e12
+
+
+def run_reference(args, w):
+    """--impl reference: the oracle, as it stands, on the host cores."""
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    from block_sparse_attention_blocks_b200 import workloads as W
+
+    q, k, v = W.make_qkv(w)
+    # warm-up and timed steps; one step = pool + select of one head in full and masked attention
+    # of one seeded query block of that head (a bounded sample of the call)
+    def step(i):
+        h = i % (w.B * w.H)
+        return oracle_sample(w, q, k, v, [h], 1, seed=i)
+
+    for i in range(args.warmup):
+        step(i)
+    samples = []
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        samples.append(step(args.warmup + i))
+    elapsed = time.perf_counter() - t0
+    flops = sum(s["attn_flops"] for s in samples)
+    value = flops / elapsed / 1e12
+    threads = samples[0]["threads"] if samples else 0
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": elapsed * 1e3 / max(args.steps, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(w, None),
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": threads, "kind": "oracle",
+                         "sample": "per step: fp64 pool + scores + hybrid selection of one head "
+                                   "in full, then masked attention of one seeded query block of "
+                                   "that head; value = that block's executed-pair FLOPs / time "
+                                   "of the whole step"},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(w, extra):
+    c = {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "block": w.bs,
+         "topk": w.topk, "topp": w.topp,
+         "latent_grid": list(w.grid),
+         "l2": f"inputs larger than L2: Q, K, V are {w.B * w.H * w.N * w.d * 2 / 1e6:.0f} MB "
+               f"each (L2 {L2_BYTES / 2**20:.0f} MiB); pooling streams Q and K every step"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+# ----------------------------------------------------------------------------------------------
+# GPU arm
+# ----------------------------------------------------------------------------------------------
+def run_gpu(args, w):
+    import torch
+
+    world, rank, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    import block_sparse_attention_blocks_b200 as bsa
+
+    q_np, k_np, v_np = make_inputs(w, rank, world)
+    as_bf16 = lambda a: torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16)
+    q, k, v = (as_bf16(a).to(dev) for a in (q_np, k_np, v_np))
+    B, H, N, d, bs, nb = w.B, w.H, w.N, w.d, w.bs, w.nb
+    qp = torch.empty(B, H, nb, d, device=dev, dtype=torch.float32)
+    kp = torch.empty_like(qp)
+    mask = torch.empty(B, H, nb, nb, device=dev, dtype=torch.uint8)
+    kv_idx = torch.empty(B, H, nb, nb, device=dev, dtype=torch.int32)
+    kv_cnt = torch.empty(B, H, nb, device=dev, dtype=torch.int32)
+    o = torch.empty_like(q)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        bsa.pool_blocks(q, k, bs, qp=qp, kp=kp)
+        if ev is not None:
+            ev[1].record(stream)
+        bsa.select_mask_topk_topp(qp, kp, w.topk, w.topp, mask=mask, kv_idx=kv_idx, kv_cnt=kv_cnt)
+        if ev is not None:
+            ev[2].record(stream)
+        bsa.block_sparse_attn_fwd(q, k, v, kv_idx, kv_cnt, bs, o=o)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    err = bsa.device_error()
+    if err:
+        raise RuntimeError(f"device error {err} during warm-up")
+    flops, pairs = executed_flops(kv_cnt, mask, N, d, bs)
+    density = pairs / float(B * H * nb * nb)
+
+    # ---------------------------------------------------------------- timed region
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.3)  # let the sampler attach before the work starts
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    ms_total = start.elapsed_time(end)
+    t_pool = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    t_sel = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    t_att = float(np.mean([e[2].elapsed_time(e[3]) for e in evs]))
+    if world > 1:
+        import torch.distributed as dist
+
+        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    err = bsa.device_error()
+    if err:
+        raise RuntimeError(f"device error {err} in the timed region")
+
+    # ---------------------------------------------------------------- end to end from the host
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = (as_bf16(a).pin_memory() for a in (q_np, k_np, v_np))
+        oh = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+        e2e_steps = max(1, min(args.steps, args.e2e_steps))
+
+        def e2e_step():
+            q.copy_(qh, non_blocking=True)
+            k.copy_(kh, non_blocking=True)
+            v.copy_(vh, non_blocking=True)
+            step()
+            oh.copy_(o, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            torch.distributed.barrier()
+        s2.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e2.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_e2e = s2.elapsed_time(e2) / e2e_steps
+        if world > 1:
+            import torch.distributed as dist
+
+            t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        nbytes = q.numel() * 2
+        e2e = {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOPS",
+               "ms_per_step": ms_e2e, "steps": e2e_steps,
+               "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
+               "path": "pinned host Q,K,V -> device, pool/select/attention through the Python "
+                       "binding of the C ABI, O -> pinned host"}
+
+    # ---------------------------------------------------------------- dense control (context)
+    dense = None
+    if not args.no_dense and rank == 0:
+        od = torch.empty_like(q)
+        bsa.dense_attn_fwd(q, k, v, o=od)
+        torch.cuda.synchronize(dev)
+        sd, ed = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        sd.record(stream)
+        for _ in range(args.dense_steps):
+            bsa.dense_attn_fwd(q, k, v, o=od)
+        ed.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_d = sd.elapsed_time(ed) / args.dense_steps
+        ld = float(N - (nb - 1) * bs)
+        dense_flops = 4.0 * d * N * N * B * H
+        dense = {"ms": ms_d, "tflops": dense_flops / (ms_d * 1e-3) / 1e12,
+                 "sparse_call_speedup": ms_d / ms_step}
+        del od
+
+    peaks, peak_src = load_peaks()
+    peak_tc = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    peak_hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    att_tflops = flops / (t_att * 1e-3) / 1e12
+    ps_bytes = (2 * q.numel() * 2 + 2 * qp.numel() * 4            # pool: read Q,K, write Qp,Kp
+                + 2 * qp.numel() * 4 + mask.numel()                 # select: read Qp,Kp, mask
+                + 4 * (kv_cnt.numel() + pairs))                     # kv_cnt + kept ids
+    ps_gbs = ps_bytes / ((t_pool + t_sel) * 1e-3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": world * flops / (ms_step * 1e-3) / 1e12,
+        "unit": "TFLOPS",
+        "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": config_dict(w, {"realized_density": density, "executed_pairs": pairs,
+                                  "effective_flops_per_call": flops}),
+        "roofline": {"kernel": "attn_fwd_kernel<128,128>", "bound": "tensor",
+                     "achieved": att_tflops, "peak": peak_tc, "unit": "TFLOP/s",
+                     "frac": att_tflops / peak_tc, "traffic": None,
+                     "peak_source": f"bf16_tflops_sustained of {peak_src}",
+                     "frac_of_burst_peak": att_tflops / peaks.get("bf16_tflops", peak_tc),
+                     "algorithmic": "4*d*rows*cols per executed (query block, key block) pair, "
+                                    "valid tokens only; x pairs per launch"},
+        "roofline_pool_select": {"bound": "hbm", "achieved": ps_gbs, "peak": peak_hbm,
+                                 "unit": "GB/s", "frac": ps_gbs / peak_hbm,
+                                 "bytes_per_call": ps_bytes,
+                                 "peak_source": f"hbm_gbs of {peak_src}"},
+        "kernels_ms": {"pool": t_pool, "select": t_sel, "attention": t_att},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk,
+    }
+    if e2e:
+        line["e2e"] = e2e
+    if dense:
+        line["dense_control"] = dense
+
+    # ---------------------------------------------------------------- oracle on the host
+    if rank == 0 and world == 1 and not args.no_cpu:
+        s = oracle_sample(w, q_np, k_np, v_np, heads=range(min(4, B * H)), qblocks_per_head=4)
+        ms_cpu, tf_cpu = cpu_estimate(w, s, flops)
+        line["cpu_baseline"] = {
+            "value": tf_cpu, "unit": "TFLOPS", "cores": s["threads"], "kind": "oracle",
+            "ms_per_call_extrapolated": ms_cpu,
+            "sample": f"fp64 pool + scores + selection of {s['heads']} heads in full "
+                      f"({s['t_pool_select']:.2f} s) and masked attention of {s['qblocks']} seeded "
+                      f"query blocks ({s['t_attn']:.2f} s); extrapolated to the call by heads and "
+                      f"by executed-pair FLOPs"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("bsa", "reference"), default="bsa")
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--topk", type=int, default=None)
+    ap.add_argument("--topp", type=float, default=None)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--dense-steps", type=int, default=3)
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    from block_sparse_attention_blocks_b200 import workloads as W
+
+    w = W.get(args.workload)
+    if args.topk is not None or args.topp is not None:
+        w = w.with_selection(args.topk if args.topk is not None else w.topk,
+                             args.topp if args.topp is not None else w.topp)
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

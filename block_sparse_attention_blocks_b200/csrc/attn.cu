@@ -30,7 +30,17 @@ struct AttnParams {
     long long units;        // BH * nbq
     float scale_log2;       // softmax scale * log2(e)
     unsigned long long wait_ns;
+    unsigned int *progress;  // optional host-mapped [grid, 8] stage words for diagnosis
 };
+
+// Stage report for diagnosis: word (cta, role) = stage << 24 | step << 12 | unit (low bits).
+__device__ __forceinline__ void report(unsigned int *progress, int role, int stage, int step,
+                                       long long unit) {
+    if (progress && (threadIdx.x & 31) == 0) {
+        volatile unsigned int *w = progress + blockIdx.x * 8 + role;
+        *w = ((unsigned)stage << 24) | (((unsigned)step & 0xFFFu) << 12) | ((unsigned)unit & 0xFFFu);
+    }
+}
 
 template <int D, int BS>
 struct AttnCfg {
@@ -60,9 +70,10 @@ __device__ __forceinline__ int clamp_block(int j, int nbk) {
 }
 
 // Waits used while unwinding after an abort: they ignore the abort flag but stay bounded.
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, unsigned long long ns) {
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, unsigned long long ns,
+                                           uint32_t tag) {
     int never = 0;
-    mbar_wait(bar, parity, ns, (volatile int *)&never);
+    mbar_wait(bar, parity, ns, (volatile int *)&never, tag, 0);
 }
 
 template <int D, int BS>
@@ -103,8 +114,10 @@ __global__ void __launch_bounds__(256, 2)
         prefetch_tmap(&tmV);
     }
     if (warp == 2) {
+        report(prm.progress, 2, 0, 0, 0);
         tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
         tmem_relinquish();
+        report(prm.progress, 2, 1, 0, 0);
     }
     tc_fence_before();
     __syncthreads();
@@ -115,8 +128,10 @@ __global__ void __launch_bounds__(256, 2)
     const unsigned long long wns = prm.wait_ns;
     const bool dense = prm.kv_idx == nullptr;
 
-    if (warp == 0 && lane == 0) {
+    if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer
+        // The whole warp walks the loop (so it reaches the final CTA barrier converged); lane 0
+        // arms the barriers and issues the copies.
         uint32_t nq = 0, nk = 0, nv = 0;
         bool ok = true;
         for (long long u = blockIdx.x; u < prm.units && ok; u += gridDim.x) {
@@ -125,35 +140,51 @@ __global__ void __launch_bounds__(256, 2)
             const int bh = (int)(u / prm.nbq);
             const int i = (int)(u - (long long)bh * prm.nbq);
             const int32_t *list = dense ? nullptr : prm.kv_idx + (size_t)u * prm.nbk;
-            if (nq > 0 && !(ok = mbar_wait(bar(B_QE), (nq - 1) & 1, wns, abort_flag))) break;
-            mbar_arrive_expect_tx(bar(B_QF), C::Q_BYTES);
+            report(prm.progress, 0, 1, 0, u);
+            if (nq > 0 && !(ok = warp_wait(bar(B_QE), (nq - 1) & 1, wns, abort_flag, 0x11, (uint32_t)u)))
+                break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bar(B_QF), C::Q_BYTES);
 #pragma unroll
-            for (int c = 0; c < C::CHUNKS; ++c)
-                tma_load_3d(sQ + c * C::Q_CHUNK, &tmQ, bar(B_QF), c * 64, i * BS, bh);
+                for (int c = 0; c < C::CHUNKS; ++c)
+                    tma_load_3d(sQ + c * C::Q_CHUNK, &tmQ, bar(B_QF), c * 64, i * BS, bh);
+            }
             ++nq;
             for (int t = 0; t < cnt; ++t) {
+                const uint32_t where = ((uint32_t)t << 16) | ((uint32_t)u & 0xFFFFu);
                 const int j = dense ? t : clamp_block(list[t], prm.nbk);
-                if (nk > 0 && !(ok = mbar_wait(bar(B_KE), (nk - 1) & 1, wns, abort_flag))) break;
-                mbar_arrive_expect_tx(bar(B_KF), C::KV_BYTES);
+                report(prm.progress, 0, 2, t, u);
+                if (nk > 0 && !(ok = warp_wait(bar(B_KE), (nk - 1) & 1, wns, abort_flag, 0x12, where)))
+                    break;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(bar(B_KF), C::KV_BYTES);
 #pragma unroll
-                for (int c = 0; c < C::CHUNKS; ++c)
-                    tma_load_3d(sK + c * C::KV_CHUNK, &tmK, bar(B_KF), c * 64, j * BS, bh);
+                    for (int c = 0; c < C::CHUNKS; ++c)
+                        tma_load_3d(sK + c * C::KV_CHUNK, &tmK, bar(B_KF), c * 64, j * BS, bh);
+                }
                 ++nk;
-                if (nv > 0 && !(ok = mbar_wait(bar(B_VE), (nv - 1) & 1, wns, abort_flag))) break;
-                mbar_arrive_expect_tx(bar(B_VF), C::KV_BYTES);
+                report(prm.progress, 0, 3, t, u);
+                if (nv > 0 && !(ok = warp_wait(bar(B_VE), (nv - 1) & 1, wns, abort_flag, 0x13, where)))
+                    break;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(bar(B_VF), C::KV_BYTES);
 #pragma unroll
-                for (int c = 0; c < C::CHUNKS; ++c)
-                    tma_load_3d(sV + c * C::KV_CHUNK, &tmV, bar(B_VF), c * 64, j * BS, bh);
+                    for (int c = 0; c < C::CHUNKS; ++c)
+                        tma_load_3d(sV + c * C::KV_CHUNK, &tmV, bar(B_VF), c * 64, j * BS, bh);
+                }
                 ++nv;
             }
         }
-        if (!ok) {  // let every copy that was started land before the CTA leaves
-            if (nq) drain_wait(bar(B_QF), (nq - 1) & 1, wns);
-            if (nk) drain_wait(bar(B_KF), (nk - 1) & 1, wns);
-            if (nv) drain_wait(bar(B_VF), (nv - 1) & 1, wns);
+        report(prm.progress, 0, 4, 0, 0);
+        if (!ok && lane == 0) {  // let every copy that was started land before the CTA leaves
+            if (nq) drain_wait(bar(B_QF), (nq - 1) & 1, wns, 0x41);
+            if (nk) drain_wait(bar(B_KF), (nk - 1) & 1, wns, 0x42);
+            if (nv) drain_wait(bar(B_VF), (nv - 1) & 1, wns, 0x43);
         }
-    } else if (warp == 1 && lane == 0) {
+    } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
+        // Converged warp like the producer; lane 0 issues the MMAs and the commits (a commit
+        // tracks the MMAs of the thread that issues it).
         constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BS, 0, 0);
         constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, 0, 1);
         uint32_t nq = 0, nk = 0, nv = 0, np = 0, npv = 0, ned = 0, units_done = 0;
@@ -161,48 +192,68 @@ __global__ void __launch_bounds__(256, 2)
         for (long long u = blockIdx.x; u < prm.units && ok; u += gridDim.x) {
             const int cnt = dense ? prm.nbk : min(max(prm.kv_cnt[u], 0), prm.nbk);
             if (cnt == 0) continue;
-            if (!(ok = mbar_wait(bar(B_QF), nq & 1, wns, abort_flag))) break;
+            report(prm.progress, 1, 1, 0, u);
+            if (!(ok = warp_wait(bar(B_QF), nq & 1, wns, abort_flag, 0x21, (uint32_t)u))) break;
             ++nq;
             for (int t = 0; t < cnt; ++t) {
-                if (!(ok = mbar_wait(bar(B_KF), nk & 1, wns, abort_flag))) break;
+                const uint32_t where = ((uint32_t)t << 16) | ((uint32_t)u & 0xFFFFu);
+                report(prm.progress, 1, 2, t, u);
+                if (!(ok = warp_wait(bar(B_KF), nk & 1, wns, abort_flag, 0x22, where))) break;
+                report(prm.progress, 1, 3, t, u);
                 ++nk;
                 // S/P columns are reused: the previous P V must have finished reading P
-                if (npv > 0 && !(ok = mbar_wait(bar(B_OD), (npv - 1) & 1, wns, abort_flag))) break;
+                if (npv > 0 && !(ok = warp_wait(bar(B_OD), (npv - 1) & 1, wns, abort_flag, 0x23, where)))
+                    break;
                 tc_fence_after();
+                if (lane == 0) {
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk & 3) * 32;  // K step inside the 128-byte swizzled row
-                    const uint64_t a = smem_desc_sw128(sQ + (kk >> 2) * C::Q_CHUNK + off, 16, 1024);
-                    const uint64_t b = smem_desc_sw128(sK + (kk >> 2) * C::KV_CHUNK + off, 16, 1024);
-                    mma_ss(tS, a, b, IDESC_S, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk & 3) * 32;  // K step inside the 128-byte swizzled row
+                        const uint64_t a = smem_desc_sw128(sQ + (kk >> 2) * C::Q_CHUNK + off, 16, 1024);
+                        const uint64_t b = smem_desc_sw128(sK + (kk >> 2) * C::KV_CHUNK + off, 16, 1024);
+                        mma_ss(tS, a, b, IDESC_S, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(bar(B_SF));
+                    mma_commit(bar(B_KE));
+                    if (t == cnt - 1) mma_commit(bar(B_QE));
                 }
-                mma_commit(bar(B_SF));
-                mma_commit(bar(B_KE));
-                if (t == cnt - 1) mma_commit(bar(B_QE));
-                if (!(ok = mbar_wait(bar(B_PF), np & 1, wns, abort_flag))) break;
+                __syncwarp();
+                report(prm.progress, 1, 4, t, u);
+                if (!(ok = warp_wait(bar(B_PF), np & 1, wns, abort_flag, 0x24, where))) break;
+                report(prm.progress, 1, 5, t, u);
                 ++np;
                 if (t == 0 && units_done > 0) {
                     // O is about to be overwritten: the previous epilogue must have read it
-                    if (!(ok = mbar_wait(bar(B_ED), ned & 1, wns, abort_flag))) break;
+                    if (!(ok = warp_wait(bar(B_ED), ned & 1, wns, abort_flag, 0x25, (uint32_t)u))) break;
                     ++ned;
                 }
-                if (!(ok = mbar_wait(bar(B_VF), nv & 1, wns, abort_flag))) break;
+                report(prm.progress, 1, 6, t, u);
+                if (!(ok = warp_wait(bar(B_VF), nv & 1, wns, abort_flag, 0x26, where))) break;
+                report(prm.progress, 1, 7, t, u);
                 ++nv;
                 tc_fence_after();
+                if (lane == 0) {
 #pragma unroll
-                for (int kk = 0; kk < BS / 16; ++kk) {
-                    const uint64_t b = smem_desc_sw128(sV + kk * 2048, C::KV_CHUNK, 1024);
-                    mma_ts(tO, tS + kk * 8, b, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < BS / 16; ++kk) {
+                        const uint64_t b = smem_desc_sw128(sV + kk * 2048, C::KV_CHUNK, 1024);
+                        mma_ts(tO, tS + kk * 8, b, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(bar(B_VE));
+                    mma_commit(bar(B_OD));
                 }
-                mma_commit(bar(B_VE));
-                mma_commit(bar(B_OD));
+                __syncwarp();
+                report(prm.progress, 1, 8, t, u);
                 ++npv;
             }
             ++units_done;
         }
-        // every MMA this thread issued must be complete before tensor memory is released
-        mma_commit(bar(B_FIN));
-        drain_wait(bar(B_FIN), 0, wns);
+        // every MMA this warp issued must be complete before tensor memory is released
+        report(prm.progress, 1, 9, 0, 0);
+        if (lane == 0) {
+            mma_commit(bar(B_FIN));
+            drain_wait(bar(B_FIN), 0, wns, 0x44);
+        }
+        report(prm.progress, 1, 10, 0, 0);
     } else if (warp >= 4) {
         // ---------------------------------------------------------------- softmax + epilogue
         const int q4 = warp & 3;
@@ -233,7 +284,8 @@ __global__ void __launch_bounds__(256, 2)
             for (int t = 0; t < cnt; ++t) {
                 const int j = dense ? t : min(max(list[t], 0), prm.nbk - 1);
                 const int valid = min(BS, prm.N - j * BS);
-                if (!(ok = mbar_wait(bar(B_SF), ns & 1, wns, abort_flag))) break;
+                report(prm.progress, 4 + q4, 1, t, u);
+                if (!(ok = warp_wait(bar(B_SF), ns & 1, wns, abort_flag, 0x31, ((uint32_t)t << 16) | ((uint32_t)u & 0xFFFFu)))) break;
                 ++ns;
                 tc_fence_after();
                 uint32_t v[32];
@@ -245,9 +297,16 @@ __global__ void __launch_bounds__(256, 2)
                     for (int e = 0; e < 32; ++e)
                         if (c * 32 + e < valid) mx = fmaxf(mx, __uint_as_float(v[e]));
                 }
+                report(prm.progress, 4 + q4, 2, t, u);
                 const float mxs = mx * sl2;
-                if (mxs > m_ref + 8.f) {
-                    const float alpha = ex2(m_ref - mxs);  // 0 on the first block
+                // Lazy rescale: a row moves its reference max only when the block max exceeds it
+                // by more than 2^8.  The decision is taken per warp (tcgen05.ld/st are
+                // .sync.aligned, so the whole warp must execute them); each lane scales by its
+                // own alpha, 1 for rows that keep their reference, 0 on the first block.
+                const bool grow = mxs > m_ref + 8.f;
+                if (__any_sync(0xffffffffu, grow)) {
+                    const float m_new = grow ? mxs : m_ref;
+                    const float alpha = ex2(m_ref - m_new);
                     if (t > 0) {
                         // the previous P V is complete: this S was issued after it finished
 #pragma unroll
@@ -260,7 +319,7 @@ __global__ void __launch_bounds__(256, 2)
                         }
                     }
                     l *= alpha;
-                    m_ref = mxs;
+                    m_ref = m_new;
                 }
 #pragma unroll 1
                 for (int c = 0; c < BS / 32; ++c) {
@@ -280,11 +339,13 @@ __global__ void __launch_bounds__(256, 2)
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(bar(B_PF));
+                report(prm.progress, 4 + q4, 3, t, u);
             }
             if (!ok) break;
             // epilogue: wait for the last P V of this query block
             npv += cnt;
-            if (!(ok = mbar_wait(bar(B_OD), (npv - 1) & 1, wns, abort_flag))) break;
+            report(prm.progress, 4 + q4, 4, 0, u);
+            if (!(ok = warp_wait(bar(B_OD), (npv - 1) & 1, wns, abort_flag, 0x32, (uint32_t)u))) break;
             tc_fence_after();
             const float inv_l = 1.f / l;
 #pragma unroll
@@ -305,13 +366,20 @@ __global__ void __launch_bounds__(256, 2)
             }
             tc_fence_before();
             mbar_arrive(bar(B_ED));
+            report(prm.progress, 4 + q4, 5, 0, u);
         }
+        report(prm.progress, 4 + q4, 6, 0, 0);
     }
 
+    __syncwarp();
+    if (warp == 2) report(prm.progress, 2, 2, 0, 0);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 2) tmem_dealloc(tbase, C::TMEM_COLS);
+    if (warp == 2) {
+        tmem_dealloc(tbase, C::TMEM_COLS);
+        report(prm.progress, 2, 3, 0, 0);
+    }
 }
 
 // ------------------------------------------------------------------------------------------
@@ -336,8 +404,9 @@ static cudaError_t launch_attn_t(const CUtensorMap &tq, const CUtensorMap &tk, c
 cudaError_t attn_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                      const int32_t *kv_idx, const int32_t *kv_cnt, void *o, long long BH, int N,
                      int d, int bs, float scale, unsigned long long wait_ns, int num_sms,
-                     cudaStream_t st) {
+                     unsigned int *progress, cudaStream_t st) {
     AttnParams p;
+    p.progress = progress;
     p.kv_idx = kv_idx;
     p.kv_cnt = kv_cnt;
     p.o = reinterpret_cast<__nv_bfloat16 *>(o);

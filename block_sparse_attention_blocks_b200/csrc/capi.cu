@@ -14,6 +14,7 @@ namespace {
 
 constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
 unsigned long long g_wait_ns = kDefaultWaitNs;
+unsigned int *g_progress = nullptr;  // host-mapped stage words of the attention kernel, or null
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -92,7 +93,7 @@ sa_status run_attention(const void *q, const void *k, const void *v, const int32
         !make_tmap(&tv, v, BH, N, d, bs))
         return SA_ERR_CUDA;
     return from_cuda(bsa::attn_fwd(tq, tk, tv, kv_idx, kv_cnt, o, BH, N, d, bs,
-                                   resolve_scale(scale, d), g_wait_ns, num_sms(dev),
+                                   resolve_scale(scale, d), g_wait_ns, num_sms(dev), g_progress,
                                    (cudaStream_t)stream));
 }
 
@@ -187,6 +188,20 @@ sa_status sa_get_device_error(void *stream) {
         return SA_ERR_CUDA;
     if (v & BSA_DEVERR_TIMEOUT) return SA_ERR_TIMEOUT;
     if (v & BSA_DEVERR_BOUNDS) return SA_ERR_INVALID_ARG;
+    return SA_OK;
+}
+
+sa_status sa_set_progress_buffer(void *words) {
+    g_progress = reinterpret_cast<unsigned int *>(words);
+    return SA_OK;
+}
+
+sa_status sa_get_wait_diagnostics(uint64_t *record) {
+    if (!record) return SA_ERR_INVALID_ARG;
+    unsigned long long v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_bsa_wait_diag, sizeof v) != cudaSuccess) return SA_ERR_CUDA;
+    if (v && cudaMemcpyToSymbol(g_bsa_wait_diag, &zero, sizeof zero) != cudaSuccess) return SA_ERR_CUDA;
+    *record = v;
     return SA_OK;
 }
 

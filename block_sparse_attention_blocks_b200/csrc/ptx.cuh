@@ -16,6 +16,8 @@
 // Device error word of the library (one per device), read and cleared by sa_get_device_error.
 // libbsa is a single translation unit, so it is defined here.
 __device__ unsigned int g_bsa_device_error = 0;
+// Where the first wait that ran out gave up: (site tag << 56) | (cta << 32) | detail.
+__device__ unsigned long long g_bsa_wait_diag = 0;
 
 namespace bsa {
 
@@ -49,14 +51,16 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                  : "memory");
 }
 
+// One poll of the barrier; a thread that finds the phase incomplete may be suspended for at most
+// ~20 us (explicit hint), so that the bounded waits below see the clock often.
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "r"(20000u)
         : "memory");
     return ok != 0;
 }
@@ -64,19 +68,57 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Wait for the phase with the given parity to complete.  Returns false on timeout or when
 // another role of the CTA has already aborted.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns,
-                                          volatile int *abort_flag) {
+                                          volatile int *abort_flag, uint32_t tag = 0,
+                                          uint32_t detail = 0) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     uint32_t spins = 0;
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((++spins & 63u) == 0) {
+        if ((++spins & 3u) == 0) {
             if (*abort_flag) return false;
             if (globaltimer_ns() - t0 > limit_ns) {
                 atomicOr(&g_bsa_device_error, BSA_DEVERR_TIMEOUT);
+                atomicCAS(&g_bsa_wait_diag, 0ull,
+                          ((unsigned long long)(tag & 0xFFu) << 56) |
+                              ((unsigned long long)(blockIdx.x & 0xFFFFFFu) << 32) | detail);
                 *abort_flag = 1;
                 return false;
             }
+        }
+    }
+}
+
+// Warp-uniform bounded wait.  Every lane polls the barrier (so every lane is ordered after the
+// phase completion it consumes) and a warp vote decides when to leave, so the warp stays
+// converged for the .sync.aligned tcgen05 instructions and the final CTA barrier that follow.
+// Lane 0 keeps the clock and decides on timeout / abort for the whole warp.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns,
+                                          volatile int *abort_flag, uint32_t tag = 0,
+                                          uint32_t detail = 0) {
+    const bool leader = (threadIdx.x & 31) == 0;
+    uint64_t t0 = 0;
+    uint32_t spins = 0;
+    while (true) {
+        const bool done = mbar_try_wait(bar, parity);
+        if (__all_sync(0xffffffffu, done)) return true;
+        if ((++spins & 3u) == 0) {
+            int stop = 0;
+            if (leader) {
+                const uint64_t now = globaltimer_ns();
+                if (t0 == 0) t0 = now;
+                if (*abort_flag) {
+                    stop = 1;
+                } else if (now - t0 > limit_ns) {
+                    atomicOr(&g_bsa_device_error, BSA_DEVERR_TIMEOUT);
+                    atomicCAS(&g_bsa_wait_diag, 0ull,
+                              ((unsigned long long)(tag & 0xFFu) << 56) |
+                                  ((unsigned long long)(blockIdx.x & 0xFFFFFFu) << 32) | detail);
+                    *abort_flag = 1;
+                    stop = 1;
+                }
+            }
+            if (__shfl_sync(0xffffffffu, stop, 0)) return false;
         }
     }
 }

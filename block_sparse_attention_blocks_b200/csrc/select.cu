@@ -10,9 +10,10 @@
 //   1. block_scores_kernel: fp32 SIMT GEMM L = scale * Qp Kp^T per (b, h), written into the
 //      kv_idx buffer (same size: nb x nb 32-bit words per head), which doubles as staging.
 //   2. select_rows_kernel: one warp per query-block row.  Softmax in fp32, bitonic sort of
-//      (probability, block id) keys in registers, warp prefix sum for the top-p cut, union with
-//      top-k, then the 0/1 mask row, the ascending kv_idx list and kv_cnt.  The row's logits are
-//      read into registers before any of the row's kv_idx entries is written.
+//      (score, block id) keys in registers (ranking by score is ranking by probability), warp
+//      prefix sum of the sorted probabilities for the top-p cut, union with top-k, then the 0/1
+//      mask row, the ascending kv_idx list and kv_cnt.  The row's logits are read into
+//      registers before any of the row's kv_idx entries is written.
 //
 // Because top-k and top-p both take prefixes of the same ranked order (probability descending,
 // lower block id first), their union is the longer of the two prefixes: |keep| = max(min(k,nb), m).
@@ -84,6 +85,16 @@ __global__ void __launch_bounds__(256) block_scores_kernel(const float *__restri
 // ------------------------------------------------------------------------------------------
 constexpr int SEL_WARPS = 4;
 
+// Order-preserving map of a finite float to uint32 (and back); -0 maps like +0.
+__device__ __forceinline__ uint32_t ord_bits(float x) {
+    uint32_t u = __float_as_uint(x);
+    if (u == 0x80000000u) u = 0u;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float from_ord(uint32_t o) {
+    return __uint_as_float((o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o);
+}
+
 template <int E>
 __global__ void __launch_bounds__(SEL_WARPS * 32) select_rows_kernel(
     const float *logits, long long rows, int nb, int topk, float topp, uint8_t *__restrict__ mask,
@@ -110,20 +121,19 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) select_rows_kernel(
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     float s = 0.f;
 #pragma unroll
-    for (int r = 0; r < E; ++r) {
-        x[r] = (lane * E + r) < nb ? expf(x[r] - mx) : 0.f;
-        s += x[r];
-    }
+    for (int r = 0; r < E; ++r) s += (lane * E + r) < nb ? expf(x[r] - mx) : 0.f;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
 
-    // keys: probability bits (non-negative floats order like their bit patterns) then ~id
+    // Keys: the logit mapped to an order-preserving unsigned pattern, then ~id.  Ranking by the
+    // logit is ranking by P (softmax is strictly increasing) but keeps the order of blocks whose
+    // fp32 probability underflows to 0.  -0 is folded into +0 so that equal scores tie.
     unsigned long long key[E];
 #pragma unroll
     for (int r = 0; r < E; ++r) {
         const int e = lane * E + r;
-        const float p = x[r] / s;
-        key[r] = e < nb ? ((unsigned long long)__float_as_uint(p) << 32) | (0xFFFFFFFFu - (uint32_t)e)
+        key[r] = e < nb ? ((unsigned long long)ord_bits(x[r]) << 32) |
+                              (0xFFFFFFFFu - (uint32_t)e)
                         : 0ull;
     }
     __syncwarp();
@@ -159,12 +169,12 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) select_rows_kernel(
         }
     }
 
-    // prefix sum of the sorted probabilities: lane-local, then across lanes
+    // prefix sum of the sorted probabilities P = exp(L - max) / sum: lane-local, then across lanes
     float cum[E];
     float run = 0.f;
 #pragma unroll
     for (int r = 0; r < E; ++r) {
-        run += __uint_as_float((uint32_t)(key[r] >> 32));
+        if (lane * E + r < nb) run += expf(from_ord((uint32_t)(key[r] >> 32)) - mx) / s;
         cum[r] = run;
     }
     float incl = run;

@@ -45,6 +45,13 @@ lib.sa_get_error_string.restype = ctypes.c_char_p
 
 SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_CUDA, SA_ERR_TIMEOUT = range(5)
 
+lib.sa_get_wait_diagnostics.argtypes = [ctypes.c_void_p]
+lib.sa_get_wait_diagnostics.restype = _I
+
+# BSA_WAIT_LIMIT_NS bounds every device-side wait of this process (default 2 s)
+if os.environ.get("BSA_WAIT_LIMIT_NS"):
+    lib.sa_set_wait_limit_ns(int(os.environ["BSA_WAIT_LIMIT_NS"]))
+
 
 class SAError(RuntimeError):
     def __init__(self, status: int, where: str):
@@ -188,6 +195,17 @@ def device_error(stream=None) -> int:
     """Synchronise and read/clear the library's device error word (an sa_status code)."""
     s = ctypes.c_void_p(stream) if stream is not None else _stream(None)
     return int(lib.sa_get_device_error(s))
+
+
+def wait_diagnostics() -> dict:
+    """Where the first device-side wait that ran out gave up (then cleared); {} if none did."""
+    rec = ctypes.c_uint64(0)
+    _check(lib.sa_get_wait_diagnostics(ctypes.byref(rec)), "sa_get_wait_diagnostics")
+    r = rec.value
+    if r == 0:
+        return {}
+    return {"site": r >> 56, "cta": (r >> 32) & 0xFFFFFF, "step": (r >> 16) & 0xFFFF,
+            "unit": r & 0xFFFF}
 
 
 def set_wait_limit_ns(ns: int):

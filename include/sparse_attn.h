@@ -142,6 +142,21 @@ sa_status sa_set_wait_limit_ns(uint64_t ns);
  */
 sa_status sa_probe_bounded_wait(void *stream);
 
+/*
+ * Where the first device-side wait that ran out since the last call gave up, then cleared:
+ * bits 56..63 identify the wait site (role and barrier), bits 32..55 the CTA, bits 0..31 the
+ * position (query-block unit and step).  0 when no wait has run out.
+ */
+sa_status sa_get_wait_diagnostics(uint64_t *record);
+
+/*
+ * Diagnosis aid: when `words` is non-null (host-mapped pinned memory, 8 x 32-bit words per CTA
+ * of the attention grid, i.e. at least 8 * 2 * SM-count words), later attention launches write
+ * each role's current stage there, readable by the host while the kernel runs.  NULL turns it
+ * off (the default).  The caller keeps the memory alive while launches that use it run.
+ */
+sa_status sa_set_progress_buffer(void *words);
+
 /* Number of key-block ids per row of kv_idx for a given N and bs, i.e. nb = ceil(N / bs). */
 int sa_num_blocks(int N, int bs);
 

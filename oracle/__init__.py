@@ -46,11 +46,13 @@ def _load():
     lib.or_num_threads.restype = ctypes.c_int
     lib.or_pool_blocks.argtypes = [P, I, I, I, I, P]
     lib.or_block_probs.argtypes = [P, P, I, I, I, I, D, P]
+    lib.or_block_logits.argtypes = [P, P, I, I, I, I, D, P]
     lib.or_softmax_rows.argtypes = [P, I, I, P]
     lib.or_select_rows.argtypes = [P, I, I, I, D, P, P, P, P, P, P, P, P]
     lib.or_masked_attention.argtypes = [P, P, P, I, I, I, P, D, P, P, I, P]
     lib.or_dense_attention.argtypes = [P, P, P, I, I, D, P, P, I, P]
-    for f in (lib.or_pool_blocks, lib.or_block_probs, lib.or_softmax_rows, lib.or_select_rows,
+    for f in (lib.or_pool_blocks, lib.or_block_probs, lib.or_block_logits, lib.or_softmax_rows,
+              lib.or_select_rows,
               lib.or_masked_attention, lib.or_dense_attention):
         f.restype = None
     _lib = lib
@@ -99,6 +101,18 @@ def block_probs(qp: np.ndarray, kp: np.ndarray, scale: float) -> np.ndarray:
     return out.reshape(*lead, nbq, nbk)
 
 
+def block_logits(qp: np.ndarray, kp: np.ndarray, scale: float) -> np.ndarray:
+    """The pooled block scores Qp Kp^T * scale (the logits of block_probs)."""
+    qp = np.ascontiguousarray(qp, np.float64)
+    kp = np.ascontiguousarray(kp, np.float64)
+    *lead, nbq, d = qp.shape
+    nbk = kp.shape[-2]
+    BH = int(np.prod(lead)) if lead else 1
+    out = np.empty((BH, nbq, nbk), np.float64)
+    _load().or_block_logits(_ptr(qp), _ptr(kp), BH, nbq, nbk, d, float(scale), _ptr(out))
+    return out.reshape(*lead, nbq, nbk)
+
+
 def softmax_rows(logits: np.ndarray) -> np.ndarray:
     x = np.ascontiguousarray(logits, np.float64)
     n = x.shape[-1]
@@ -116,6 +130,7 @@ class Selection:
         self.tau_k, self.tau_p, self.m_p = tau_k, tau_p, m_p
         self.cum_lo, self.cum_hi, self.rank = cum_lo, cum_hi, rank
         self.prob, self.topk, self.topp = prob, topk, topp
+        self.logit = None  # block scores, when the selection was made from scores
 
 
 def select_from_probs(prob: np.ndarray, topk: int, topp: float) -> Selection:
@@ -140,12 +155,16 @@ def select_from_probs(prob: np.ndarray, topk: int, topp: float) -> Selection:
 
 
 def select_from_logits(logits: np.ndarray, topk: int, topp: float) -> Selection:
-    return select_from_probs(softmax_rows(logits), topk, topp)
+    sel = select_from_probs(softmax_rows(logits), topk, topp)
+    sel.logit = np.ascontiguousarray(logits, np.float64)
+    return sel
 
 
 def select(qp: np.ndarray, kp: np.ndarray, topk: int, topp: float, scale: float) -> Selection:
     """Block scores, row softmax and hybrid selection from pooled Q and K."""
-    return select_from_probs(block_probs(qp, kp, scale), topk, topp)
+    sel = select_from_probs(block_probs(qp, kp, scale), topk, topp)
+    sel.logit = block_logits(qp, kp, scale)
+    return sel
 
 
 def masked_attention(q_bits, k_bits, v_bits, mask, bs: int, scale: float, sel=None):

@@ -108,6 +108,26 @@ void or_block_probs(const double *qp, const double *kp, int64_t BH, int64_t nbq,
     }
 }
 
+/* The block scores themselves, L[i, j] = Qp_i . Kp_j * scale (the logits of the softmax above).
+ * [SVG2] 2.B calls them the estimated attention scores; the near-threshold rule of the parity
+ * tests is stated on them. */
+void or_block_logits(const double *qp, const double *kp, int64_t BH, int64_t nbq, int64_t nbk,
+                     int64_t d, double scale, double *logit) {
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t bh = 0; bh < BH; ++bh) {
+        for (int64_t i = 0; i < nbq; ++i) {
+            const double *q = qp + (bh * nbq + i) * d;
+            double *row = logit + (bh * nbq + i) * nbk;
+            for (int64_t j = 0; j < nbk; ++j) {
+                const double *k = kp + (bh * nbk + j) * d;
+                double s = 0.0;
+                for (int64_t c = 0; c < d; ++c) s += q[c] * k[c];
+                row[j] = s * scale;
+            }
+        }
+    }
+}
+
 /* softmax of given logits, row by row (used to feed hand-made rows into the selection) */
 void or_softmax_rows(const double *logits, int64_t rows, int64_t n, double *prob) {
 #pragma omp parallel for schedule(static)

@@ -2,8 +2,11 @@
 
 Masks: the GPU selection runs in fp32 and the oracle in fp64, so the two may disagree only on
 blocks the rounding can flip:
-  - near-threshold blocks: |P_j - tau| <= 1e-5 * tau for tau the probability of the last block
-    of the top-k set or of the top-p set (ranking near-ties);
+  - near-threshold blocks: the block's score lies within 1e-5 relative of the score of the row's
+    threshold block (the last block of the top-k set or of the top-p set):
+    |L_j - L_tau| <= 1e-5 * max(|L_tau|, 1), L the block score Qp.Kp*scale.  For |L_tau| <= 1
+    this is the same as the probability being within 1e-5 relative of the threshold
+    probability; it is also accepted in that probability form;
   - an ambiguous top-p cut: the block just before the cut when the mass before it is within
     1e-5 of p, or the block just after it when the mass at the cut is within 1e-5 of p.
 Every other block must match bit for bit.  kv_idx / kv_cnt must be exactly the ascending list
@@ -46,6 +49,8 @@ def compare_masks(gpu_mask, gpu_idx, gpu_cnt, sel):
         if not np.array_equal(got, want):
             raise AssertionError(f"row {r}: kv_idx {got[:16]} != mask ids {want[:16]}")
 
+    L = None if sel.logit is None else np.asarray(sel.logit).reshape(-1, nb)
+    kk = min(int(sel.topk), nb)
     rows, cols = np.nonzero(gm != om)
     stats = {"rows": gm.shape[0], "blocks": gm.size, "mismatch": int(rows.size), "near_tau": 0,
              "ambiguous_cut": 0, "oracle_kept": int(om.sum()), "gpu_kept": int(gm.sum())}
@@ -57,6 +62,14 @@ def compare_masks(gpu_mask, gpu_idx, gpu_cnt, sel):
             near = True
         if mp[r] > 0 and np.isfinite(tp[r]) and abs(pj - tp[r]) <= REL_TAU * tp[r]:
             near = True
+        if not near and L is not None:
+            for thr_rank in ((kk - 1) if kk > 0 else None, (mp[r] - 1) if mp[r] > 0 else None):
+                if thr_rank is None:
+                    continue
+                jt = np.nonzero(rank[r] == thr_rank)[0][0]
+                lt = L[r, jt]
+                if abs(L[r, j] - lt) <= REL_TAU * max(abs(lt), 1.0):
+                    near = True
         if near:
             stats["near_tau"] += 1
             continue

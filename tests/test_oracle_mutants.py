@@ -19,7 +19,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 MUTANTS = {
     "pool divides by bs, not the valid count": ("double n = (double)(t1 - t0);",
                                                 "double n = (double)bs;"),
-    "score scale dropped": ("row[j] = s * scale;", "row[j] = s;"),
+    "score scale dropped": ("row[j] = s * scale;\n                if (row[j] > mx)", "row[j] = s;\n                if (row[j] > mx)"),
+    "block logits scale dropped": ("row[j] = s * scale;\n            }", "row[j] = s;\n            }"),
     "top-p uses > instead of >=": ("if (cum >= topp) { m = q + 1; break; }",
                                    "if (cum > topp) { m = q + 1; break; }"),
     "top-p cut one block short": ("if (cum >= topp) { m = q + 1; break; }",

@@ -72,6 +72,22 @@ def test_block_probs_match_scipy(orc):
     np.testing.assert_allclose(P.sum(-1), 1.0, rtol=0, atol=1e-12)
 
 
+def test_block_logits_match_einsum_and_feed_the_probs(orc):
+    from scipy.special import softmax
+
+    rng = np.random.default_rng(22)
+    qp = rng.standard_normal((3, 5, 8))
+    kp = rng.standard_normal((3, 6, 8))
+    L = orc.block_logits(qp, kp, 0.7)
+    np.testing.assert_allclose(L, np.einsum("bic,bjc->bij", qp, kp) * 0.7, rtol=1e-14, atol=1e-14)
+    np.testing.assert_allclose(orc.block_probs(qp, kp, 0.7), softmax(L, axis=-1), rtol=1e-13,
+                               atol=1e-15)
+    np.testing.assert_allclose(orc.softmax_rows(L), softmax(L, axis=-1), rtol=1e-13, atol=1e-15)
+    # asymmetric: Qp_i . Kp_j, not Kp_i . Qp_j
+    L2 = orc.block_logits(np.array([[[1.0, 0.0], [0.0, 1.0]]]), np.array([[[3.0, 0.0], [0.0, 0.0]]]), 1.0)
+    assert L2[0, 0, 0] == 3.0 and L2[0, 1, 0] == 0.0 and L2[0, 0, 1] == 0.0
+
+
 def test_block_probs_uniform_and_two_blocks(orc):
     P = orc.block_probs(np.zeros((1, 3, 4)), np.ones((1, 5, 4)), 1.0)
     assert np.allclose(P, 0.2, rtol=0, atol=1e-15)
