@@ -475,6 +475,8 @@ def main():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--dense-steps", type=int, default=3)
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="run only the first H heads (small cases for profiling; not a bench line)")
     args = ap.parse_args()
     from block_sparse_attention_blocks_b200 import workloads as W
 
@@ -482,6 +484,10 @@ def main():
     if args.topk is not None or args.topp is not None:
         w = w.with_selection(args.topk if args.topk is not None else w.topk,
                              args.topp if args.topp is not None else w.topp)
+    if args.heads is not None:
+        from dataclasses import replace
+
+        w = replace(w, H=args.heads, sink_heads=tuple(h for h in w.sink_heads if h < args.heads))
     if args.impl == "reference":
         return run_reference(args, w)
     return run_gpu(args, w)

@@ -57,6 +57,13 @@ struct AttnCfg {
     static constexpr int SMEM = OFF_BAR + 128 + 1024;  // barriers + slack for 1024-byte alignment
     static constexpr uint32_t TMEM_COLS = 256;
     static constexpr uint32_t COL_S = 0, COL_O = 128;
+    // Register split per thread: the launch gives every thread LAUNCH_REGS (256 threads, two
+    // CTAs per SM); warps 0-3 (producer, MMA issuer, allocator, idle) give registers to the
+    // softmax warpgroup, which holds a whole S row.  REGS_LO + REGS_HI == 2 * LAUNCH_REGS.
+    static constexpr int LAUNCH_REGS = 128;
+    static constexpr int REGS_LO = 56;
+    static constexpr int REGS_HI = 200;
+    static_assert(REGS_LO + REGS_HI == 2 * LAUNCH_REGS, "register split must match the launch");
 };
 
 enum { B_QF, B_QE, B_KF, B_KE, B_VF, B_VE, B_SF, B_PF, B_OD, B_ED, B_FIN, B_COUNT };
@@ -129,6 +136,7 @@ __global__ void __launch_bounds__(256, 2)
     const bool dense = prm.kv_idx == nullptr;
 
     if (warp == 0) {
+        regs_dec<C::REGS_LO>();
         // ---------------------------------------------------------------- TMA producer
         // The whole warp walks the loop (so it reaches the final CTA barrier converged); lane 0
         // arms the barriers and issues the copies.
@@ -182,6 +190,7 @@ __global__ void __launch_bounds__(256, 2)
             if (nv) drain_wait(bar(B_VF), (nv - 1) & 1, wns, 0x43);
         }
     } else if (warp == 1) {
+        regs_dec<C::REGS_LO>();
         // ---------------------------------------------------------------- MMA issuer
         // Converged warp like the producer; lane 0 issues the MMAs and the commits (a commit
         // tracks the MMAs of the thread that issues it).
@@ -201,9 +210,8 @@ __global__ void __launch_bounds__(256, 2)
                 if (!(ok = warp_wait(bar(B_KF), nk & 1, wns, abort_flag, 0x22, where))) break;
                 report(prm.progress, 1, 3, t, u);
                 ++nk;
-                // S/P columns are reused: the previous P V must have finished reading P
-                if (npv > 0 && !(ok = warp_wait(bar(B_OD), (npv - 1) & 1, wns, abort_flag, 0x23, where)))
-                    break;
+                // S overwrites the columns the previous P V reads P from: tcgen05.mma operations
+                // issued by one thread execute in issue order, so no wait is needed here.
                 tc_fence_after();
                 if (lane == 0) {
 #pragma unroll
@@ -254,7 +262,10 @@ __global__ void __launch_bounds__(256, 2)
             drain_wait(bar(B_FIN), 0, wns, 0x44);
         }
         report(prm.progress, 1, 10, 0, 0);
-    } else if (warp >= 4) {
+    } else if (warp < 4) {
+        regs_dec<C::REGS_LO>();  // allocator and idle warp: nothing to do until the end
+    } else {
+        regs_inc<C::REGS_HI>();
         // ---------------------------------------------------------------- softmax + epilogue
         const int q4 = warp & 3;
         const int r = q4 * 32 + lane;  // query row inside the tile == TMEM lane
@@ -288,15 +299,18 @@ __global__ void __launch_bounds__(256, 2)
                 if (!(ok = warp_wait(bar(B_SF), ns & 1, wns, abort_flag, 0x31, ((uint32_t)t << 16) | ((uint32_t)u & 0xFFFFu)))) break;
                 ++ns;
                 tc_fence_after();
-                uint32_t v[32];
-                float mx = -INFINITY;
-#pragma unroll 1
-                for (int c = 0; c < BS / 32; ++c) {
-                    tmem_ld32(tSr + c * 32, v);
+                // the whole S row of this thread: BS fp32 scores, one TMEM round trip
+                uint32_t s[BS];
+                tmem_ld_cols<BS>(tSr, s);
+                if (valid < BS) {  // ragged last key block (warp-uniform branch)
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (c * 32 + e < valid) mx = fmaxf(mx, __uint_as_float(v[e]));
+                    for (int e = 0; e < BS; ++e)
+                        if (e >= valid) s[e] = __float_as_uint(-INFINITY);
                 }
+                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                for (int e = 0; e < BS; ++e) m4[e & 3] = fmaxf(m4[e & 3], __uint_as_float(s[e]));
+                const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
                 report(prm.progress, 4 + q4, 2, t, u);
                 const float mxs = mx * sl2;
                 // Lazy rescale: a row moves its reference max only when the block max exceeds it
@@ -308,9 +322,10 @@ __global__ void __launch_bounds__(256, 2)
                     const float m_new = grow ? mxs : m_ref;
                     const float alpha = ex2(m_ref - m_new);
                     if (t > 0) {
-                        // the previous P V is complete: this S was issued after it finished
-#pragma unroll
+                        // the previous P V is complete: this S was issued after it, in order
+#pragma unroll 1
                         for (int c = 0; c < D / 32; ++c) {
+                            uint32_t v[32];
                             tmem_ld32(tOr + c * 32, v);
 #pragma unroll
                             for (int e = 0; e < 32; ++e)
@@ -321,21 +336,21 @@ __global__ void __launch_bounds__(256, 2)
                     l *= alpha;
                     m_ref = m_new;
                 }
-#pragma unroll 1
-                for (int c = 0; c < BS / 32; ++c) {
-                    tmem_ld32(tSr + c * 32, v);
-                    uint32_t pk[16];
+                // P = 2^(s*scale*log2e - m), packed bf16 pairs written over the consumed S columns
+                const float nm = -m_ref;
+                float l4[4] = {0.f, 0.f, 0.f, 0.f};
+                uint32_t pk[BS / 2];
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const float p0 = (c * 32 + e < valid)
-                                             ? ex2(fmaf(__uint_as_float(v[e]), sl2, -m_ref)) : 0.f;
-                        const float p1 = (c * 32 + e + 1 < valid)
-                                             ? ex2(fmaf(__uint_as_float(v[e + 1]), sl2, -m_ref)) : 0.f;
-                        l += p0 + p1;
-                        pk[e >> 1] = pack_bf16(p0, p1);
-                    }
-                    tmem_st16(tSr + c * 16, pk);  // P (bf16 pairs) over the consumed S columns
+                for (int e = 0; e < BS; e += 2) {
+                    const float p0 = ex2(fmaf(__uint_as_float(s[e]), sl2, nm));
+                    const float p1 = ex2(fmaf(__uint_as_float(s[e + 1]), sl2, nm));
+                    l4[(e >> 1) & 3] += p0 + p1;
+                    pk[e >> 1] = pack_bf16(p0, p1);
                 }
+                l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+#pragma unroll
+                for (int c = 0; c < BS / 64; ++c)
+                    tmem_st32(tSr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[c * 32]));
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(bar(B_PF));
@@ -394,6 +409,12 @@ static cudaError_t launch_attn_t(const CUtensorMap &tq, const CUtensorMap &tk, c
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, BS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
+    // setmaxnreg.inc only succeeds within the registers the CTA was launched with: refuse to
+    // launch a build whose per-thread count differs from the split's assumption.
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, BS>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != C::LAUNCH_REGS) return cudaErrorInvalidConfiguration;
     long long grid = 2LL * num_sms;
     if (grid > p.units) grid = p.units;
     if (grid <= 0) return cudaSuccess;
