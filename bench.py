@@ -131,6 +131,18 @@ def executed_flops(kv_cnt, mask, N, d, bs):
     return flops, pairs
 
 
+def max_over_ranks(x: float, device=None) -> float:
+    """The largest value of x over all ranks (identity on one process)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def make_inputs(w, rank, world):
     """Seeded inputs; rank 0 generates them once and shares them through /dev/shm."""
     from block_sparse_attention_blocks_b200 import workloads as W
@@ -139,7 +151,6 @@ def make_inputs(w, rank, world):
         return W.make_qkv(w)
     import torch.distributed as dist
 
-    shm = f"/dev/shm/bsa_bench_{w.name}_{os.getpid() if rank == 0 else 0}"
     names = None
     if rank == 0:
         q, k, v = W.make_qkv(w)
@@ -333,12 +344,7 @@ def run_gpu(args, w):
     t_pool = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
     t_sel = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
     t_att = float(np.mean([e[2].elapsed_time(e[3]) for e in evs]))
-    if world > 1:
-        import torch.distributed as dist
-
-        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, dev)
     ms_step = ms_total / args.steps
     err = bsa.device_error()
     if err:
@@ -368,13 +374,7 @@ def run_gpu(args, w):
             e2e_step()
         e2.record(stream)
         torch.cuda.synchronize(dev)
-        ms_e2e = s2.elapsed_time(e2) / e2e_steps
-        if world > 1:
-            import torch.distributed as dist
-
-            t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
+        ms_e2e = max_over_ranks(s2.elapsed_time(e2) / e2e_steps, dev)
         nbytes = q.numel() * 2
         e2e = {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOPS",
                "ms_per_step": ms_e2e, "steps": e2e_steps,

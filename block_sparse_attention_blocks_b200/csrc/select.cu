@@ -9,11 +9,11 @@
 // Two launches:
 //   1. block_scores_kernel: fp32 SIMT GEMM L = scale * Qp Kp^T per (b, h), written into the
 //      kv_idx buffer (same size: nb x nb 32-bit words per head), which doubles as staging.
-//   2. select_rows_kernel: one warp per query-block row.  Softmax in fp32, bitonic sort of
-//      (score, block id) keys in registers (ranking by score is ranking by probability), warp
-//      prefix sum of the sorted probabilities for the top-p cut, union with top-k, then the 0/1
-//      mask row, the ascending kv_idx list and kv_cnt.  The row's logits are read into
-//      registers before any of the row's kv_idx entries is written.
+//   2. select_rows_kernel: one warp per query-block row.  Softmax in fp32, then the two
+//      prefixes of the ranked order (score descending, id ascending; ranking by score is ranking
+//      by probability) found by exact threshold searches over order-preserving score keys
+//      instead of a full sort, the union, the 0/1 mask row, the ascending kv_idx list and
+//      kv_cnt.  The row's logits are read into registers before any kv_idx entry is written.
 //
 // Because top-k and top-p both take prefixes of the same ranked order (probability descending,
 // lower block id first), their union is the longer of the two prefixes: |keep| = max(min(k,nb), m).
@@ -85,152 +85,174 @@ __global__ void __launch_bounds__(256) block_scores_kernel(const float *__restri
 // ------------------------------------------------------------------------------------------
 constexpr int SEL_WARPS = 4;
 
-// Order-preserving map of a finite float to uint32 (and back); -0 maps like +0.
+// Order-preserving map of a finite float to uint32 (-0 maps like +0); 0 is below every score.
 __device__ __forceinline__ uint32_t ord_bits(float x) {
     uint32_t u = __float_as_uint(x);
     if (u == 0x80000000u) u = 0u;
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
-__device__ __forceinline__ float from_ord(uint32_t o) {
-    return __uint_as_float((o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o);
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+__device__ __forceinline__ int warp_isum(int v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
 }
 
+// One warp per query-block row; element e = r*32 + lane (coalesced, index order is r-major).
+//
+// The ranked order is (score descending, block id ascending); key[e] is the score mapped to an
+// order-preserving uint32, so "rank < R" is "key > T, or key == T and among the first few
+// tied ids" for the right threshold T.  Both sets the pages define are prefixes of this order:
+//   top-p: T_p = the largest key value whose mass  sum{P_e : key_e >= T_p} >= p  (bitwise
+//          search, 32 steps, fp32 sums in a fixed order so they are monotone in T); then the
+//          tied blocks at T_p are taken in id order until the mass reaches p;  m = their count
+//          plus the blocks above T_p.
+//   top-k: same search with the count  #{e : key_e >= T} >= k.
+// Their union is the longer prefix, |keep| = max(min(k, nb), m).
 template <int E>
 __global__ void __launch_bounds__(SEL_WARPS * 32) select_rows_kernel(
     const float *logits, long long rows, int nb, int topk, float topp, uint8_t *__restrict__ mask,
     int32_t *kv_idx, int32_t *__restrict__ kv_cnt) {
-    __shared__ __align__(16) uint8_t mrow_all[SEL_WARPS][32 * E];
     const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const long long row = (long long)blockIdx.x * SEL_WARPS + warp;
+    const long long row = (long long)blockIdx.x * SEL_WARPS + (threadIdx.x >> 5);
     if (row >= rows) return;
-    uint8_t *mrow = mrow_all[warp];
     const float *lg = logits + (size_t)row * nb;
+    const uint32_t lt_mask = (1u << lane) - 1u;
 
-    // element e = lane * E + r
     float x[E];
 #pragma unroll
     for (int r = 0; r < E; ++r) {
-        const int e = lane * E + r;
+        const int e = r * 32 + lane;
         x[r] = e < nb ? lg[e] : -INFINITY;
     }
+    __syncwarp();  // every lane has read the row before any lane writes kv_idx (same buffer)
     float mx = -INFINITY;
 #pragma unroll
     for (int r = 0; r < E; ++r) mx = fmaxf(mx, x[r]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float s = 0.f;
+    float z = 0.f;
 #pragma unroll
-    for (int r = 0; r < E; ++r) s += (lane * E + r) < nb ? expf(x[r] - mx) : 0.f;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-
-    // Keys: the logit mapped to an order-preserving unsigned pattern, then ~id.  Ranking by the
-    // logit is ranking by P (softmax is strictly increasing) but keeps the order of blocks whose
-    // fp32 probability underflows to 0.  -0 is folded into +0 so that equal scores tie.
-    unsigned long long key[E];
+    for (int r = 0; r < E; ++r) z += (r * 32 + lane) < nb ? expf(x[r] - mx) : 0.f;
+    z = warp_sum(z);
+    float p[E];
+    uint32_t key[E];
 #pragma unroll
     for (int r = 0; r < E; ++r) {
-        const int e = lane * E + r;
-        key[r] = e < nb ? ((unsigned long long)ord_bits(x[r]) << 32) |
-                              (0xFFFFFFFFu - (uint32_t)e)
-                        : 0ull;
+        const bool ok = (r * 32 + lane) < nb;
+        p[r] = ok ? expf(x[r] - mx) / z : 0.f;
+        key[r] = ok ? ord_bits(x[r]) : 0u;
     }
-    __syncwarp();
 
-    // bitonic sort, descending, over 32*E elements
+    // ---- top-p cut m
+    int m;
+    uint32_t T = 0u;  // final threshold and the number of tied blocks taken at it
+    int take = 0;
+    bool decided = false;
+    if (!(topp > 0.f)) {
+        m = 0;
+    } else if (topp >= 1.f) {
+        m = nb;
+    } else {
+        float tot = 0.f;
 #pragma unroll
-    for (int k = 2; k <= 32 * E; k <<= 1) {
+        for (int r = 0; r < E; ++r) tot += p[r];
+        if (!(warp_sum(tot) >= topp)) {
+            m = nb;
+        } else {
+            uint32_t tp = 0u;
+#pragma unroll 1
+            for (int bit = 31; bit >= 0; --bit) {
+                const uint32_t cand = tp | (1u << bit);
+                float ms = 0.f;
 #pragma unroll
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            if (j < E) {
-#pragma unroll
-                for (int r = 0; r < E; ++r) {
-                    const int l = r ^ j;
-                    if (l > r) {
-                        const bool up = ((lane * E + r) & k) == 0;
-                        const unsigned long long a = key[r], b = key[l];
-                        const bool swap = up ? (a < b) : (a > b);
-                        key[r] = swap ? b : a;
-                        key[l] = swap ? a : b;
-                    }
-                }
-            } else {
-                const int lx = j / E;
-                const bool lower = (lane & lx) == 0;
-                const bool up = ((lane * E) & k) == 0;
-                const bool keep_max = (lower == up);
-#pragma unroll
-                for (int r = 0; r < E; ++r) {
-                    const unsigned long long o = __shfl_xor_sync(0xffffffffu, key[r], lx);
-                    key[r] = keep_max ? (key[r] > o ? key[r] : o) : (key[r] < o ? key[r] : o);
-                }
+                for (int r = 0; r < E; ++r) ms += key[r] >= cand ? p[r] : 0.f;
+                if (warp_sum(ms) >= topp) tp = cand;
             }
+            int above = 0;
+            float base = 0.f;
+#pragma unroll
+            for (int r = 0; r < E; ++r) {
+                above += key[r] > tp ? 1 : 0;
+                base += key[r] > tp ? p[r] : 0.f;
+            }
+            above = warp_isum(above);
+            base = warp_sum(base);
+            // blocks tied at tp, in id order, until the mass reaches p (at least one)
+            int ntie = 0, need = 0;
+            float run = base;
+#pragma unroll
+            for (int r = 0; r < E; ++r) {
+                const bool tied = key[r] == tp;
+                const uint32_t bal = __ballot_sync(0xffffffffu, tied);
+                float v = tied ? p[r] : 0.f;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, v, o);
+                    if (lane >= o) v += y;
+                }
+                need += __popc(__ballot_sync(0xffffffffu, tied && run + v < topp));
+                run += __shfl_sync(0xffffffffu, v, 31);
+                ntie += __popc(bal);
+            }
+            const int ntake = min(need + 1, ntie);
+            m = above + ntake;
+            T = tp;
+            take = ntake;
+            decided = true;  // valid if the union is the top-p set
+        }
+    }
+    const int kk = min(topk, nb);
+    const int keep = max(kk, m);
+
+    if (!(decided && keep == m)) {
+        if (keep >= nb) {
+            T = 0u;  // every valid block (valid keys are > 0, padding is 0)
+            take = 0;
+        } else if (keep <= 0) {
+            T = 0xFFFFFFFFu;
+            take = 0;
+        } else {
+            // the keep-th largest key by count
+            uint32_t tk = 0u;
+#pragma unroll 1
+            for (int bit = 31; bit >= 0; --bit) {
+                const uint32_t cand = tk | (1u << bit);
+                int c = 0;
+#pragma unroll
+                for (int r = 0; r < E; ++r) c += key[r] >= cand ? 1 : 0;
+                if (warp_isum(c) >= keep) tk = cand;
+            }
+            int above = 0;
+#pragma unroll
+            for (int r = 0; r < E; ++r) above += key[r] > tk ? 1 : 0;
+            T = tk;
+            take = keep - warp_isum(above);
         }
     }
 
-    // prefix sum of the sorted probabilities P = exp(L - max) / sum: lane-local, then across lanes
-    float cum[E];
-    float run = 0.f;
-#pragma unroll
-    for (int r = 0; r < E; ++r) {
-        if (lane * E + r < nb) run += expf(from_ord((uint32_t)(key[r] >> 32)) - mx) / s;
-        cum[r] = run;
-    }
-    float incl = run;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const float y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-    }
-    float excl = __shfl_up_sync(0xffffffffu, incl, 1);
-    if (lane == 0) excl = 0.f;
-    int nlt = 0;
-#pragma unroll
-    for (int r = 0; r < E; ++r) nlt += ((lane * E + r) < nb && excl + cum[r] < topp) ? 1 : 0;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) nlt += __shfl_xor_sync(0xffffffffu, nlt, o);
-    int m;
-    if (!(topp > 0.f))
-        m = 0;
-    else if (topp >= 1.f)
-        m = nb;
-    else
-        m = nlt < nb ? nlt + 1 : nb;
-    const int keep = max(min(topk, nb), m);
-
-    // mask row in shared memory, by block id
-#pragma unroll
-    for (int r = 0; r < E; ++r) mrow[lane * E + r] = 0;
-    __syncwarp();
-#pragma unroll
-    for (int r = 0; r < E; ++r) {
-        const int e = lane * E + r;
-        const uint32_t id = 0xFFFFFFFFu - (uint32_t)key[r];
-        if (e < keep && id < (uint32_t)nb) mrow[id] = 1;
-    }
-    __syncwarp();
-    uint8_t *mout = mask + (size_t)row * nb;
-    for (int j = lane; j < nb; j += 32) mout[j] = mrow[j];
-
-    // ascending compaction of kept ids
-    int c = 0;
-#pragma unroll
-    for (int r = 0; r < E; ++r) c += mrow[lane * E + r];
-    int ic = c;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, ic, o);
-        if (lane >= o) ic += y;
-    }
-    int off = ic - c;
+    // ---- mark, write the mask row and the ascending id list
+    uint8_t *mrow = mask + (size_t)row * nb;
     int32_t *idx = kv_idx + (size_t)row * nb;
+    int tied_before = 0, pos = 0;
 #pragma unroll
     for (int r = 0; r < E; ++r) {
-        const int j = lane * E + r;
-        if (mrow[j]) idx[off++] = j;
+        const int e = r * 32 + lane;
+        const bool tied = key[r] == T;
+        const uint32_t tb = __ballot_sync(0xffffffffu, tied);
+        const bool kept = e < nb && (key[r] > T || (tied && tied_before + __popc(tb & lt_mask) < take));
+        tied_before += __popc(tb);
+        const uint32_t kb = __ballot_sync(0xffffffffu, kept);
+        if (e < nb) mrow[e] = kept ? 1 : 0;
+        if (kept) idx[pos + __popc(kb & lt_mask)] = e;
+        pos += __popc(kb);
     }
-    if (lane == 31) kv_cnt[row] = ic;
+    if (lane == 0) kv_cnt[row] = pos;
 }
 
 template <int E>
@@ -250,7 +272,10 @@ cudaError_t select_rows(const float *logits, long long rows, int nb, int topk, f
     if (nb <= 64) return launch_select_rows<2>(logits, rows, nb, topk, topp, mask, kv_idx, kv_cnt, st);
     if (nb <= 128) return launch_select_rows<4>(logits, rows, nb, topk, topp, mask, kv_idx, kv_cnt, st);
     if (nb <= 256) return launch_select_rows<8>(logits, rows, nb, topk, topp, mask, kv_idx, kv_cnt, st);
+    if (nb <= 384) return launch_select_rows<12>(logits, rows, nb, topk, topp, mask, kv_idx, kv_cnt, st);
     if (nb <= 512) return launch_select_rows<16>(logits, rows, nb, topk, topp, mask, kv_idx, kv_cnt, st);
+    if (nb <= 640) return launch_select_rows<20>(logits, rows, nb, topk, topp, mask, kv_idx, kv_cnt, st);
+    if (nb <= 768) return launch_select_rows<24>(logits, rows, nb, topk, topp, mask, kv_idx, kv_cnt, st);
     if (nb <= 1024) return launch_select_rows<32>(logits, rows, nb, topk, topp, mask, kv_idx, kv_cnt, st);
     return cudaErrorInvalidValue;
 }
