@@ -10,7 +10,8 @@
 // for BS = 64, rows of the next query block inside the 128-row tile) are computed but not
 // stored.  A query block with an empty list writes zeros.
 //
-// CTA roles (256 threads, two CTAs per SM, persistent over query blocks):
+// CTA roles (256 threads, two CTAs per SM, persistent; query blocks are claimed dynamically
+// from a counter in the caller's workspace, in head-major order):
 //   warp 0 lane 0  TMA producer: Q tile once per query block, then K_j and V_j per kept block
 //   warp 1 lane 0  MMA issuer:   S = Q K_j^T (SS form), O += P V_j (P read from tensor memory)
 //   warp 2         tensor-memory allocator (256 columns: S/P at 0, O at 128)
@@ -31,6 +32,7 @@ struct AttnParams {
     float scale_log2;       // softmax scale * log2(e)
     unsigned long long wait_ns;
     unsigned int *progress;  // optional host-mapped [grid, 8] stage words for diagnosis
+    unsigned int *next_unit; // work counter in the caller's workspace, zero at launch
 };
 
 // Stage report for diagnosis: word (cta, role) = stage << 24 | step << 12 | unit (low bits).
@@ -54,7 +56,8 @@ struct AttnCfg {
     static constexpr int OFF_K = OFF_Q + Q_BYTES;
     static constexpr int OFF_V = OFF_K + KV_BYTES;
     static constexpr int OFF_BAR = OFF_V + KV_BYTES;
-    static constexpr int SMEM = OFF_BAR + 128 + 1024;  // barriers + slack for 1024-byte alignment
+    static constexpr int OFF_UNITS = OFF_BAR + 8 * 24;  // after the barriers and two words
+    static constexpr int SMEM = OFF_UNITS + 16 + 1024;  // unit ring + slack for 1024-byte alignment
     static constexpr uint32_t TMEM_COLS = 256;
     static constexpr uint32_t COL_S = 0, COL_O = 128;
     // Register split per thread: the launch gives every thread LAUNCH_REGS (256 threads, two
@@ -66,7 +69,11 @@ struct AttnCfg {
     static_assert(REGS_LO + REGS_HI == 2 * LAUNCH_REGS, "register split must match the launch");
 };
 
-enum { B_QF, B_QE, B_KF, B_KE, B_VF, B_VE, B_SF, B_PF, B_OD, B_ED, B_FIN, B_COUNT };
+enum { B_QF, B_QE, B_KF, B_KE, B_VF, B_VE, B_SF, B_PF, B_OD, B_ED, B_FIN,
+       B_UF0, B_UF1, B_UF2, B_UF3,   // unit ring slot published (producer -> consumers)
+       B_UE0, B_UE1, B_UE2, B_UE3,   // unit ring slot consumed (MMA warp + 4 softmax warps)
+       B_COUNT };
+constexpr int UNIT_RING = 4;
 
 __device__ __forceinline__ int clamp_block(int j, int nbk) {
     if (j < 0 || j >= nbk) {
@@ -94,6 +101,8 @@ __global__ void __launch_bounds__(256, 2)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_BAR + 8 * B_COUNT);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_BAR + 8 * B_COUNT + 4);
+    volatile int *s_unit = reinterpret_cast<volatile int *>(smem + C::OFF_UNITS);
+    static_assert(8 * B_COUNT + 8 <= C::OFF_UNITS - C::OFF_BAR, "barrier area overflow");
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -114,6 +123,10 @@ __global__ void __launch_bounds__(256, 2)
         mbar_init(bar(B_OD), 1);
         mbar_init(bar(B_ED), 128);
         mbar_init(bar(B_FIN), 1);
+        for (int r = 0; r < UNIT_RING; ++r) {
+            mbar_init(bar(B_UF0 + r), 1);
+            mbar_init(bar(B_UE0 + r), 5);
+        }
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tmap(&tmQ);
@@ -140,9 +153,24 @@ __global__ void __launch_bounds__(256, 2)
         // ---------------------------------------------------------------- TMA producer
         // The whole warp walks the loop (so it reaches the final CTA barrier converged); lane 0
         // arms the barriers and issues the copies.
+        // Units (query blocks) are claimed from a global counter in head-major order, so all
+        // CTAs stay within about one head of each other and that head's K/V stay in L2; each
+        // claimed index is published to the MMA and softmax warps through a 4-slot ring.
         uint32_t nq = 0, nk = 0, nv = 0;
         bool ok = true;
-        for (long long u = blockIdx.x; u < prm.units && ok; u += gridDim.x) {
+        for (uint32_t kth = 0; ok; ++kth) {
+            const int slot = kth & (UNIT_RING - 1);
+            if (kth >= UNIT_RING &&
+                !(ok = warp_wait(bar(B_UE0 + slot), ((kth / UNIT_RING) - 1) & 1, wns, abort_flag, 0x14, kth)))
+                break;
+            long long u = 0;
+            if (lane == 0) {
+                u = (long long)atomicAdd(prm.next_unit, 1u);
+                s_unit[slot] = u < prm.units ? (int)u : -1;
+                mbar_arrive(bar(B_UF0 + slot));
+            }
+            u = __shfl_sync(0xffffffffu, u, 0);
+            if (u >= prm.units) break;
             const int cnt = dense ? prm.nbk : min(max(prm.kv_cnt[u], 0), prm.nbk);
             if (cnt == 0) continue;
             const int bh = (int)(u / prm.nbq);
@@ -158,9 +186,11 @@ __global__ void __launch_bounds__(256, 2)
                     tma_load_3d(sQ + c * C::Q_CHUNK, &tmQ, bar(B_QF), c * 64, i * BS, bh);
             }
             ++nq;
+            int jn = dense ? 0 : list[0];
             for (int t = 0; t < cnt; ++t) {
                 const uint32_t where = ((uint32_t)t << 16) | ((uint32_t)u & 0xFFFFu);
-                const int j = dense ? t : clamp_block(list[t], prm.nbk);
+                const int j = dense ? t : clamp_block(jn, prm.nbk);
+                if (!dense && t + 1 < cnt) jn = list[t + 1];  // next id, fetched early
                 report(prm.progress, 0, 2, t, u);
                 if (nk > 0 && !(ok = warp_wait(bar(B_KE), (nk - 1) & 1, wns, abort_flag, 0x12, where)))
                     break;
@@ -198,7 +228,14 @@ __global__ void __launch_bounds__(256, 2)
         constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, 0, 1);
         uint32_t nq = 0, nk = 0, nv = 0, np = 0, npv = 0, ned = 0, units_done = 0;
         bool ok = true;
-        for (long long u = blockIdx.x; u < prm.units && ok; u += gridDim.x) {
+        for (uint32_t kth = 0; ok; ++kth) {
+            const int slot = kth & (UNIT_RING - 1);
+            if (!(ok = warp_wait(bar(B_UF0 + slot), (kth / UNIT_RING) & 1, wns, abort_flag, 0x27, kth)))
+                break;
+            const long long u = s_unit[slot];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_UE0 + slot));
+            if (u < 0) break;
             const int cnt = dense ? prm.nbk : min(max(prm.kv_cnt[u], 0), prm.nbk);
             if (cnt == 0) continue;
             report(prm.progress, 1, 1, 0, u);
@@ -274,7 +311,14 @@ __global__ void __launch_bounds__(256, 2)
         const float sl2 = prm.scale_log2;
         uint32_t ns = 0, npv = 0;
         bool ok = true;
-        for (long long u = blockIdx.x; u < prm.units && ok; u += gridDim.x) {
+        for (uint32_t kth = 0; ok; ++kth) {
+            const int slot = kth & (UNIT_RING - 1);
+            if (!(ok = warp_wait(bar(B_UF0 + slot), (kth / UNIT_RING) & 1, wns, abort_flag, 0x33, kth)))
+                break;
+            const long long u = s_unit[slot];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_UE0 + slot));
+            if (u < 0) break;
             const int cnt = dense ? prm.nbk : min(max(prm.kv_cnt[u], 0), prm.nbk);
             const int bh = (int)(u / prm.nbq);
             const int i = (int)(u - (long long)bh * prm.nbq);
@@ -292,8 +336,10 @@ __global__ void __launch_bounds__(256, 2)
             const int32_t *list = dense ? nullptr : prm.kv_idx + (size_t)u * prm.nbk;
             float m_ref = -INFINITY;  // running max, log2 domain
             float l = 0.f;            // running sum
+            int jn = dense ? 0 : list[0];
             for (int t = 0; t < cnt; ++t) {
-                const int j = dense ? t : min(max(list[t], 0), prm.nbk - 1);
+                const int j = dense ? t : min(max(jn, 0), prm.nbk - 1);
+                if (!dense && t + 1 < cnt) jn = list[t + 1];  // next id, fetched early
                 const int valid = min(BS, prm.N - j * BS);
                 report(prm.progress, 4 + q4, 1, t, u);
                 if (!(ok = warp_wait(bar(B_SF), ns & 1, wns, abort_flag, 0x31, ((uint32_t)t << 16) | ((uint32_t)u & 0xFFFFu)))) break;
@@ -309,8 +355,10 @@ __global__ void __launch_bounds__(256, 2)
                 }
                 float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                for (int e = 0; e < BS; ++e) m4[e & 3] = fmaxf(m4[e & 3], __uint_as_float(s[e]));
-                const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+                for (int e = 0; e < BS; e += 2)
+                    m4[(e >> 1) & 3] = fmax3f(m4[(e >> 1) & 3], __uint_as_float(s[e]),
+                                              __uint_as_float(s[e + 1]));
+                const float mx = fmax3f(fmaxf(m4[0], m4[1]), m4[2], m4[3]);
                 report(prm.progress, 4 + q4, 2, t, u);
                 const float mxs = mx * sl2;
                 // Lazy rescale: a row moves its reference max only when the block max exceeds it
@@ -336,18 +384,29 @@ __global__ void __launch_bounds__(256, 2)
                     l *= alpha;
                     m_ref = m_new;
                 }
-                // P = 2^(s*scale*log2e - m), packed bf16 pairs written over the consumed S columns
-                const float nm = -m_ref;
-                float l4[4] = {0.f, 0.f, 0.f, 0.f};
+                // P = 2^(s*scale*log2e - m), packed bf16 pairs written over the consumed S columns.
+                // Three of every four pairs go through the SFU (ex2), one through the FMA-pipe
+                // polynomial, so that neither pipe limits the softmax; bf16 packing runs on the
+                // integer pipe.
+                const float2 sl2v = make_float2(sl2, sl2);
+                const float2 nmv = make_float2(-m_ref, -m_ref);
+                float2 lacc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
                 uint32_t pk[BS / 2];
 #pragma unroll
                 for (int e = 0; e < BS; e += 2) {
-                    const float p0 = ex2(fmaf(__uint_as_float(s[e]), sl2, nm));
-                    const float p1 = ex2(fmaf(__uint_as_float(s[e + 1]), sl2, nm));
-                    l4[(e >> 1) & 3] += p0 + p1;
-                    pk[e >> 1] = pack_bf16(p0, p1);
+                    const float2 xv = __ffma2_rn(
+                        make_float2(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), sl2v, nmv);
+                    float2 pv;
+                    if ((e & 6) == 6) {
+                        pv = exp2_poly2(xv);
+                    } else {
+                        pv.x = ex2(xv.x);
+                        pv.y = ex2(xv.y);
+                    }
+                    lacc[(e >> 1) & 1] = __fadd2_rn(lacc[(e >> 1) & 1], pv);
+                    pk[e >> 1] = pack_bf16_int(pv.x, pv.y);
                 }
-                l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+                l += (lacc[0].x + lacc[0].y) + (lacc[1].x + lacc[1].y);
 #pragma unroll
                 for (int c = 0; c < BS / 64; ++c)
                     tmem_st32(tSr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[c * 32]));
@@ -418,6 +477,8 @@ static cudaError_t launch_attn_t(const CUtensorMap &tq, const CUtensorMap &tk, c
     long long grid = 2LL * num_sms;
     if (grid > p.units) grid = p.units;
     if (grid <= 0) return cudaSuccess;
+    e = cudaMemsetAsync(p.next_unit, 0, sizeof(unsigned int), st);
+    if (e != cudaSuccess) return e;
     attn_fwd_kernel<D, BS><<<(unsigned)grid, 256, smem, st>>>(tq, tk, tv, p);
     return cudaGetLastError();
 }
@@ -425,9 +486,10 @@ static cudaError_t launch_attn_t(const CUtensorMap &tq, const CUtensorMap &tk, c
 cudaError_t attn_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                      const int32_t *kv_idx, const int32_t *kv_cnt, void *o, long long BH, int N,
                      int d, int bs, float scale, unsigned long long wait_ns, int num_sms,
-                     unsigned int *progress, cudaStream_t st) {
+                     unsigned int *progress, unsigned int *workspace, cudaStream_t st) {
     AttnParams p;
     p.progress = progress;
+    p.next_unit = workspace;
     p.kv_idx = kv_idx;
     p.kv_cnt = kv_cnt;
     p.o = reinterpret_cast<__nv_bfloat16 *>(o);

@@ -21,8 +21,10 @@ cudaError_t select_rows(const float *logits, long long rows, int nb, int topk, f
 cudaError_t attn_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                      const int32_t *kv_idx, const int32_t *kv_cnt, void *o, long long BH, int N,
                      int d, int bs, float scale, unsigned long long wait_ns, int num_sms,
-                     unsigned int *progress, cudaStream_t st);
+                     unsigned int *progress, unsigned int *workspace, cudaStream_t st);
 
 cudaError_t bounded_wait_probe(unsigned long long wait_ns, cudaStream_t st);
+
+cudaError_t exp2_poly_eval(const float *x, float *y, int n, cudaStream_t st);
 
 }  // namespace bsa

@@ -82,9 +82,11 @@ bool make_tmap(CUtensorMap *m, const void *base, long long BH, int N, int d, int
 
 sa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SA_OK : SA_ERR_CUDA; }
 
+constexpr size_t kAttnWorkspaceBytes = 256;
+
 sa_status run_attention(const void *q, const void *k, const void *v, const int32_t *kv_idx,
                         const int32_t *kv_cnt, void *o, int B, int H, int N, int d, int bs,
-                        float scale, void *stream) {
+                        float scale, void *workspace, void *stream) {
     int dev;
     if (!select_device(o, &dev)) return SA_ERR_INVALID_ARG;
     const long long BH = (long long)B * H;
@@ -94,6 +96,7 @@ sa_status run_attention(const void *q, const void *k, const void *v, const int32
         return SA_ERR_CUDA;
     return from_cuda(bsa::attn_fwd(tq, tk, tv, kv_idx, kv_cnt, o, BH, N, d, bs,
                                    resolve_scale(scale, d), g_wait_ns, num_sms(dev), g_progress,
+                                   reinterpret_cast<unsigned int *>(workspace),
                                    (cudaStream_t)stream));
 }
 
@@ -113,6 +116,8 @@ const char *sa_get_error_string(sa_status s) {
 }
 
 int sa_num_blocks(int N, int bs) { return (N > 0 && bs > 0) ? (N + bs - 1) / bs : 0; }
+
+size_t sa_attn_workspace_bytes(void) { return kAttnWorkspaceBytes; }
 
 sa_status sa_set_wait_limit_ns(uint64_t ns) {
     g_wait_ns = ns ? (unsigned long long)ns : kDefaultWaitNs;
@@ -162,22 +167,28 @@ sa_status sa_select_mask_topk_topp(const float *qp, const float *kp, int B, int 
 
 sa_status sa_block_sparse_attn_fwd(const void *q, const void *k, const void *v,
                                    const int32_t *kv_idx, const int32_t *kv_cnt, void *o, int B,
-                                   int H, int N, int d, int bs, float scale, void *stream) {
+                                   int H, int N, int d, int bs, float scale, void *workspace,
+                                   size_t workspace_bytes, void *stream) {
     if (!q || !k || !v || !kv_idx || !kv_cnt || !o || !shape_ok(B, H, N)) return SA_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < kAttnWorkspaceBytes || !aligned16(workspace))
+        return SA_ERR_INVALID_ARG;
     if (!dims_supported(d, bs)) return SA_ERR_UNSUPPORTED;
     if (sa_num_blocks(N, bs) > 1024) return SA_ERR_UNSUPPORTED;
     if (isnan(scale)) return SA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SA_ERR_INVALID_ARG;
-    return run_attention(q, k, v, kv_idx, kv_cnt, o, B, H, N, d, bs, scale, stream);
+    return run_attention(q, k, v, kv_idx, kv_cnt, o, B, H, N, d, bs, scale, workspace, stream);
 }
 
 sa_status sa_dense_attn_fwd(const void *q, const void *k, const void *v, void *o, int B, int H,
-                            int N, int d, float scale, void *stream) {
+                            int N, int d, float scale, void *workspace, size_t workspace_bytes,
+                            void *stream) {
     if (!q || !k || !v || !o || !shape_ok(B, H, N)) return SA_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < kAttnWorkspaceBytes || !aligned16(workspace))
+        return SA_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return SA_ERR_UNSUPPORTED;
     if (isnan(scale)) return SA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SA_ERR_INVALID_ARG;
-    return run_attention(q, k, v, nullptr, nullptr, o, B, H, N, d, 128, scale, stream);
+    return run_attention(q, k, v, nullptr, nullptr, o, B, H, N, d, 128, scale, workspace, stream);
 }
 
 sa_status sa_get_device_error(void *stream) {
@@ -203,6 +214,13 @@ sa_status sa_get_wait_diagnostics(uint64_t *record) {
     if (v && cudaMemcpyToSymbol(g_bsa_wait_diag, &zero, sizeof zero) != cudaSuccess) return SA_ERR_CUDA;
     *record = v;
     return SA_OK;
+}
+
+sa_status sa_test_exp2_poly(const float *x, float *y, int n, void *stream) {
+    if (!x || !y || n < 0) return SA_ERR_INVALID_ARG;
+    int dev;
+    if (!select_device(y, &dev)) return SA_ERR_INVALID_ARG;
+    return from_cuda(bsa::exp2_poly_eval(x, y, n, (cudaStream_t)stream));
 }
 
 sa_status sa_probe_bounded_wait(void *stream) {

@@ -17,6 +17,25 @@ __global__ void bounded_wait_probe_kernel(unsigned long long wait_ns) {
     if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, wait_ns, (volatile int *)&abort_flag);
 }
 
+// Evaluates the softmax's FMA-pipe 2^x (exp2_poly2) element-wise, for tests against exp2f.
+__global__ void exp2_poly_kernel(const float *x, float *y, int n) {
+    const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+    if (i + 1 < n) {
+        const float2 r = exp2_poly2(make_float2(x[i], x[i + 1]));
+        y[i] = r.x;
+        y[i + 1] = r.y;
+    } else if (i < n) {
+        y[i] = exp2_poly2(make_float2(x[i], x[i])).x;
+    }
+}
+
+cudaError_t exp2_poly_eval(const float *x, float *y, int n, cudaStream_t st) {
+    if (n <= 0) return cudaSuccess;
+    const int pairs = (n + 1) / 2;
+    exp2_poly_kernel<<<(pairs + 255) / 256, 256, 0, st>>>(x, y, n);
+    return cudaGetLastError();
+}
+
 cudaError_t bounded_wait_probe(unsigned long long wait_ns, cudaStream_t st) {
     bounded_wait_probe_kernel<<<1, 32, 0, st>>>(wait_ns);
     return cudaGetLastError();

@@ -309,6 +309,38 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// max of three floats (sm_100 three-input max)
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// 2^x for a pair on the FMA pipe (instead of the SFU), x <= 8: n = round(x) by the 1.5*2^23
+// trick, f = x - n in [-1/2, 1/2], 2^f by a degree-3 minimax polynomial (relative error
+// 7.5e-5, coefficients from fit_exp2_poly.py), 2^n added to the exponent field.  Inputs below
+// -126 (including -inf) are clamped there, giving ~1e-38 instead of 0.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+    const float kMagic = 12582912.0f;  // 1.5 * 2^23
+    x.x = fmaxf(x.x, -126.f);
+    x.y = fmaxf(x.y, -126.f);
+    const float2 t = __fadd2_rn(x, make_float2(kMagic, kMagic));
+    const float2 n = __fadd2_rn(t, make_float2(-kMagic, -kMagic));
+    const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+    float2 p = __ffma2_rn(make_float2(0.0551716685295105f, 0.0551716685295105f), f,
+                          make_float2(0.2426111251115799f, 0.2426111251115799f));
+    p = __ffma2_rn(p, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
+    p = __ffma2_rn(p, f, make_float2(0.9999280571937561f, 0.9999280571937561f));
+    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                       __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
+// two non-negative finite floats rounded to bf16 (nearest, ties away from zero) on the integer
+// pipe, `lo` in the low half
+__device__ __forceinline__ uint32_t pack_bf16_int(float lo, float hi) {
+    return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
+}
+
 // pack two floats into bf16x2, `lo` in the low half
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);

@@ -29,8 +29,11 @@ _F = ctypes.c_float
 lib.sa_pool_blocks.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]
 lib.sa_select_mask_topk_topp.argtypes = [_P, _P, _I, _I, _I, _I, _I, _F, _F, _P, _P, _P, _P]
 lib.sa_select_from_logits.argtypes = [_P, _I, _I, _I, _I, _F, _P, _P, _P, _P]
-lib.sa_block_sparse_attn_fwd.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]
-lib.sa_dense_attn_fwd.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P]
+_Z = ctypes.c_size_t
+lib.sa_block_sparse_attn_fwd.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _Z, _P]
+lib.sa_dense_attn_fwd.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _Z, _P]
+lib.sa_attn_workspace_bytes.argtypes = []
+lib.sa_attn_workspace_bytes.restype = _Z
 lib.sa_get_error_string.argtypes = [_I]
 lib.sa_get_error_string.restype = ctypes.c_char_p
 lib.sa_get_device_error.argtypes = [_P]
@@ -81,6 +84,22 @@ def _need(t: torch.Tensor, name: str, dtype, ndim: int):
         raise ValueError(f"{name} must be a CUDA tensor")
     if t.dim() != ndim or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous {ndim}-d tensor, got shape {tuple(t.shape)}")
+
+
+_WORKSPACES = {}
+
+
+def _workspace(device):
+    """A small device workspace per (device, current stream): launches on one stream run in
+    order, so they can share it; launches on different streams get their own."""
+    st = torch.cuda.current_stream(device)
+    key = (device.index, st.cuda_stream)
+    ws = _WORKSPACES.get(key)
+    if ws is None:
+        n = int(lib.sa_attn_workspace_bytes())
+        ws = torch.empty(n, dtype=torch.uint8, device=device)
+        _WORKSPACES[key] = ws
+    return ws
 
 
 def num_blocks(N: int, bs: int) -> int:
@@ -150,9 +169,10 @@ def block_sparse_attn_fwd(q, k, v, kv_idx, kv_cnt, bs: int, scale: float | None 
     B, H, N, d = q.shape
     o = o if o is not None else torch.empty_like(q)
     _need(o, "o", torch.bfloat16, 4)
+    ws = _workspace(q.device)
     _check(lib.sa_block_sparse_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_idx), _ptr(kv_cnt),
-                                        _ptr(o), B, H, N, d, bs, float(scale or 0.0),
-                                        _stream(q.device)), "sa_block_sparse_attn_fwd")
+                                        _ptr(o), B, H, N, d, bs, float(scale or 0.0), _ptr(ws),
+                                        ws.numel(), _stream(q.device)), "sa_block_sparse_attn_fwd")
     return o
 
 
@@ -163,8 +183,10 @@ def dense_attn_fwd(q, k, v, scale: float | None = None, o=None):
     B, H, N, d = q.shape
     o = o if o is not None else torch.empty_like(q)
     _need(o, "o", torch.bfloat16, 4)
+    ws = _workspace(q.device)
     _check(lib.sa_dense_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d,
-                                 float(scale or 0.0), _stream(q.device)), "sa_dense_attn_fwd")
+                                 float(scale or 0.0), _ptr(ws), ws.numel(), _stream(q.device)),
+           "sa_dense_attn_fwd")
     return o
 
 
@@ -206,6 +228,17 @@ def wait_diagnostics() -> dict:
         return {}
     return {"site": r >> 56, "cta": (r >> 32) & 0xFFFFFF, "step": (r >> 16) & 0xFFFF,
             "unit": r & 0xFFFF}
+
+
+def exp2_poly(x: torch.Tensor) -> torch.Tensor:
+    """The softmax's FMA-pipe 2^x evaluated on a CUDA fp32 tensor (test hook)."""
+    _need(x, "x", torch.float32, x.dim())
+    y = torch.empty_like(x)
+    lib.sa_test_exp2_poly.argtypes = [_P, _P, _I, _P]
+    lib.sa_test_exp2_poly.restype = _I
+    _check(lib.sa_test_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(x.device)),
+           "sa_test_exp2_poly")
+    return y
 
 
 def set_wait_limit_ns(ns: int):

@@ -27,7 +27,9 @@
  *
  * Conventions for every entry point:
  *   - Tensor pointers are DEVICE pointers owned by the caller.  The library allocates and frees
- *     nothing; it never synchronises the stream except in sa_get_device_error.
+ *     nothing; it never synchronises the stream except in sa_get_device_error.  The attention
+ *     entry points take a small caller-owned device workspace (sa_attn_workspace_bytes()) that
+ *     holds their work counter; calls that may overlap on the GPU need separate workspaces.
  *   - Tensors are dense and row-major with the last dimension contiguous.  bf16 tensors are
  *     passed as void*; their base addresses must be 16-byte aligned, fp32 tensors too.
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  The call
@@ -106,18 +108,25 @@ sa_status sa_select_from_logits(const float *logits, int B, int H, int nb, int t
  *           (as written by sa_select_mask_topk_topp).  kv_cnt : [B, H, nb] int32 in [0, nb].
  *           Ids outside [0, nb) are clamped and flagged in the device error word.
  * bs      : block size of both query and key blocks.  scale : <= 0 selects 1/sqrt(d).
+ * workspace: device memory of at least sa_attn_workspace_bytes() bytes, 16-byte aligned, owned
+ *           by the caller; the call zeroes its counter on `stream` before the kernel starts.
  * Arithmetic: bf16 operands, fp32 accumulation on the tensor cores, P rounded to bf16.
  */
 sa_status sa_block_sparse_attn_fwd(const void *q, const void *k, const void *v,
                                    const int32_t *kv_idx, const int32_t *kv_cnt, void *o, int B,
-                                   int H, int N, int d, int bs, float scale, void *stream);
+                                   int H, int N, int d, int bs, float scale, void *workspace,
+                                   size_t workspace_bytes, void *stream);
 
 /*
  * Dense attention forward, the 0 %-sparsity control: O = softmax(scale Q K^T) V over all N keys.
- * Same layouts and arithmetic as sa_block_sparse_attn_fwd (internally bs = 128).
+ * Same layouts, workspace and arithmetic as sa_block_sparse_attn_fwd (internally bs = 128).
  */
 sa_status sa_dense_attn_fwd(const void *q, const void *k, const void *v, void *o, int B, int H,
-                            int N, int d, float scale, void *stream);
+                            int N, int d, float scale, void *workspace, size_t workspace_bytes,
+                            void *stream);
+
+/* Bytes of device workspace the attention entry points need (a small constant). */
+size_t sa_attn_workspace_bytes(void);
 
 /* Human-readable name of a status code (static storage). */
 const char *sa_get_error_string(sa_status status);
@@ -156,6 +165,14 @@ sa_status sa_get_wait_diagnostics(uint64_t *record);
  * off (the default).  The caller keeps the memory alive while launches that use it run.
  */
 sa_status sa_set_progress_buffer(void *words);
+
+/*
+ * Test hook: y[i] = the FMA-pipe 2^x the attention softmax uses for a quarter of its
+ * probabilities (range reduction to [-1/2, 1/2] and a degree-3 minimax polynomial, relative
+ * error below 1e-4 where the result is a normal float; inputs below -126 give values below 2e-38).
+ * x, y: n fp32 device values.
+ */
+sa_status sa_test_exp2_poly(const float *x, float *y, int n, void *stream);
 
 /* Number of key-block ids per row of kv_idx for a given N and bs, i.e. nb = ceil(N / bs). */
 int sa_num_blocks(int N, int bs);

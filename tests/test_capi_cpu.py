@@ -105,18 +105,26 @@ def test_select_argument_checks(lib):
 
 
 def test_attention_argument_checks(lib):
+    lib.sa_attn_workspace_bytes.restype = ctypes.c_size_t
+    W = lib.sa_attn_workspace_bytes()
+    assert 8 <= W <= 4096
     f = lib.sa_block_sparse_attn_fwd
-    f.argtypes = [ctypes.c_void_p] * 6 + [ctypes.c_int] * 5 + [ctypes.c_float, ctypes.c_void_p]
-    assert f(A, A, A, NUL, A, A, 1, 1, 256, 128, 128, 0.0, S) == 1
-    assert f(A, A, A, A, A, A, 1, 1, 256, 256, 128, 0.0, S) == 2
-    assert f(A, A, A, A, A, A, 1, 1, 256, 128, 256, 0.0, S) == 2
-    assert f(A, A, A, A, A, A, 1, 1, 128 * 1025, 128, 128, 0.0, S) == 2
-    assert f(A, A, A, A, A, MIS, 1, 1, 256, 128, 128, 0.0, S) == 1
-    assert f(A, A, A, A, A, A, 1, 1, 256, 128, 128, float("nan"), S) == 1
+    f.argtypes = [ctypes.c_void_p] * 6 + [ctypes.c_int] * 5 + [ctypes.c_float, ctypes.c_void_p,
+                                                                ctypes.c_size_t, ctypes.c_void_p]
+    assert f(A, A, A, NUL, A, A, 1, 1, 256, 128, 128, 0.0, A2, W, S) == 1
+    assert f(A, A, A, A, A, A, 1, 1, 256, 256, 128, 0.0, A2, W, S) == 2
+    assert f(A, A, A, A, A, A, 1, 1, 256, 128, 256, 0.0, A2, W, S) == 2
+    assert f(A, A, A, A, A, A, 1, 1, 128 * 1025, 128, 128, 0.0, A2, W, S) == 2
+    assert f(A, A, A, A, A, MIS, 1, 1, 256, 128, 128, 0.0, A2, W, S) == 1
+    assert f(A, A, A, A, A, A, 1, 1, 256, 128, 128, float("nan"), A2, W, S) == 1
+    assert f(A, A, A, A, A, A, 1, 1, 256, 128, 128, 0.0, NUL, W, S) == 1
+    assert f(A, A, A, A, A, A, 1, 1, 256, 128, 128, 0.0, A2, W - 1, S) == 1
     g = lib.sa_dense_attn_fwd
-    g.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 4 + [ctypes.c_float, ctypes.c_void_p]
-    assert g(A, A, NUL, A, 1, 1, 256, 128, 0.0, S) == 1
-    assert g(A, A, A, A, 1, 1, 256, 32, 0.0, S) == 2
+    g.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 4 + [ctypes.c_float, ctypes.c_void_p,
+                                                                ctypes.c_size_t, ctypes.c_void_p]
+    assert g(A, A, NUL, A, 1, 1, 256, 128, 0.0, A2, W, S) == 1
+    assert g(A, A, A, A, 1, 1, 256, 32, 0.0, A2, W, S) == 2
+    assert g(A, A, A, A, 1, 1, 256, 128, 0.0, NUL, W, S) == 1
 
 
 def test_python_binding_imports():

@@ -242,3 +242,17 @@ def test_host_inputs_roundtrip(orc):
     assert not o.is_cuda
     ref = orc.dense_attention(q[0], k[0], v[0], 1 / 8.0).reshape(N, d)
     compare_attention(bf16_bits_to_f32(o.view(torch.int16).numpy().view(np.uint16))[0, 0], ref)
+
+
+def test_exp2_polynomial_against_cuda_exp2():
+    # the FMA-pipe 2^x of the softmax against CUDA's exp2f, over the range the softmax feeds it
+    # normal results (the exponent-field add does not model subnormals, which bf16 P flushes)
+    x = torch.cat([torch.linspace(-120.0, 8.0, 1_000_001, device=DEV),
+                   torch.rand(1_000_000, device=DEV) * -30.0,
+                   torch.tensor([0.0, -0.5, 0.5, -1.0, 8.0, -119.5], device=DEV)])
+    y = bsa.sparse_attn.exp2_poly(x)
+    ref = torch.exp2(x.double())
+    rel = ((y.double() - ref).abs() / ref).max().item()
+    assert rel < 1e-4, rel
+    tiny = bsa.sparse_attn.exp2_poly(torch.tensor([-float("inf"), -300.0, -125.7], device=DEV))
+    assert (tiny >= 0).all() and tiny.max() < 2e-38
