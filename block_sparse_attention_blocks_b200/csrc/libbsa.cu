@@ -5,3 +5,4 @@
 #include "attn.cu"
 #include "probe.cu"
 #include "capi.cu"
+#include "noalloc.cu"

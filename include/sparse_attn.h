@@ -128,6 +128,28 @@ sa_status sa_dense_attn_fwd(const void *q, const void *k, const void *v, void *o
 /* Bytes of device workspace the attention entry points need (a small constant). */
 size_t sa_attn_workspace_bytes(void);
 
+/*
+ * Block-sparse attention forward for callers that cannot provide device memory beyond their
+ * inputs and outputs (the pages have no counterpart: this is a deployment variant of
+ * sa_block_sparse_attn_fwd).  Some callers cannot lend the library a workspace: their device
+ * memory belongs to another runtime's allocator and they have no spare buffer, or they may not
+ * call cudaMalloc where attention runs because it can synchronise the device.  This entry point
+ * allocates nothing: its scratch (the work counter) lives in a fixed 256-byte array in the
+ * library's device image, which every GPU that loads the library holds until the process exits.
+ * Arguments, layouts and results are those of sa_block_sparse_attn_fwd without the workspace.
+ * - The first call on a device resolves the array's device address (cudaGetSymbolAddress, with
+ *   that device current) and caches it; make that first call before any stream capture.
+ * - Every call shares the one array, which keeps the last call's contents; each call zeroes
+ *   the counter on `stream` before its kernel.  Calls that overlap on the GPU (different
+ *   streams, or several host threads) race on the array and must be serialised by the caller.
+ * - Returns SA_ERR_UNSUPPORTED if the scratch the call needs exceeds the 256-byte array, and the
+ *   errors of sa_block_sparse_attn_fwd otherwise.
+ */
+sa_status sa_block_sparse_attn_fwd_noalloc(const void *q, const void *k, const void *v,
+                                           const int32_t *kv_idx, const int32_t *kv_cnt, void *o,
+                                           int B, int H, int N, int d, int bs, float scale,
+                                           void *stream);
+
 /* Human-readable name of a status code (static storage). */
 const char *sa_get_error_string(sa_status status);
 
