@@ -7,7 +7,7 @@
 // softmax(Qp Kp^T * scale) over pooled blocks.
 //
 // Two launches:
-//   1. block_scores_kernel: fp32 SIMT GEMM L = scale * Qp Kp^T per (b, h), written into the
+//   1. block_scores_kernel: fp32 FFMA GEMM L = scale * Qp Kp^T per (b, h), written into the
 //      kv_idx buffer (same size: nb x nb 32-bit words per head), which doubles as staging.
 //   2. select_rows_kernel: one warp per query-block row.  Softmax in fp32, then the two
 //      prefixes of the ranked order (score descending, id ascending; ranking by score is ranking
@@ -24,57 +24,80 @@ namespace bsa {
 // ------------------------------------------------------------------------------------------
 // 1. block scores
 // ------------------------------------------------------------------------------------------
-constexpr int SC_TILE = 64;
-constexpr int SC_KC = 16;
+constexpr int SC_TILE = 128;  // output tile: 128 query blocks x 128 key blocks of one head
+constexpr int SC_KC = 8;      // reduction chunk
 
+// fp32 FFMA GEMM L = scale * Qp Kp^T for one head, 256 threads, each 8 x 8 outputs (rows
+// ty*4 + {0..3} and 64 + ty*4 + {0..3}, likewise columns), operands staged transposed in shared
+// memory and double buffered.  Each output is an fp32 dot product accumulated in ascending c.
 __global__ void __launch_bounds__(256) block_scores_kernel(const float *__restrict__ qp,
                                                            const float *__restrict__ kp,
                                                            float *__restrict__ logits, int nb,
                                                            int d, float scale) {
-    __shared__ __align__(16) float As[SC_KC][SC_TILE + 4];
-    __shared__ __align__(16) float Bs[SC_KC][SC_TILE + 4];
+    __shared__ __align__(16) float As[2][SC_KC][SC_TILE + 4];
+    __shared__ __align__(16) float Bs[2][SC_KC][SC_TILE + 4];
     const int bh = blockIdx.z;
     const int i0 = blockIdx.y * SC_TILE;
     const int j0 = blockIdx.x * SC_TILE;
     const float *A = qp + (size_t)bh * nb * d;
     const float *Bm = kp + (size_t)bh * nb * d;
     const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-    const int lr = threadIdx.x / 4, lk = (threadIdx.x % 4) * 4;
+    const int lr = threadIdx.x / 2, lk = (threadIdx.x % 2) * 4;  // loader: row, k offset
 
-    float acc[4][4];
+    float acc[8][8];
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+    for (int a = 0; a < 8; ++a)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+        for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
 
-    for (int c0 = 0; c0 < d; c0 += SC_KC) {
-        float4 va = make_float4(0.f, 0.f, 0.f, 0.f), vb = va;
+    auto load = [&](int c0, float4 &va, float4 &vb) {
+        va = make_float4(0.f, 0.f, 0.f, 0.f);
+        vb = va;
         if (i0 + lr < nb) va = *reinterpret_cast<const float4 *>(A + (size_t)(i0 + lr) * d + c0 + lk);
         if (j0 + lr < nb) vb = *reinterpret_cast<const float4 *>(Bm + (size_t)(j0 + lr) * d + c0 + lk);
-        __syncthreads();
-        As[lk + 0][lr] = va.x; As[lk + 1][lr] = va.y; As[lk + 2][lr] = va.z; As[lk + 3][lr] = va.w;
-        Bs[lk + 0][lr] = vb.x; Bs[lk + 1][lr] = vb.y; Bs[lk + 2][lr] = vb.z; Bs[lk + 3][lr] = vb.w;
-        __syncthreads();
+    };
+    auto stash = [&](int buf, const float4 &va, const float4 &vb) {
+        As[buf][lk + 0][lr] = va.x; As[buf][lk + 1][lr] = va.y;
+        As[buf][lk + 2][lr] = va.z; As[buf][lk + 3][lr] = va.w;
+        Bs[buf][lk + 0][lr] = vb.x; Bs[buf][lk + 1][lr] = vb.y;
+        Bs[buf][lk + 2][lr] = vb.z; Bs[buf][lk + 3][lr] = vb.w;
+    };
+
+    float4 va, vb;
+    load(0, va, vb);
+    stash(0, va, vb);
+    __syncthreads();
+    int buf = 0;
+    for (int c0 = 0; c0 < d; c0 += SC_KC) {
+        const bool more = c0 + SC_KC < d;
+        if (more) load(c0 + SC_KC, va, vb);
 #pragma unroll
         for (int kk = 0; kk < SC_KC; ++kk) {
-            const float4 a = *reinterpret_cast<const float4 *>(&As[kk][ty * 4]);
-            const float4 b = *reinterpret_cast<const float4 *>(&Bs[kk][tx * 4]);
-            const float av[4] = {a.x, a.y, a.z, a.w};
-            const float bv[4] = {b.x, b.y, b.z, b.w};
+            const float4 a0 = *reinterpret_cast<const float4 *>(&As[buf][kk][ty * 4]);
+            const float4 a1 = *reinterpret_cast<const float4 *>(&As[buf][kk][64 + ty * 4]);
+            const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[buf][kk][tx * 4]);
+            const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[buf][kk][64 + tx * 4]);
+            const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-            for (int x = 0; x < 4; ++x)
+            for (int x = 0; x < 8; ++x)
 #pragma unroll
-                for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
+                for (int y = 0; y < 8; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
+        }
+        if (more) {
+            stash(buf ^ 1, va, vb);
+            __syncthreads();
+            buf ^= 1;
         }
     }
 #pragma unroll
-    for (int x = 0; x < 4; ++x) {
-        const int i = i0 + ty * 4 + x;
+    for (int x = 0; x < 8; ++x) {
+        const int i = i0 + (x < 4 ? ty * 4 + x : 64 + ty * 4 + x - 4);
         if (i >= nb) continue;
         float *row = logits + ((size_t)bh * nb + i) * nb;
 #pragma unroll
-        for (int y = 0; y < 4; ++y) {
-            const int j = j0 + tx * 4 + y;
+        for (int y = 0; y < 8; ++y) {
+            const int j = j0 + (y < 4 ? tx * 4 + y : 64 + tx * 4 + y - 4);
             if (j < nb) row[j] = acc[x][y] * scale;
         }
     }
@@ -97,10 +120,28 @@ __device__ __forceinline__ float warp_sum(float v) {
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
 }
-__device__ __forceinline__ int warp_isum(int v) {
+
+// The two thresholds by one 32-step bitwise search over EE blocks per lane:
+//   tp = the largest key T with fixed-point mass  sum{P : key >= T} >= pfix,
+//   tk = the largest key T with  #{key >= T} >= kk.
+template <int EE>
+__device__ __forceinline__ void search_thresholds(const uint32_t (&key)[EE], const uint32_t (&pf)[EE],
+                                                  uint32_t pfix, int kk, uint32_t &tp,
+                                                  uint32_t &tk) {
+    tp = 0u;
+    tk = 0u;
+#pragma unroll 1
+    for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t cp = tp | (1u << bit), ck = tk | (1u << bit);
+        uint32_t ms = 0u, c = 0u;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
+        for (int r = 0; r < EE; ++r) {
+            ms += key[r] >= cp ? pf[r] : 0u;
+            c += key[r] >= ck ? 1u : 0u;
+        }
+        if (__reduce_add_sync(0xffffffffu, ms) >= pfix) tp = cp;
+        if ((int)__reduce_add_sync(0xffffffffu, c) >= kk) tk = ck;
+    }
 }
 
 // One warp per query-block row; element e = r*32 + lane (coalesced, index order is r-major).
@@ -108,12 +149,15 @@ __device__ __forceinline__ int warp_isum(int v) {
 // The ranked order is (score descending, block id ascending); key[e] is the score mapped to an
 // order-preserving uint32, so "rank < R" is "key > T, or key == T and among the first few
 // tied ids" for the right threshold T.  Both sets the pages define are prefixes of this order:
-//   top-p: T_p = the largest key value whose mass  sum{P_e : key_e >= T_p} >= p  (bitwise
-//          search, 32 steps, fp32 sums in a fixed order so they are monotone in T); then the
+//   top-p: T_p = the largest key value whose mass  sum{P_e : key_e >= T_p} >= p;  then the
 //          tied blocks at T_p are taken in id order until the mass reaches p;  m = their count
 //          plus the blocks above T_p.
-//   top-k: same search with the count  #{e : key_e >= T} >= k.
-// Their union is the longer prefix, |keep| = max(min(k, nb), m).
+//   top-k: T_k = the largest key value with  #{e : key_e >= T_k} >= k.
+// Both thresholds are found together by one 32-step bitwise search.  Masses are summed in fixed
+// point (round(P * 2^26) in 32 bits), so every warp sum is exact, independent of the order of
+// addition, and one redux.sync instruction; the fixed-point rounding (<= 2^-27 per block, under
+// 8e-6 over a row) stays below the 1e-5 resolution of the cut.  The union is the longer prefix,
+// |keep| = max(min(k, nb), m).
 template <int E>
 __global__ void __launch_bounds__(SEL_WARPS * 32) select_rows_kernel(
     const float *logits, long long rows, int nb, int topk, float topp, uint8_t *__restrict__ mask,
@@ -123,6 +167,7 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) select_rows_kernel(
     if (row >= rows) return;
     const float *lg = logits + (size_t)row * nb;
     const uint32_t lt_mask = (1u << lane) - 1u;
+    constexpr float kFix = 67108864.0f;  // 2^26
 
     float x[E];
 #pragma unroll
@@ -140,100 +185,86 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) select_rows_kernel(
 #pragma unroll
     for (int r = 0; r < E; ++r) z += (r * 32 + lane) < nb ? expf(x[r] - mx) : 0.f;
     z = warp_sum(z);
-    float p[E];
-    uint32_t key[E];
+
+    // per block: order key and fixed-point probability round(P * 2^26) (sums over <= 1024 blocks
+    // stay below 2^32 and differ from the exact sum by at most 1024 * 2^-27 < 8e-6)
+    uint32_t key[E], pf[E];
+    uint32_t tsum = 0u;
 #pragma unroll
     for (int r = 0; r < E; ++r) {
         const bool ok = (r * 32 + lane) < nb;
-        p[r] = ok ? expf(x[r] - mx) / z : 0.f;
+        pf[r] = ok ? __float2uint_rn((expf(x[r] - mx) / z) * kFix) : 0u;
         key[r] = ok ? ord_bits(x[r]) : 0u;
+        tsum += pf[r];
     }
+    const uint32_t total = __reduce_add_sync(0xffffffffu, tsum);
+    const uint32_t pfix = __float2uint_rn(fminf(fmaxf(topp, 0.f), 1.f) * kFix);
+    const int kk = topk < nb ? topk : nb;
+    const bool want_p = topp > 0.f && topp < 1.f && total >= pfix;
+    const bool all_kept = topp >= 1.f || (topp > 0.f && !want_p) || kk >= nb;
 
-    // ---- top-p cut m
-    int m;
-    uint32_t T = 0u;  // final threshold and the number of tied blocks taken at it
-    int take = 0;
-    bool decided = false;
+    // ---- both thresholds, one bitwise search
+    uint32_t tp = 0u, tk = 0u;
+    if (!all_kept) search_thresholds<E>(key, pf, pfix, kk, tp, tk);
+
+    // ---- top-p count m (ties at tp taken in id order until the mass reaches p)
+    int m, ntake = 0;
     if (!(topp > 0.f)) {
         m = 0;
-    } else if (topp >= 1.f) {
-        m = nb;
+    } else if (!want_p) {
+        m = nb;  // p >= 1, or the fixed-point total falls short of p
+    } else if (all_kept) {
+        m = nb;  // k >= nb keeps everything; the top-p cut does not matter
     } else {
-        float tot = 0.f;
+        uint32_t as = 0u, ac = 0u;
 #pragma unroll
-        for (int r = 0; r < E; ++r) tot += p[r];
-        if (!(warp_sum(tot) >= topp)) {
-            m = nb;
-        } else {
-            uint32_t tp = 0u;
-#pragma unroll 1
-            for (int bit = 31; bit >= 0; --bit) {
-                const uint32_t cand = tp | (1u << bit);
-                float ms = 0.f;
+        for (int r = 0; r < E; ++r) {
+            const bool gt = key[r] > tp;
+            as += gt ? pf[r] : 0u;
+            ac += gt ? 1u : 0u;
+        }
+        uint32_t run = __reduce_add_sync(0xffffffffu, as);
+        const int above = (int)__reduce_add_sync(0xffffffffu, ac);
+        int need = 0, ntie = 0;
 #pragma unroll
-                for (int r = 0; r < E; ++r) ms += key[r] >= cand ? p[r] : 0.f;
-                if (warp_sum(ms) >= topp) tp = cand;
-            }
-            int above = 0;
-            float base = 0.f;
-#pragma unroll
-            for (int r = 0; r < E; ++r) {
-                above += key[r] > tp ? 1 : 0;
-                base += key[r] > tp ? p[r] : 0.f;
-            }
-            above = warp_isum(above);
-            base = warp_sum(base);
-            // blocks tied at tp, in id order, until the mass reaches p (at least one)
-            int ntie = 0, need = 0;
-            float run = base;
-#pragma unroll
-            for (int r = 0; r < E; ++r) {
-                const bool tied = key[r] == tp;
-                const uint32_t bal = __ballot_sync(0xffffffffu, tied);
-                float v = tied ? p[r] : 0.f;
+        for (int r = 0; r < E; ++r) {
+            const bool tied = key[r] == tp;
+            const uint32_t bal = __ballot_sync(0xffffffffu, tied);
+            if (bal) {  // warp-uniform; usually a single block
+                uint32_t v = tied ? pf[r] : 0u;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, v, o);
+                    const uint32_t y = __shfl_up_sync(0xffffffffu, v, o);
                     if (lane >= o) v += y;
                 }
-                need += __popc(__ballot_sync(0xffffffffu, tied && run + v < topp));
+                need += __popc(__ballot_sync(0xffffffffu, tied && run + v < pfix));
                 run += __shfl_sync(0xffffffffu, v, 31);
                 ntie += __popc(bal);
             }
-            const int ntake = min(need + 1, ntie);
-            m = above + ntake;
-            T = tp;
-            take = ntake;
-            decided = true;  // valid if the union is the top-p set
         }
+        ntake = min(need + 1, ntie);
+        m = above + ntake;
     }
-    const int kk = min(topk, nb);
     const int keep = max(kk, m);
 
-    if (!(decided && keep == m)) {
-        if (keep >= nb) {
-            T = 0u;  // every valid block (valid keys are > 0, padding is 0)
-            take = 0;
-        } else if (keep <= 0) {
-            T = 0xFFFFFFFFu;
-            take = 0;
-        } else {
-            // the keep-th largest key by count
-            uint32_t tk = 0u;
-#pragma unroll 1
-            for (int bit = 31; bit >= 0; --bit) {
-                const uint32_t cand = tk | (1u << bit);
-                int c = 0;
+    // ---- the kept prefix: key > T, plus the first `take` blocks tied at T
+    uint32_t T;
+    int take;
+    if (keep >= nb) {
+        T = 0u;  // every valid block (valid keys are > 0, padding is 0)
+        take = 0;
+    } else if (keep <= 0) {
+        T = 0xFFFFFFFFu;
+        take = 0;
+    } else if (want_p && m >= kk) {
+        T = tp;
+        take = ntake;
+    } else {
+        uint32_t above = 0u;
 #pragma unroll
-                for (int r = 0; r < E; ++r) c += key[r] >= cand ? 1 : 0;
-                if (warp_isum(c) >= keep) tk = cand;
-            }
-            int above = 0;
-#pragma unroll
-            for (int r = 0; r < E; ++r) above += key[r] > tk ? 1 : 0;
-            T = tk;
-            take = keep - warp_isum(above);
-        }
+        for (int r = 0; r < E; ++r) above += key[r] > tk ? 1u : 0u;
+        T = tk;
+        take = kk - (int)__reduce_add_sync(0xffffffffu, above);
     }
 
     // ---- mark, write the mask row and the ascending id list
