@@ -90,6 +90,50 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, unsign
     mbar_wait(bar, parity, ns, (volatile int *)&never, tag, 0);
 }
 
+// Largest P a block may produce before the reference max of its rows moves.
+constexpr float kMaxP = 1073741824.0f;  // 2^30
+constexpr float kMaxLog2P = 30.f;
+
+// Row max of BS fp32 scores (three-input max, four independent chains).
+template <int BS>
+__device__ __forceinline__ float row_max(const uint32_t (&s)[BS]) {
+    float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+    for (int e = 0; e < BS; e += 2)
+        m4[(e >> 1) & 3] = fmax3f(m4[(e >> 1) & 3], __uint_as_float(s[e]), __uint_as_float(s[e + 1]));
+    return fmax3f(fmaxf(m4[0], m4[1]), m4[2], m4[3]);
+}
+
+// P = 2^(s * sl2 - m) for a row of BS scores: bf16 pairs into pk, returns the row sum.  Three of
+// every four pairs go through the SFU (ex2), one through the FMA-pipe polynomial; bf16 packing
+// runs on the integer pipe.  The SFU gives +inf above 2^128, which the sum shows; the polynomial
+// is only valid below 2^127, so the largest exponent it was given is returned in xpoly.
+template <int BS>
+__device__ __forceinline__ float exp_row(const uint32_t (&s)[BS], float sl2, float m,
+                                         uint32_t (&pk)[BS / 2], float &xpoly) {
+    const float2 sl2v = make_float2(sl2, sl2);
+    const float2 nmv = make_float2(-m, -m);
+    float2 lacc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+    float xp = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < BS; e += 2) {
+        const float2 xv = __ffma2_rn(make_float2(__uint_as_float(s[e]), __uint_as_float(s[e + 1])),
+                                     sl2v, nmv);
+        float2 pv;
+        if ((e & 6) == 6) {
+            pv = exp2_poly2(xv);
+            xp = fmax3f(xp, xv.x, xv.y);
+        } else {
+            pv.x = ex2(xv.x);
+            pv.y = ex2(xv.y);
+        }
+        lacc[(e >> 1) & 1] = __fadd2_rn(lacc[(e >> 1) & 1], pv);
+        pk[e >> 1] = pack_bf16_int(pv.x, pv.y);
+    }
+    xpoly = xp;
+    return (lacc[0].x + lacc[0].y) + (lacc[1].x + lacc[1].y);
+}
+
 template <int D, int BS>
 __global__ void __launch_bounds__(256, 2)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -228,6 +272,13 @@ __global__ void __launch_bounds__(256, 2)
         constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, 0, 1);
         uint32_t nq = 0, nk = 0, nv = 0, np = 0, npv = 0, ned = 0, units_done = 0;
         bool ok = true;
+        // Descriptors of the first 16-column step of each operand; step kk is reached by adding
+        // its byte offset / 16 to the start-address field (shared addresses stay below 2^18, so
+        // the 14-bit field never carries).  Few instructions per MMA matter: this warp shares
+        // its issue slots with softmax warps.
+        const uint64_t dQ = smem_desc_sw128(sQ, 16, 1024);
+        const uint64_t dK = smem_desc_sw128(sK, 16, 1024);
+        const uint64_t dV = smem_desc_sw128(sV, C::KV_CHUNK, 1024);
         for (uint32_t kth = 0; ok; ++kth) {
             const int slot = kth & (UNIT_RING - 1);
             if (!(ok = warp_wait(bar(B_UF0 + slot), (kth / UNIT_RING) & 1, wns, abort_flag, 0x27, kth)))
@@ -253,10 +304,10 @@ __global__ void __launch_bounds__(256, 2)
                 if (lane == 0) {
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk & 3) * 32;  // K step inside the 128-byte swizzled row
-                        const uint64_t a = smem_desc_sw128(sQ + (kk >> 2) * C::Q_CHUNK + off, 16, 1024);
-                        const uint64_t b = smem_desc_sw128(sK + (kk >> 2) * C::KV_CHUNK + off, 16, 1024);
-                        mma_ss(tS, a, b, IDESC_S, kk > 0 ? 1u : 0u);
+                        // K step kk: 32 bytes inside the 128-byte swizzled row, then the next chunk
+                        const uint64_t oq = (uint64_t)(((kk >> 2) * C::Q_CHUNK + (kk & 3) * 32) >> 4);
+                        const uint64_t ok = (uint64_t)(((kk >> 2) * C::KV_CHUNK + (kk & 3) * 32) >> 4);
+                        mma_ss(tS, dQ + oq, dK + ok, IDESC_S, kk > 0 ? 1u : 0u);
                     }
                     mma_commit(bar(B_SF));
                     mma_commit(bar(B_KE));
@@ -280,8 +331,9 @@ __global__ void __launch_bounds__(256, 2)
                 if (lane == 0) {
 #pragma unroll
                     for (int kk = 0; kk < BS / 16; ++kk) {
-                        const uint64_t b = smem_desc_sw128(sV + kk * 2048, C::KV_CHUNK, 1024);
-                        mma_ts(tO, tS + kk * 8, b, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+                        // 16 keys = 16 rows of 128 bytes
+                        mma_ts(tO, tS + kk * 8, dV + (uint64_t)((kk * 2048) >> 4), IDESC_PV,
+                               (t > 0 || kk > 0) ? 1u : 0u);
                     }
                     mma_commit(bar(B_VE));
                     mma_commit(bar(B_OD));
@@ -334,7 +386,7 @@ __global__ void __launch_bounds__(256, 2)
                 continue;
             }
             const int32_t *list = dense ? nullptr : prm.kv_idx + (size_t)u * prm.nbk;
-            float m_ref = -INFINITY;  // running max, log2 domain
+            float m_ref = 0.f;        // reference max, log2 domain (set by the first block)
             float l = 0.f;            // running sum
             int jn = dense ? 0 : list[0];
             for (int t = 0; t < cnt; ++t) {
@@ -353,22 +405,26 @@ __global__ void __launch_bounds__(256, 2)
                     for (int e = 0; e < BS; ++e)
                         if (e >= valid) s[e] = __float_as_uint(-INFINITY);
                 }
-                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                // Reference max: the first block of a query block sets it from its own scores.
+                // Later blocks reuse it while their P stays below 2^30 (bf16 and the fp32 sums
+                // have room for that), which the block's row sum shows, so the row max is not
+                // needed per block.  A block that overflows moves the reference to its max,
+                // rescales O and l, and is exponentiated again.
+                if (t == 0) m_ref = row_max<BS>(s) * sl2;
+                uint32_t pk[BS / 2];
+                float xpoly;
+                float ts = exp_row<BS>(s, sl2, m_ref, pk, xpoly);
+                // warp-uniform (tcgen05.ld/st are .sync.aligned); a NaN sum also overflows
+                if (__any_sync(0xffffffffu, !(ts < kMaxP) || xpoly > kMaxLog2P)) {
+                    // rare: S is read again from tensor memory (still intact: P is written below)
+                    tmem_ld_cols<BS>(tSr, s);
+                    if (valid < BS) {
 #pragma unroll
-                for (int e = 0; e < BS; e += 2)
-                    m4[(e >> 1) & 3] = fmax3f(m4[(e >> 1) & 3], __uint_as_float(s[e]),
-                                              __uint_as_float(s[e + 1]));
-                const float mx = fmax3f(fmaxf(m4[0], m4[1]), m4[2], m4[3]);
-                report(prm.progress, 4 + q4, 2, t, u);
-                const float mxs = mx * sl2;
-                // Lazy rescale: a row moves its reference max only when the block max exceeds it
-                // by more than 2^8.  The decision is taken per warp (tcgen05.ld/st are
-                // .sync.aligned, so the whole warp must execute them); each lane scales by its
-                // own alpha, 1 for rows that keep their reference, 0 on the first block.
-                const bool grow = mxs > m_ref + 8.f;
-                if (__any_sync(0xffffffffu, grow)) {
-                    const float m_new = grow ? mxs : m_ref;
-                    const float alpha = ex2(m_ref - m_new);
+                        for (int e = 0; e < BS; ++e)
+                            if (e >= valid) s[e] = __float_as_uint(-INFINITY);
+                    }
+                    const float m_new = fmaxf(m_ref, row_max<BS>(s) * sl2);
+                    const float alpha = ex2(m_ref - m_new);  // 1 for rows that keep theirs
                     if (t > 0) {
                         // the previous P V is complete: this S was issued after it, in order
 #pragma unroll 1
@@ -383,30 +439,9 @@ __global__ void __launch_bounds__(256, 2)
                     }
                     l *= alpha;
                     m_ref = m_new;
+                    ts = exp_row<BS>(s, sl2, m_ref, pk, xpoly);  // now every P <= 1
                 }
-                // P = 2^(s*scale*log2e - m), packed bf16 pairs written over the consumed S columns.
-                // Three of every four pairs go through the SFU (ex2), one through the FMA-pipe
-                // polynomial, so that neither pipe limits the softmax; bf16 packing runs on the
-                // integer pipe.
-                const float2 sl2v = make_float2(sl2, sl2);
-                const float2 nmv = make_float2(-m_ref, -m_ref);
-                float2 lacc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-                uint32_t pk[BS / 2];
-#pragma unroll
-                for (int e = 0; e < BS; e += 2) {
-                    const float2 xv = __ffma2_rn(
-                        make_float2(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), sl2v, nmv);
-                    float2 pv;
-                    if ((e & 6) == 6) {
-                        pv = exp2_poly2(xv);
-                    } else {
-                        pv.x = ex2(xv.x);
-                        pv.y = ex2(xv.y);
-                    }
-                    lacc[(e >> 1) & 1] = __fadd2_rn(lacc[(e >> 1) & 1], pv);
-                    pk[e >> 1] = pack_bf16_int(pv.x, pv.y);
-                }
-                l += (lacc[0].x + lacc[0].y) + (lacc[1].x + lacc[1].y);
+                l += ts;
 #pragma unroll
                 for (int c = 0; c < BS / 64; ++c)
                     tmem_st32(tSr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[c * 32]));
