@@ -54,6 +54,11 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def launches_per_step(bh: int) -> int:
+    """Kernels of one step: pooling, block scores, row selection, attention."""
+    return 4
+
+
 def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -302,17 +307,16 @@ def run_gpu(args, w):
     stream = torch.cuda.current_stream(dev)
 
     def step(ev=None):
+        # pooling and selection in one call, then attention
         if ev is not None:
             ev[0].record(stream)
-        bsa.pool_blocks(q, k, bs, qp=qp, kp=kp)
+        bsa.pool_select_topk_topp(q, k, bs, w.topk, w.topp, qp=qp, kp=kp, mask=mask,
+                                  kv_idx=kv_idx, kv_cnt=kv_cnt)
         if ev is not None:
             ev[1].record(stream)
-        bsa.select_mask_topk_topp(qp, kp, w.topk, w.topp, mask=mask, kv_idx=kv_idx, kv_cnt=kv_cnt)
-        if ev is not None:
-            ev[2].record(stream)
         bsa.block_sparse_attn_fwd(q, k, v, kv_idx, kv_cnt, bs, o=o)
         if ev is not None:
-            ev[3].record(stream)
+            ev[2].record(stream)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -324,7 +328,7 @@ def run_gpu(args, w):
     density = pairs / float(B * H * nb * nb)
 
     # ---------------------------------------------------------------- timed region
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
     if world > 1:
@@ -341,9 +345,8 @@ def run_gpu(args, w):
     if world > 1:
         torch.distributed.barrier()
     ms_total = start.elapsed_time(end)
-    t_pool = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
-    t_sel = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
-    t_att = float(np.mean([e[2].elapsed_time(e[3]) for e in evs]))
+    t_ps = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    t_att = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
     ms_total = max_over_ranks(ms_total, dev)
     ms_step = ms_total / args.steps
     err = bsa.device_error()
@@ -408,7 +411,7 @@ def run_gpu(args, w):
     ps_bytes = (2 * q.numel() * 2 + 2 * qp.numel() * 4            # pool: read Q,K, write Qp,Kp
                 + 2 * qp.numel() * 4 + mask.numel()                 # select: read Qp,Kp, mask
                 + 4 * (kv_cnt.numel() + pairs))                     # kv_cnt + kept ids
-    ps_gbs = ps_bytes / ((t_pool + t_sel) * 1e-3) / 1e9
+    ps_gbs = ps_bytes / (t_ps * 1e-3) / 1e9
     line = {
         "metric": METRIC,
         "value": world * flops / (ms_step * 1e-3) / 1e12,
@@ -432,9 +435,11 @@ def run_gpu(args, w):
         "roofline_pool_select": {"bound": "hbm", "achieved": ps_gbs, "peak": peak_hbm,
                                  "unit": "GB/s", "frac": ps_gbs / peak_hbm,
                                  "bytes_per_call": ps_bytes,
+                                 "timed": "sa_pool_select_topk_topp: pooling, block scores "
+                                          "and row selection kernels",
                                  "peak_source": f"hbm_gbs of {peak_src}"},
-        "kernels_ms": {"pool": t_pool, "select": t_sel, "attention": t_att},
-        "gpu_launches": 4 * args.steps,
+        "kernels_ms": {"pool_select": t_ps, "attention": t_att},
+        "gpu_launches": launches_per_step(B * H) * args.steps,
         "clocks": clk,
     }
     if e2e:

@@ -5,4 +5,5 @@
 #include "attn.cu"
 #include "probe.cu"
 #include "capi.cu"
+#include "pipeline.cu"
 #include "noalloc.cu"

@@ -29,6 +29,8 @@ _F = ctypes.c_float
 lib.sa_pool_blocks.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]
 lib.sa_select_mask_topk_topp.argtypes = [_P, _P, _I, _I, _I, _I, _I, _F, _F, _P, _P, _P, _P]
 lib.sa_select_from_logits.argtypes = [_P, _I, _I, _I, _I, _F, _P, _P, _P, _P]
+lib.sa_pool_select_topk_topp.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _F, _P, _P,
+                                         _P, _P]
 _Z = ctypes.c_size_t
 lib.sa_block_sparse_attn_fwd.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _Z, _P]
 lib.sa_dense_attn_fwd.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _Z, _P]
@@ -41,6 +43,7 @@ lib.sa_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
 lib.sa_probe_bounded_wait.argtypes = [_P]
 lib.sa_num_blocks.argtypes = [_I, _I]
 for _f in (lib.sa_pool_blocks, lib.sa_select_mask_topk_topp, lib.sa_select_from_logits,
+           lib.sa_pool_select_topk_topp,
            lib.sa_block_sparse_attn_fwd, lib.sa_dense_attn_fwd, lib.sa_get_device_error,
            lib.sa_set_wait_limit_ns, lib.sa_probe_bounded_wait, lib.sa_num_blocks):
     _f.restype = _I
@@ -149,6 +152,26 @@ def select_mask_topk_topp(qp, kp, topk: int, topp: float, scale: float | None = 
     return mask, kv_idx, kv_cnt
 
 
+def pool_select_topk_topp(q, k, bs: int, topk: int, topp: float, scale: float | None = None,
+                          qp=None, kp=None, mask=None, kv_idx=None, kv_cnt=None):
+    """Pooling and selection in one call (selection overlapped with pooling) ->
+    (qp, kp, mask, kv_idx, kv_cnt), the same values pool_blocks + select_mask_topk_topp give."""
+    for n, t in (("q", q), ("k", k)):
+        _need(t, n, torch.bfloat16, 4)
+    B, H, N, d = q.shape
+    nb = num_blocks(N, bs)
+    qp = qp if qp is not None else torch.empty(B, H, nb, d, dtype=torch.float32, device=q.device)
+    kp = kp if kp is not None else torch.empty(B, H, nb, d, dtype=torch.float32, device=q.device)
+    _need(qp, "qp", torch.float32, 4)
+    _need(kp, "kp", torch.float32, 4)
+    mask, kv_idx, kv_cnt = _sel_outputs(B, H, nb, q.device, mask, kv_idx, kv_cnt)
+    _check(lib.sa_pool_select_topk_topp(_ptr(q), _ptr(k), _ptr(qp), _ptr(kp), B, H, N, d, bs,
+                                        int(topk), float(topp), float(scale or 0.0), _ptr(mask),
+                                        _ptr(kv_idx), _ptr(kv_cnt), _stream(q.device)),
+           "sa_pool_select_topk_topp")
+    return qp, kp, mask, kv_idx, kv_cnt
+
+
 def select_from_logits(logits, topk: int, topp: float, mask=None, kv_idx=None, kv_cnt=None):
     """Selection from given block scores [B, H, nb, nb] fp32 -> (mask, kv_idx, kv_cnt)."""
     _need(logits, "logits", torch.float32, 4)
@@ -203,8 +226,7 @@ def sparse_attention(q, k, v, bs: int, topk: int, topp: float, scale: float | No
         dev = torch.device(device) if device is not None else torch.device("cuda",
                                                                            torch.cuda.current_device())
         q, k, v = (t.to(dev, non_blocking=True) for t in (q, k, v))
-    qp, kp = pool_blocks(q, k, bs)
-    mask, kv_idx, kv_cnt = select_mask_topk_topp(qp, kp, topk, topp, scale)
+    _, _, mask, kv_idx, kv_cnt = pool_select_topk_topp(q, k, bs, topk, topp, scale)
     o = block_sparse_attn_fwd(q, k, v, kv_idx, kv_cnt, bs, scale)
     if on_host:
         o = o.to("cpu")

@@ -91,6 +91,14 @@ sa_status sa_select_mask_topk_topp(const float *qp, const float *kp, int B, int 
                                    int32_t *kv_idx, int32_t *kv_cnt, void *stream);
 
 /*
+ * Pooling and selection in one call: sa_pool_blocks followed by sa_select_mask_topk_topp (same
+ * arguments, same outputs, bit for bit), all on `stream`.  Needs nb <= 1024.
+ */
+sa_status sa_pool_select_topk_topp(const void *q, const void *k, float *qp, float *kp, int B,
+                                   int H, int N, int d, int bs, int topk, float topp, float scale,
+                                   uint8_t *mask, int32_t *kv_idx, int32_t *kv_cnt, void *stream);
+
+/*
  * Selection from caller-provided block scores (the second half of sa_select_mask_topk_topp,
  * exposed for tests that feed hand-made rows).  logits: [B, H, nb, nb] fp32 scores already
  * scaled; the row softmax, ranking, top-k union top-p and outputs are as above.  logits may be

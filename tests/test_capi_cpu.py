@@ -30,6 +30,7 @@ def _declared():
 def test_header_declares_the_path():
     names = _declared()
     for required in ("sa_pool_blocks", "sa_select_mask_topk_topp", "sa_block_sparse_attn_fwd",
+                     "sa_pool_select_topk_topp",
                      "sa_dense_attn_fwd", "sa_get_error_string", "sa_get_device_error",
                      "sa_select_from_logits"):
         assert required in names
@@ -102,6 +103,28 @@ def test_select_argument_checks(lib):
     assert g(NUL, 1, 1, 16, 2, 0.5, A, A, A, S) == 1
     assert g(A, 1, 1, 2000, 2, 0.5, A, A, A, S) == 2
     assert g(A, 1, 1, 16, 2, 2.0, A, A, A, S) == 1
+
+
+def test_pool_select_argument_checks(lib):
+    f = lib.sa_pool_select_topk_topp
+    f.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 6 + [ctypes.c_float] * 2 + \
+        [ctypes.c_void_p] * 4
+    ok = dict(B=1, H=1, N=256, d=128, bs=128, k=2, p=0.5, s=0.0)
+
+    def call(q=A, qp=A2, idx=A, **kw):
+        a = {**ok, **kw}
+        return f(q, A, qp, A2, a["B"], a["H"], a["N"], a["d"], a["bs"], a["k"], a["p"], a["s"],
+                 A, idx, A2, S)
+
+    assert call(q=NUL) == 1
+    assert call(k=-1) == 1
+    assert call(p=1.5) == 1
+    assert call(s=float("nan")) == 1
+    assert call(d=96) == 2
+    assert call(bs=32) == 2
+    assert call(N=128 * 1025) == 2
+    assert call(qp=MIS) == 1
+    assert call(idx=MIS) == 1
 
 
 def test_attention_argument_checks(lib):

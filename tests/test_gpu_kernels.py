@@ -233,6 +233,28 @@ def test_full_path_small(orc):
     compare_attention(got, ref)
 
 
+@pytest.mark.parametrize("B,H,N,d,bs", [(1, 3, 1500, 128, 128), (2, 11, 777, 64, 64),
+                                          (1, 1, 200, 128, 128)])
+def test_pool_select_fused_equals_separate_calls(B, H, N, d, bs):
+    # the one-call path must give the separate calls' results bit for bit
+    rng = np.random.default_rng(15)
+    q = to_dev_bf16(rand_bits(rng, (B, H, N, d), 1.0))
+    k = to_dev_bf16(rand_bits(rng, (B, H, N, d), 1.0))
+    topk, topp = 3, 0.7
+    qp, kp = bsa.pool_blocks(q, k, bs)
+    mask, idx, cnt = bsa.select_mask_topk_topp(qp, kp, topk, topp)
+    qp2, kp2, mask2, idx2, cnt2 = bsa.pool_select_topk_topp(q, k, bs, topk, topp)
+    torch.cuda.synchronize()
+    assert torch.equal(qp, qp2) and torch.equal(kp, kp2)
+    assert torch.equal(mask, mask2) and torch.equal(cnt, cnt2)
+    nb = cnt.shape[-1]
+    c = cnt.reshape(-1).cpu().numpy()
+    a1 = idx.reshape(-1, nb).cpu().numpy()
+    a2 = idx2.reshape(-1, nb).cpu().numpy()
+    for r in range(a1.shape[0]):
+        assert np.array_equal(a1[r, :c[r]], a2[r, :c[r]])
+
+
 def test_host_inputs_roundtrip(orc):
     rng = np.random.default_rng(14)
     B, H, N, d, bs = 1, 1, 600, 64, 128
