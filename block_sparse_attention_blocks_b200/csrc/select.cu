@@ -121,26 +121,61 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-// The two thresholds by one 32-step bitwise search over EE blocks per lane:
+// The two thresholds by one bitwise search (bit 31 down to 0) over EE blocks per lane:
 //   tp = the largest key T with fixed-point mass  sum{P : key >= T} >= pfix,
 //   tk = the largest key T with  #{key >= T} >= kk.
+// Each search keeps the invariant that its current threshold satisfies its condition, and stops
+// as soon as the answer is known:
+//   top-k: once exactly kk keys are >= tk, the answer is the least of them;
+//   top-p: once the mass of the keys above m (m the least key >= tp) falls short of pfix, the
+//          answer is m (checked every fourth bit, and at the end).
+// A search that is not wanted (do_p / do_k false) is skipped.
 template <int EE>
 __device__ __forceinline__ void search_thresholds(const uint32_t (&key)[EE], const uint32_t (&pf)[EE],
-                                                  uint32_t pfix, int kk, uint32_t &tp,
-                                                  uint32_t &tk) {
+                                                  uint32_t pfix, int kk, bool do_p, bool do_k,
+                                                  uint32_t &tp, uint32_t &tk) {
     tp = 0u;
     tk = 0u;
+    bool dp = !do_p, dk = !do_k;
 #pragma unroll 1
-    for (int bit = 31; bit >= 0; --bit) {
-        const uint32_t cp = tp | (1u << bit), ck = tk | (1u << bit);
-        uint32_t ms = 0u, c = 0u;
+    for (int bit = 31; bit >= 0 && !(dp && dk); --bit) {
+        if (!dp) {
+            const uint32_t cp = tp | (1u << bit);
+            uint32_t ms = 0u;
 #pragma unroll
-        for (int r = 0; r < EE; ++r) {
-            ms += key[r] >= cp ? pf[r] : 0u;
-            c += key[r] >= ck ? 1u : 0u;
+            for (int r = 0; r < EE; ++r) ms += key[r] >= cp ? pf[r] : 0u;
+            if (__reduce_add_sync(0xffffffffu, ms) >= pfix) tp = cp;
+            if ((bit & 3) == 0) {
+                uint32_t lo = 0xFFFFFFFFu;
+#pragma unroll
+                for (int r = 0; r < EE; ++r) lo = key[r] >= tp ? min(lo, key[r]) : lo;
+                const uint32_t m = __reduce_min_sync(0xffffffffu, lo);
+                uint32_t above = 0u;
+#pragma unroll
+                for (int r = 0; r < EE; ++r) above += key[r] > m ? pf[r] : 0u;
+                if (__reduce_add_sync(0xffffffffu, above) < pfix) {
+                    tp = m;
+                    dp = true;
+                }
+            }
         }
-        if (__reduce_add_sync(0xffffffffu, ms) >= pfix) tp = cp;
-        if ((int)__reduce_add_sync(0xffffffffu, c) >= kk) tk = ck;
+        if (!dk) {
+            const uint32_t ck = tk | (1u << bit);
+            uint32_t c = 0u;
+#pragma unroll
+            for (int r = 0; r < EE; ++r) c += key[r] >= ck ? 1u : 0u;
+            const int cc = (int)__reduce_add_sync(0xffffffffu, c);
+            if (cc >= kk) {
+                tk = ck;
+                if (cc == kk) {
+                    uint32_t lo = 0xFFFFFFFFu;
+#pragma unroll
+                    for (int r = 0; r < EE; ++r) lo = key[r] >= tk ? min(lo, key[r]) : lo;
+                    tk = __reduce_min_sync(0xffffffffu, lo);
+                    dk = true;
+                }
+            }
+        }
     }
 }
 
@@ -153,7 +188,7 @@ __device__ __forceinline__ void search_thresholds(const uint32_t (&key)[EE], con
 //          tied blocks at T_p are taken in id order until the mass reaches p;  m = their count
 //          plus the blocks above T_p.
 //   top-k: T_k = the largest key value with  #{e : key_e >= T_k} >= k.
-// Both thresholds are found together by one 32-step bitwise search.  Masses are summed in fixed
+// Both thresholds are found together by one bitwise search that stops early.  Masses are summed in fixed
 // point (round(P * 2^26) in 32 bits), so every warp sum is exact, independent of the order of
 // addition, and one redux.sync instruction; the fixed-point rounding (<= 2^-27 per block, under
 // 8e-6 over a row) stays below the 1e-5 resolution of the cut.  The union is the longer prefix,
@@ -181,20 +216,23 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) select_rows_kernel(
     for (int r = 0; r < E; ++r) mx = fmaxf(mx, x[r]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float z = 0.f;
-#pragma unroll
-    for (int r = 0; r < E; ++r) z += (r * 32 + lane) < nb ? expf(x[r] - mx) : 0.f;
-    z = warp_sum(z);
-
-    // per block: order key and fixed-point probability round(P * 2^26) (sums over <= 1024 blocks
-    // stay below 2^32 and differ from the exact sum by at most 1024 * 2^-27 < 8e-6)
+    // per block: order key, exp(x - max), then the fixed-point probability round(P * 2^26) (sums
+    // over <= 1024 blocks stay below 2^32 and differ from the exact sum by < 8e-6)
     uint32_t key[E], pf[E];
-    uint32_t tsum = 0u;
+    float z = 0.f;
 #pragma unroll
     for (int r = 0; r < E; ++r) {
         const bool ok = (r * 32 + lane) < nb;
-        pf[r] = ok ? __float2uint_rn((expf(x[r] - mx) / z) * kFix) : 0u;
         key[r] = ok ? ord_bits(x[r]) : 0u;
+        x[r] = ok ? expf(x[r] - mx) : 0.f;
+        z += x[r];
+    }
+    z = warp_sum(z);
+    const float to_fix = kFix / z;
+    uint32_t tsum = 0u;
+#pragma unroll
+    for (int r = 0; r < E; ++r) {
+        pf[r] = __float2uint_rn(x[r] * to_fix);
         tsum += pf[r];
     }
     const uint32_t total = __reduce_add_sync(0xffffffffu, tsum);
@@ -203,9 +241,9 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) select_rows_kernel(
     const bool want_p = topp > 0.f && topp < 1.f && total >= pfix;
     const bool all_kept = topp >= 1.f || (topp > 0.f && !want_p) || kk >= nb;
 
-    // ---- both thresholds, one bitwise search
+    // ---- both thresholds, one bitwise search (top-k only matters when k > 0)
     uint32_t tp = 0u, tk = 0u;
-    if (!all_kept) search_thresholds<E>(key, pf, pfix, kk, tp, tk);
+    if (!all_kept) search_thresholds<E>(key, pf, pfix, kk, want_p, kk > 0, tp, tk);
 
     // ---- top-p count m (ties at tp taken in id order until the mass reaches p)
     int m, ntake = 0;
