@@ -54,6 +54,38 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fwd_kernel_wan14b_720p_traffic.txt")
+KERNEL_SOURCES = ("block_sparse_attention_blocks_b200/csrc/attn.cu",
+                  "block_sparse_attention_blocks_b200/csrc/ptx.cuh")
+
+
+def attention_traffic(workload: str, heads: int, pairs: int):
+    """DRAM bytes (read + write) of one attention launch from the committed ncu capture, or None
+    when the kernel sources changed since the capture or the workload is not the captured one."""
+    import hashlib
+
+    try:
+        fields = {}
+        with open(TRAFFIC_FILE) as f:
+            for line in f:
+                if line.startswith("#") or ":" not in line:
+                    continue
+                k, v = line.split(":", 1)
+                fields[k.strip()] = v.strip()
+        h = hashlib.sha256()
+        for rel in KERNEL_SOURCES:
+            with open(os.path.join(ROOT, rel), "rb") as f:
+                h.update(f.read())
+    except OSError:
+        return None
+    if fields.get("source_sha256") != h.hexdigest():
+        return None
+    if not fields.get("workload", "").startswith(workload + " ") or f"({pairs} executed" not in \
+            fields.get("workload", "") or heads != 40:
+        return None
+    return int(fields["dram_bytes_read"]) + int(fields["dram_bytes_write"])
+
+
 def launches_per_step(bh: int) -> int:
     """Kernels of one step: pooling, block scores, row selection, attention."""
     return 4
@@ -427,7 +459,11 @@ def run_gpu(args, w):
                                   "effective_flops_per_call": flops}),
         "roofline": {"kernel": "attn_fwd_kernel<128,128>", "bound": "tensor",
                      "achieved": att_tflops, "peak": peak_tc, "unit": "TFLOP/s",
-                     "frac": att_tflops / peak_tc, "traffic": None,
+                     "frac": att_tflops / peak_tc,
+                     "traffic": attention_traffic(w.name, B * H, pairs),
+                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one "
+                                       "full-size launch (profiles/attn_fwd_kernel_wan14b_720p_"
+                                       "traffic.txt); null when the kernel changed since",
                      "peak_source": f"bf16_tflops_sustained of {peak_src}",
                      "frac_of_burst_peak": att_tflops / peaks.get("bf16_tflops", peak_tc),
                      "algorithmic": "4*d*rows*cols per executed (query block, key block) pair, "
