@@ -158,8 +158,8 @@ sa_status sa_select_mask_topk_topp(const float *qp, const float *kp, int B, int 
     if (!select_device(kv_idx, &dev)) return SA_ERR_INVALID_ARG;
     const long long BH = (long long)B * H;
     float *logits = reinterpret_cast<float *>(kv_idx);  // staging: same size, row-owned
-    cudaError_t e = bsa::block_scores(qp, kp, logits, BH, nb, d, resolve_scale(scale, d),
-                                      (cudaStream_t)stream);
+    cudaError_t e = bsa::block_scores_tc(qp, kp, logits, BH, nb, d, resolve_scale(scale, d),
+                                         g_wait_ns, (cudaStream_t)stream);
     if (e != cudaSuccess) return SA_ERR_CUDA;
     return from_cuda(bsa::select_rows(logits, BH * nb, nb, topk, topp, mask, kv_idx, kv_cnt,
                                       (cudaStream_t)stream));

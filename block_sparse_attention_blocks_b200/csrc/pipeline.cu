@@ -22,7 +22,8 @@ extern "C" sa_status sa_pool_select_topk_topp(const void *q, const void *k, floa
     const long long BH = (long long)B * H;
     cudaError_t e = bsa::pool_blocks(q, k, qp, kp, BH, N, d, bs, st);
     float *logits = reinterpret_cast<float *>(kv_idx);  // staging: same size, row-owned
-    if (e == cudaSuccess) e = bsa::block_scores(qp, kp, logits, BH, nb, d, resolve_scale(scale, d), st);
+    if (e == cudaSuccess)
+        e = bsa::block_scores_tc(qp, kp, logits, BH, nb, d, resolve_scale(scale, d), g_wait_ns, st);
     if (e == cudaSuccess) e = bsa::select_rows(logits, BH * nb, nb, topk, topp, mask, kv_idx, kv_cnt, st);
     return from_cuda(e);
 }

@@ -103,6 +103,168 @@ __global__ void __launch_bounds__(256) block_scores_kernel(const float *__restri
     }
 }
 
+// Tensor-core form of the same scores.  Each fp32 operand x is split exactly into three bf16
+// parts, x = h + m + l: h keeps the sign, exponent and top 7 fraction bits of x (the low 16 bits
+// cleared), m the same of x - h, and l = x - h - m, which has at most 8 significant bits left
+// (each difference is exact in fp32).  The dot product is the sum of the six part products whose
+// weight is at least 2^-16 relative (l.h, m.m, h.l, m.h, h.m, h.h, smallest first), each a
+// tcgen05.mma.kind::f16 accumulating in one fp32 tensor-memory tile.  The products of bf16 parts
+// are exact in fp32, so the result differs from the fp32 FFMA dot product by accumulation
+// rounding of the same order.  One CTA computes one 128 x 128 tile (128 query blocks x 128 key
+// blocks of one head) in 64-channel chunks: 256 threads load a chunk of both fp32 row tiles
+// (coalesced), split it into the six bf16 tiles in shared memory (the 128-byte swizzled K-major
+// layout the MMA descriptor reads), and thread 0 issues the 6 x 4 MMAs of the chunk; the finished tile goes
+// through shared memory to coalesced row stores.  96 KB of shared memory, two CTAs per SM, so one
+// CTA's loads and stores overlap the other's MMAs.
+constexpr int TC_ROWS = 128;
+
+struct ScoresTcCfg {
+    static constexpr int PART = TC_ROWS * 128;        // one bf16 tile: 128 rows x 64 channels
+    static constexpr int OFF_Q = 0;                   // 3 parts of the query-block chunk
+    static constexpr int OFF_K = 3 * PART;            // 3 parts of the key-block chunk
+    static constexpr int OFF_BAR = 6 * PART;          // mbarrier, TMEM address
+    static constexpr int OUT_LD = TC_ROWS + 4;        // padded fp32 row of the output staging
+    static_assert(TC_ROWS * OUT_LD * 4 <= 6 * PART, "output staging must fit in the operands");
+    static constexpr int SMEM = OFF_BAR + 16 + 1024;  // + alignment slack
+};
+
+// 8-byte shared-memory store through a shared-window address
+__device__ __forceinline__ void st_shared_v2(uint32_t addr, uint32_t a, uint32_t b) {
+    asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
+}
+
+// byte offset of element (row, col) of a 128-row x 64-column bf16 tile in the 128-byte swizzled
+// layout: the 16-byte unit u = col / 8 of a row is stored at unit u ^ (row % 8)
+__device__ __forceinline__ uint32_t sw128_offset(int row, int col) {
+    return (uint32_t)(row * 128 + ((((col >> 3) ^ row) & 7) << 4));
+}
+
+template <int D>
+__global__ void __launch_bounds__(256, 2) block_scores_tc_kernel(const float *__restrict__ qp,
+                                                                 const float *__restrict__ kp,
+                                                                 float *__restrict__ logits,
+                                                                 int nb, float scale,
+                                                                 unsigned long long wait_ns) {
+    using C = ScoresTcCfg;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_BAR + 8);
+    const int bh = blockIdx.z, i0 = blockIdx.y * TC_ROWS, j0 = blockIdx.x * TC_ROWS;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    if (tid == 0) {
+        mbar_init(smem_u32(bar), 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(tmem_holder), 128);
+        tmem_relinquish();
+    }
+    int never = 0;
+    bool done = true;
+    uint32_t tmem = 0;
+    constexpr uint32_t IDESC = idesc_bf16_f32(128, 128, 0, 0);
+
+#pragma unroll 1
+    for (int dc = 0; dc < D / 64; ++dc) {
+        // 128 rows x 64 channels of each operand: float4 f = v * 256 + tid is row f / 16,
+        // channels 4 (f % 16) .. + 3, so 16 lanes read one row's 256 contiguous bytes; every
+        // load of the chunk is issued before any store
+        float4 xq[8], xk[8];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+            const int f = v * 256 + tid, row = f >> 4, ch = dc * 64 + (f & 15) * 4;
+            const int gi = i0 + row, gj = j0 + row;
+            xq[v] = gi < nb ? *reinterpret_cast<const float4 *>(qp + ((size_t)bh * nb + gi) * D + ch)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+            xk[v] = gj < nb ? *reinterpret_cast<const float4 *>(kp + ((size_t)bh * nb + gj) * D + ch)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        if (dc > 0) {
+            // the previous chunk's MMAs must have read the parts before they are overwritten
+            done = done && mbar_wait(smem_u32(bar), (dc - 1) & 1, wait_ns, (volatile int *)&never, 0x51, 0);
+        }
+        // 4 channels -> 8 bytes of each bf16 part, half of a swizzled 16-byte unit
+        auto stash = [&](const float4 (&x)[8], uint32_t base) {
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+                const int f = v * 256 + tid, row = f >> 4, col = (f & 15) * 4;
+                const float xv[4] = {x[v].x, x[v].y, x[v].z, x[v].w};
+                uint32_t hb[4], mb[4], lb[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    hb[q] = __float_as_uint(xv[q]) & 0xFFFF0000u;
+                    const float rm = xv[q] - __uint_as_float(hb[q]);  // exact
+                    mb[q] = __float_as_uint(rm) & 0xFFFF0000u;
+                    lb[q] = __float_as_uint(rm - __uint_as_float(mb[q]));  // exact, low half zero
+                }
+                // the high halves of two words are the bf16 parts, the lower channel in the low half
+                const uint32_t off = smem_u32(smem) + base + sw128_offset(row, col) + (col & 4) * 2;
+                st_shared_v2(off, __byte_perm(hb[0], hb[1], 0x7632), __byte_perm(hb[2], hb[3], 0x7632));
+                st_shared_v2(off + C::PART, __byte_perm(mb[0], mb[1], 0x7632), __byte_perm(mb[2], mb[3], 0x7632));
+                st_shared_v2(off + 2 * C::PART, __byte_perm(lb[0], lb[1], 0x7632), __byte_perm(lb[2], lb[3], 0x7632));
+            }
+        };
+        stash(xq, C::OFF_Q);
+        stash(xk, C::OFF_K);
+        // the tensor core reads shared memory through the async proxy
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        tmem = *tmem_holder;
+        if (tid == 0) {
+            const uint64_t dq = smem_desc_sw128(smem_u32(smem + C::OFF_Q), 16, 1024);
+            const uint64_t dk = smem_desc_sw128(smem_u32(smem + C::OFF_K), 16, 1024);
+            // (query part, key part): l.h, m.m, h.l, m.h, h.m, h.h (0 = h, 1 = m, 2 = l)
+            const int pa[6] = {2, 1, 0, 1, 0, 0}, pb[6] = {0, 1, 2, 0, 1, 0};
+#pragma unroll
+            for (int p = 0; p < 6; ++p) {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)  // 16 channels = 32 bytes of the swizzled row
+                    mma_ss(tmem, dq + (uint64_t)((pa[p] * C::PART + kk * 32) >> 4),
+                           dk + (uint64_t)((pb[p] * C::PART + kk * 32) >> 4), IDESC,
+                           (dc > 0 || p > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(smem_u32(bar));
+        }
+    }
+    done = done && mbar_wait(smem_u32(bar), (D / 64 - 1) & 1, wait_ns, (volatile int *)&never, 0x51, 0);
+    tc_fence_after();
+    // TMEM -> registers -> padded shared tile (the operand tiles are no longer read)
+    float *outs = reinterpret_cast<float *>(smem);
+    {
+        const int lr = (warp & 3) * 32 + lane;  // TMEM lane = query row of the tile
+        const int cb = (warp >> 2) * 64;        // this warp's 64 columns
+        uint32_t v[32];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + cb + c * 32, v);
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+                *reinterpret_cast<float4 *>(&outs[lr * C::OUT_LD + cb + c * 32 + e]) =
+                    make_float4(__uint_as_float(v[e]) * scale, __uint_as_float(v[e + 1]) * scale,
+                                __uint_as_float(v[e + 2]) * scale, __uint_as_float(v[e + 3]) * scale);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 128);
+    if (!done) return;  // a wait ran out: the device error word says so; store nothing
+    // coalesced rows: warp w stores rows w, w + 8, ...
+    const int ncol = min(TC_ROWS, nb - j0);
+    for (int rr = warp; rr < TC_ROWS; rr += 8) {
+        const int i = i0 + rr;
+        if (i >= nb) break;
+        float *dst = logits + ((size_t)bh * nb + i) * nb + j0;
+#pragma unroll
+        for (int c = lane; c < TC_ROWS; c += 32)
+            if (c < ncol) dst[c] = outs[rr * C::OUT_LD + c];
+    }
+}
+
 // ------------------------------------------------------------------------------------------
 // 2. per-row selection
 // ------------------------------------------------------------------------------------------
@@ -355,6 +517,27 @@ cudaError_t block_scores(const float *qp, const float *kp, float *logits, long l
     dim3 grid((nb + SC_TILE - 1) / SC_TILE, (nb + SC_TILE - 1) / SC_TILE, (unsigned)BH);
     block_scores_kernel<<<grid, 256, 0, st>>>(qp, kp, logits, nb, d, scale);
     return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_scores_tc(const float *qp, const float *kp, float *logits, long long BH,
+                                    int nb, float scale, unsigned long long wait_ns, cudaStream_t st) {
+    using C = ScoresTcCfg;
+    cudaError_t e = cudaFuncSetAttribute(block_scores_tc_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    const int t = (nb + TC_ROWS - 1) / TC_ROWS;
+    dim3 grid((unsigned)t, (unsigned)t, (unsigned)BH);
+    block_scores_tc_kernel<D><<<grid, 256, C::SMEM, st>>>(qp, kp, logits, nb, scale, wait_ns);
+    return cudaGetLastError();
+}
+
+cudaError_t block_scores_tc(const float *qp, const float *kp, float *logits, long long BH, int nb,
+                            int d, float scale, unsigned long long wait_ns, cudaStream_t st) {
+    if (BH == 0 || nb == 0) return cudaSuccess;
+    if (d == 128) return launch_scores_tc<128>(qp, kp, logits, BH, nb, scale, wait_ns, st);
+    if (d == 64) return launch_scores_tc<64>(qp, kp, logits, BH, nb, scale, wait_ns, st);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace bsa
