@@ -12,9 +12,6 @@ namespace bsa {
 cudaError_t pool_blocks(const void *q, const void *k, float *qp, float *kp, long long BH, int N,
                         int d, int bs, cudaStream_t st);
 
-cudaError_t block_scores(const float *qp, const float *kp, float *logits, long long BH, int nb,
-                         int d, float scale, cudaStream_t st);
-
 cudaError_t block_scores_tc(const float *qp, const float *kp, float *logits, long long BH, int nb,
                             int d, float scale, unsigned long long wait_ns, cudaStream_t st);
 

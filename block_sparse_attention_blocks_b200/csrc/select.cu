@@ -7,8 +7,9 @@
 // softmax(Qp Kp^T * scale) over pooled blocks.
 //
 // Two launches:
-//   1. block_scores_kernel: fp32 FFMA GEMM L = scale * Qp Kp^T per (b, h), written into the
-//      kv_idx buffer (same size: nb x nb 32-bit words per head), which doubles as staging.
+//   1. block_scores_tc_kernel: L = scale * Qp Kp^T per (b, h) on the tensor cores at fp32
+//      accuracy, written into the kv_idx buffer (same size: nb x nb 32-bit words per head),
+//      which doubles as staging.
 //   2. select_rows_kernel: one warp per query-block row.  Softmax in fp32, then the two
 //      prefixes of the ranked order (score descending, id ascending; ranking by score is ranking
 //      by probability) found by exact threshold searches over order-preserving score keys
@@ -24,93 +25,15 @@ namespace bsa {
 // ------------------------------------------------------------------------------------------
 // 1. block scores
 // ------------------------------------------------------------------------------------------
-constexpr int SC_TILE = 128;  // output tile: 128 query blocks x 128 key blocks of one head
-constexpr int SC_KC = 8;      // reduction chunk
-
-// fp32 FFMA GEMM L = scale * Qp Kp^T for one head, 256 threads, each 8 x 8 outputs (rows
-// ty*4 + {0..3} and 64 + ty*4 + {0..3}, likewise columns), operands staged transposed in shared
-// memory and double buffered.  Each output is an fp32 dot product accumulated in ascending c.
-__global__ void __launch_bounds__(256) block_scores_kernel(const float *__restrict__ qp,
-                                                           const float *__restrict__ kp,
-                                                           float *__restrict__ logits, int nb,
-                                                           int d, float scale) {
-    __shared__ __align__(16) float As[2][SC_KC][SC_TILE + 4];
-    __shared__ __align__(16) float Bs[2][SC_KC][SC_TILE + 4];
-    const int bh = blockIdx.z;
-    const int i0 = blockIdx.y * SC_TILE;
-    const int j0 = blockIdx.x * SC_TILE;
-    const float *A = qp + (size_t)bh * nb * d;
-    const float *Bm = kp + (size_t)bh * nb * d;
-    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-    const int lr = threadIdx.x / 2, lk = (threadIdx.x % 2) * 4;  // loader: row, k offset
-
-    float acc[8][8];
-#pragma unroll
-    for (int a = 0; a < 8; ++a)
-#pragma unroll
-        for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
-
-    auto load = [&](int c0, float4 &va, float4 &vb) {
-        va = make_float4(0.f, 0.f, 0.f, 0.f);
-        vb = va;
-        if (i0 + lr < nb) va = *reinterpret_cast<const float4 *>(A + (size_t)(i0 + lr) * d + c0 + lk);
-        if (j0 + lr < nb) vb = *reinterpret_cast<const float4 *>(Bm + (size_t)(j0 + lr) * d + c0 + lk);
-    };
-    auto stash = [&](int buf, const float4 &va, const float4 &vb) {
-        As[buf][lk + 0][lr] = va.x; As[buf][lk + 1][lr] = va.y;
-        As[buf][lk + 2][lr] = va.z; As[buf][lk + 3][lr] = va.w;
-        Bs[buf][lk + 0][lr] = vb.x; Bs[buf][lk + 1][lr] = vb.y;
-        Bs[buf][lk + 2][lr] = vb.z; Bs[buf][lk + 3][lr] = vb.w;
-    };
-
-    float4 va, vb;
-    load(0, va, vb);
-    stash(0, va, vb);
-    __syncthreads();
-    int buf = 0;
-    for (int c0 = 0; c0 < d; c0 += SC_KC) {
-        const bool more = c0 + SC_KC < d;
-        if (more) load(c0 + SC_KC, va, vb);
-#pragma unroll
-        for (int kk = 0; kk < SC_KC; ++kk) {
-            const float4 a0 = *reinterpret_cast<const float4 *>(&As[buf][kk][ty * 4]);
-            const float4 a1 = *reinterpret_cast<const float4 *>(&As[buf][kk][64 + ty * 4]);
-            const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[buf][kk][tx * 4]);
-            const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[buf][kk][64 + tx * 4]);
-            const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-            for (int x = 0; x < 8; ++x)
-#pragma unroll
-                for (int y = 0; y < 8; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
-        }
-        if (more) {
-            stash(buf ^ 1, va, vb);
-            __syncthreads();
-            buf ^= 1;
-        }
-    }
-#pragma unroll
-    for (int x = 0; x < 8; ++x) {
-        const int i = i0 + (x < 4 ? ty * 4 + x : 64 + ty * 4 + x - 4);
-        if (i >= nb) continue;
-        float *row = logits + ((size_t)bh * nb + i) * nb;
-#pragma unroll
-        for (int y = 0; y < 8; ++y) {
-            const int j = j0 + (y < 4 ? tx * 4 + y : 64 + tx * 4 + y - 4);
-            if (j < nb) row[j] = acc[x][y] * scale;
-        }
-    }
-}
-
-// Tensor-core form of the same scores.  Each fp32 operand x is split exactly into three bf16
+// L = scale * Qp Kp^T on the tensor cores.  Each fp32 operand x is split exactly into three bf16
 // parts, x = h + m + l: h keeps the sign, exponent and top 7 fraction bits of x (the low 16 bits
 // cleared), m the same of x - h, and l = x - h - m, which has at most 8 significant bits left
 // (each difference is exact in fp32).  The dot product is the sum of the six part products whose
 // weight is at least 2^-16 relative (l.h, m.m, h.l, m.h, h.m, h.h, smallest first), each a
 // tcgen05.mma.kind::f16 accumulating in one fp32 tensor-memory tile.  The products of bf16 parts
-// are exact in fp32, so the result differs from the fp32 FFMA dot product by accumulation
-// rounding of the same order.  One CTA computes one 128 x 128 tile (128 query blocks x 128 key
+// are exact in fp32, so the result differs from an fp32 FFMA dot product by accumulation
+// rounding of the same order (fp32, not bf16 or TF32: the mask decision needs the scores to
+// ~1e-6).  One CTA computes one 128 x 128 tile (128 query blocks x 128 key
 // blocks of one head) in 64-channel chunks: 256 threads load a chunk of both fp32 row tiles
 // (coalesced), split it into the six bf16 tiles in shared memory (the 128-byte swizzled K-major
 // layout the MMA descriptor reads), and thread 0 issues the 6 x 4 MMAs of the chunk; the finished tile goes
@@ -378,15 +301,16 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) select_rows_kernel(
     for (int r = 0; r < E; ++r) mx = fmaxf(mx, x[r]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    // per block: order key, exp(x - max), then the fixed-point probability round(P * 2^26) (sums
-    // over <= 1024 blocks stay below 2^32 and differ from the exact sum by < 8e-6)
+    // per block: order key, exp(x - max) on the SFU (relative error ~2^-22, under a tenth of the
+    // 1e-5 resolution of the cut), then the fixed-point probability round(P * 2^26) (sums over
+    // <= 1024 blocks stay below 2^32 and differ from the exact sum by < 8e-6)
     uint32_t key[E], pf[E];
     float z = 0.f;
 #pragma unroll
     for (int r = 0; r < E; ++r) {
         const bool ok = (r * 32 + lane) < nb;
         key[r] = ok ? ord_bits(x[r]) : 0u;
-        x[r] = ok ? expf(x[r] - mx) : 0.f;
+        x[r] = ok ? ex2((x[r] - mx) * 1.4426950408889634f) : 0.f;  // SFU exp; see the fixed point
         z += x[r];
     }
     z = warp_sum(z);
@@ -403,9 +327,9 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) select_rows_kernel(
     const bool want_p = topp > 0.f && topp < 1.f && total >= pfix;
     const bool all_kept = topp >= 1.f || (topp > 0.f && !want_p) || kk >= nb;
 
-    // ---- both thresholds, one bitwise search (top-k only matters when k > 0)
+    // ---- the top-p threshold first; the top-k one only if the top-p prefix is shorter than k
     uint32_t tp = 0u, tk = 0u;
-    if (!all_kept) search_thresholds<E>(key, pf, pfix, kk, want_p, kk > 0, tp, tk);
+    if (!all_kept && want_p) search_thresholds<E>(key, pf, pfix, kk, true, false, tp, tk);
 
     // ---- top-p count m (ties at tp taken in id order until the mass reaches p)
     int m, ntake = 0;
@@ -460,6 +384,8 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) select_rows_kernel(
         T = tp;
         take = ntake;
     } else {
+        uint32_t unused;
+        search_thresholds<E>(key, pf, pfix, kk, false, true, unused, tk);
         uint32_t above = 0u;
 #pragma unroll
         for (int r = 0; r < E; ++r) above += key[r] > tk ? 1u : 0u;
@@ -509,14 +435,6 @@ cudaError_t select_rows(const float *logits, long long rows, int nb, int topk, f
     if (nb <= 768) return launch_select_rows<24>(logits, rows, nb, topk, topp, mask, kv_idx, kv_cnt, st);
     if (nb <= 1024) return launch_select_rows<32>(logits, rows, nb, topk, topp, mask, kv_idx, kv_cnt, st);
     return cudaErrorInvalidValue;
-}
-
-cudaError_t block_scores(const float *qp, const float *kp, float *logits, long long BH, int nb,
-                         int d, float scale, cudaStream_t st) {
-    if (BH == 0 || nb == 0) return cudaSuccess;
-    dim3 grid((nb + SC_TILE - 1) / SC_TILE, (nb + SC_TILE - 1) / SC_TILE, (unsigned)BH);
-    block_scores_kernel<<<grid, 256, 0, st>>>(qp, kp, logits, nb, d, scale);
-    return cudaGetLastError();
 }
 
 template <int D>
