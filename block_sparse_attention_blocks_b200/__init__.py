@@ -5,7 +5,8 @@ Python functions re-exported here are argument marshalling around that library; 
 loads it and fails loudly if it has not been built.  ``workloads`` (seeded inputs) does not need
 the library.
 """
-_API = ("pool_blocks", "select_mask_topk_topp", "pool_select_topk_topp", "select_from_logits",
+_API = ("pool_blocks", "select_mask_topk_topp", "pool_select_topk_topp", "block_scores",
+        "select_from_logits",
         "block_sparse_attn_fwd",
         "dense_attn_fwd", "sparse_attention", "num_blocks", "device_error", "set_wait_limit_ns",
         "probe_bounded_wait", "SAError", "lib")

@@ -146,6 +146,18 @@ sa_status sa_select_from_logits(const float *logits, int B, int H, int nb, int t
                                       kv_cnt, (cudaStream_t)stream));
 }
 
+sa_status sa_block_scores(const float *qp, const float *kp, int B, int H, int nb, int d, float scale,
+                          float *logits, void *stream) {
+    if (!qp || !kp || !logits || !shape_ok(B, H, nb)) return SA_ERR_INVALID_ARG;
+    if (isnan(scale)) return SA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return SA_ERR_UNSUPPORTED;
+    if (!aligned16(qp) || !aligned16(kp) || !aligned16(logits)) return SA_ERR_INVALID_ARG;
+    int dev;
+    if (!select_device(logits, &dev)) return SA_ERR_INVALID_ARG;
+    return from_cuda(bsa::block_scores_tc(qp, kp, logits, (long long)B * H, nb, d,
+                                          resolve_scale(scale, d), g_wait_ns, (cudaStream_t)stream));
+}
+
 sa_status sa_select_mask_topk_topp(const float *qp, const float *kp, int B, int H, int nb, int d,
                                    int topk, float topp, float scale, uint8_t *mask,
                                    int32_t *kv_idx, int32_t *kv_cnt, void *stream) {

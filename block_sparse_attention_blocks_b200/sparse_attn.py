@@ -29,6 +29,7 @@ _F = ctypes.c_float
 lib.sa_pool_blocks.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]
 lib.sa_select_mask_topk_topp.argtypes = [_P, _P, _I, _I, _I, _I, _I, _F, _F, _P, _P, _P, _P]
 lib.sa_select_from_logits.argtypes = [_P, _I, _I, _I, _I, _F, _P, _P, _P, _P]
+lib.sa_block_scores.argtypes = [_P, _P, _I, _I, _I, _I, _F, _P, _P]
 lib.sa_pool_select_topk_topp.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _F, _P, _P,
                                          _P, _P]
 _Z = ctypes.c_size_t
@@ -43,7 +44,7 @@ lib.sa_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
 lib.sa_probe_bounded_wait.argtypes = [_P]
 lib.sa_num_blocks.argtypes = [_I, _I]
 for _f in (lib.sa_pool_blocks, lib.sa_select_mask_topk_topp, lib.sa_select_from_logits,
-           lib.sa_pool_select_topk_topp,
+           lib.sa_pool_select_topk_topp, lib.sa_block_scores,
            lib.sa_block_sparse_attn_fwd, lib.sa_dense_attn_fwd, lib.sa_get_device_error,
            lib.sa_set_wait_limit_ns, lib.sa_probe_bounded_wait, lib.sa_num_blocks):
     _f.restype = _I
@@ -170,6 +171,19 @@ def pool_select_topk_topp(q, k, bs: int, topk: int, topp: float, scale: float | 
                                         _ptr(kv_idx), _ptr(kv_cnt), _stream(q.device)),
            "sa_pool_select_topk_topp")
     return qp, kp, mask, kv_idx, kv_cnt
+
+
+def block_scores(qp, kp, scale: float | None = None, logits=None):
+    """The pooled block scores scale * Qp Kp^T -> [B, H, nb, nb] fp32."""
+    _need(qp, "qp", torch.float32, 4)
+    _need(kp, "kp", torch.float32, 4)
+    B, H, nb, d = qp.shape
+    logits = logits if logits is not None else torch.empty(B, H, nb, nb, dtype=torch.float32,
+                                                           device=qp.device)
+    _need(logits, "logits", torch.float32, 4)
+    _check(lib.sa_block_scores(_ptr(qp), _ptr(kp), B, H, nb, d, float(scale or 0.0), _ptr(logits),
+                               _stream(qp.device)), "sa_block_scores")
+    return logits
 
 
 def select_from_logits(logits, topk: int, topp: float, mask=None, kv_idx=None, kv_cnt=None):

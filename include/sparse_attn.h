@@ -99,6 +99,17 @@ sa_status sa_pool_select_topk_topp(const void *q, const void *k, float *qp, floa
                                    uint8_t *mask, int32_t *kv_idx, int32_t *kv_cnt, void *stream);
 
 /*
+ * The pooled block scores alone (the first half of sa_select_mask_topk_topp):
+ *   logits[b,h,i,j] = scale * qp[b,h,i,:] . kp[b,h,j,:]
+ * computed on the tensor cores at fp32 accuracy (each fp32 operand split exactly into three
+ * bf16 parts; the six part products of weight >= 2^-16 accumulate in fp32).
+ * qp, kp : [B, H, nb, d] fp32.  logits : [B, H, nb, nb] fp32, written.  d in {64, 128}.
+ * scale  : <= 0 selects 1/sqrt(d).
+ */
+sa_status sa_block_scores(const float *qp, const float *kp, int B, int H, int nb, int d, float scale,
+                          float *logits, void *stream);
+
+/*
  * Selection from caller-provided block scores (the second half of sa_select_mask_topk_topp,
  * exposed for tests that feed hand-made rows).  logits: [B, H, nb, nb] fp32 scores already
  * scaled; the row softmax, ranking, top-k union top-p and outputs are as above.  logits may be

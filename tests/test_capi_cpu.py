@@ -155,3 +155,37 @@ def test_python_binding_imports():
 
     assert callable(pkg.sparse_attention)
     assert pkg.num_blocks(75600, 128) == 591
+
+
+def test_block_scores_argument_checks(lib):
+    f = lib.sa_block_scores
+    f.argtypes = [ctypes.c_void_p] * 2 + [ctypes.c_int] * 4 + [ctypes.c_float] + [ctypes.c_void_p] * 2
+    assert f(NUL, A, 1, 1, 16, 128, 0.0, A2, S) == 1
+    assert f(A, A, 1, 1, 16, 96, 0.0, A2, S) == 2
+    assert f(A, A, 1, 1, 16, 128, float("nan"), A2, S) == 1
+    assert f(A, A, 1, 1, 16, 128, 0.0, MIS, S) == 1
+    assert f(A, A, 0, 1, 16, 128, 0.0, A2, S) == 1
+
+
+def test_bf16_three_way_split_is_exact():
+    # The tensor-core block scores split every fp32 operand x into bf16 parts by masking: h = x
+    # with the low 16 bits cleared, m the same of x - h, l = x - h - m.  The split must be exact
+    # (h + m + l == x) with l representable in bf16 (low 16 bits zero), for any sign and scale.
+    import numpy as np
+
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal(200000) * np.exp2(rng.integers(-60, 60, 200000))).astype(np.float32)
+    x = np.concatenate([x, np.float32([0.0, -0.0, 1.0, -1.0, 3.0e38, -3.0e38, 1.0e-30])])
+    mask = np.uint32(0xFFFF0000)
+    h = (x.view(np.uint32) & mask).view(np.float32)
+    rm = (x - h).astype(np.float32)
+    m = (rm.view(np.uint32) & mask).view(np.float32)
+    low = (rm - m).astype(np.float32)
+    assert np.all((low.view(np.uint32) & np.uint32(0xFFFF)) == 0)
+    assert np.array_equal(h.astype(np.float64) + m.astype(np.float64) + low.astype(np.float64),
+                          x.astype(np.float64))
+    # the dropped products m*l, l*m, l*l are below 2^-15 of |x|^2 each (|m| < 2^-7 |x|,
+    # |l| < 2^-14 |x| for normal x)
+    nz = np.abs(x) > 1e-30
+    assert np.all(np.abs(m[nz]) <= np.abs(x[nz]) * 2.0 ** -7)
+    assert np.all(np.abs(low[nz]) <= np.abs(x[nz]) * 2.0 ** -14)

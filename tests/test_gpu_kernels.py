@@ -65,6 +65,28 @@ def _gpu_select_logits(logits32, topk, topp):
     return mask.cpu().numpy(), idx.cpu().numpy(), cnt.cpu().numpy()
 
 
+@pytest.mark.parametrize("nb,d", [(591, 128), (130, 64), (7, 128), (256, 64)])
+def test_block_scores_against_oracle(orc, nb, d):
+    # tensor-core scores (bf16 x3 parts, fp32 accumulation) vs the fp64 definition; the bound is
+    # fp32 accumulation of the 6 x d part products plus the three dropped ones (< 2^-24 |q k|
+    # each), relative to the sum of |terms| of each dot product
+    rng = np.random.default_rng(nb + d)
+    B, H = 1, 2
+    qp = (rng.standard_normal((B, H, nb, d)) * 2.0).astype(np.float32)
+    kp = (rng.standard_normal((B, H, nb, d)) * 2.0).astype(np.float32)
+    scale = 1.0 / math.sqrt(d)
+    got = bsa.block_scores(torch.from_numpy(qp).to(DEV), torch.from_numpy(kp).to(DEV), scale)
+    torch.cuda.synchronize()
+    got = got.cpu().numpy().astype(np.float64)
+    ref = orc.block_logits(qp.astype(np.float64), kp.astype(np.float64), scale)
+    absum = np.einsum("bhic,bhjc->bhij", np.abs(qp.astype(np.float64)),
+                      np.abs(kp.astype(np.float64))) * scale
+    err = np.abs(got - ref)
+    assert np.all(err <= 64 * 2.0 ** -24 * absum + 1e-30), float((err / absum).max())
+    # a transposed operand or a misplaced tile would be off by O(1)
+    assert float((err / absum).max()) < 1e-6
+
+
 def test_select_handmade_rows(orc):
     nb = 24
     rows = []
