@@ -322,7 +322,9 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) select_rows_kernel(
         tsum += pf[r];
     }
     const uint32_t total = __reduce_add_sync(0xffffffffu, tsum);
-    const uint32_t pfix = __float2uint_rn(fminf(fmaxf(topp, 0.f), 1.f) * kFix);
+    // a positive p needs at least one block (the least count whose cumulative P reaches p), also
+    // when p is below the fixed-point resolution
+    const uint32_t pfix = max(__float2uint_rn(fminf(fmaxf(topp, 0.f), 1.f) * kFix), topp > 0.f ? 1u : 0u);
     const int kk = topk < nb ? topk : nb;
     const bool want_p = topp > 0.f && topp < 1.f && total >= pfix;
     const bool all_kept = topp >= 1.f || (topp > 0.f && !want_p) || kk >= nb;
