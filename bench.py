@@ -452,6 +452,32 @@ def run_gpu(args, w):
                  "sparse_call_speedup": ms_d / ms_step}
         del od
 
+    # ---------------------------------------------------------------- static pattern (context)
+    static = None
+    if not args.no_static and rank == 0:
+        # every head: a diagonal band of half-width 7 blocks plus the first 16 key blocks (a
+        # vertical stripe), about the realized density of the hybrid selection at this shape
+        pats = [(5, 7, 0, 16)] * H
+        ms_, ix_, ct_ = bsa.static_mask(pats, B, nb, device=dev)
+        bsa.block_sparse_attn_fwd(q, k, v, ix_, ct_, bs, o=o)
+        torch.cuda.synchronize(dev)
+        s0, s1, s2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        reps = 5
+        s0.record(stream)
+        for _ in range(reps):
+            bsa.static_mask(pats, B, nb, device=dev, mask=ms_, kv_idx=ix_, kv_cnt=ct_)
+        s1.record(stream)
+        for _ in range(reps):
+            bsa.block_sparse_attn_fwd(q, k, v, ix_, ct_, bs, o=o)
+        s2.record(stream)
+        torch.cuda.synchronize(dev)
+        f_st, p_st = executed_flops(ct_, ms_, N, d, bs)
+        ms_att = s1.elapsed_time(s2) / reps
+        static = {"pattern": "per head: |i - j| <= 7 blocks, or j < 16 (band + vertical stripe)",
+                  "density": p_st / float(B * H * nb * nb), "mask_ms": s0.elapsed_time(s1) / reps,
+                  "attention_ms": ms_att, "attention_tflops": f_st / (ms_att * 1e-3) / 1e12}
+        del ms_, ix_, ct_
+
     peaks, peak_src = load_peaks()
     peak_tc = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     peak_hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
@@ -498,6 +524,8 @@ def run_gpu(args, w):
         line["e2e"] = e2e
     if dense:
         line["dense_control"] = dense
+    if static:
+        line["static_pattern"] = static
 
     # ---------------------------------------------------------------- oracle on the host
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -532,6 +560,7 @@ def main():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--dense-steps", type=int, default=3)
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-static", action="store_true", help="skip the static-pattern timing")
     ap.add_argument("--heads", type=int, default=None,
                     help="run only the first H heads (small cases for profiling; not a bench line)")
     args = ap.parse_args()

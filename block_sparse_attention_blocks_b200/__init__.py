@@ -5,7 +5,7 @@ Python functions re-exported here are argument marshalling around that library; 
 loads it and fails loudly if it has not been built.  ``workloads`` (seeded inputs) does not need
 the library.
 """
-_API = ("pool_blocks", "select_mask_topk_topp", "pool_select_topk_topp", "block_scores",
+_API = ("pool_blocks", "select_mask_topk_topp", "pool_select_topk_topp", "block_scores", "static_mask",
         "select_from_logits",
         "block_sparse_attn_fwd",
         "dense_attn_fwd", "sparse_attention", "num_blocks", "device_error", "set_wait_limit_ns",

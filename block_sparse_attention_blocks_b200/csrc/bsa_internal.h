@@ -15,6 +15,9 @@ cudaError_t pool_blocks(const void *q, const void *k, float *qp, float *kp, long
 cudaError_t block_scores_tc(const float *qp, const float *kp, float *logits, long long BH, int nb,
                             int d, float scale, unsigned long long wait_ns, cudaStream_t st);
 
+cudaError_t static_mask(const int32_t *patterns, long long BH, int H, int nb, uint8_t *mask,
+                        int32_t *kv_idx, int32_t *kv_cnt, cudaStream_t st);
+
 cudaError_t select_rows(const float *logits, long long rows, int nb, int topk, float topp,
                         uint8_t *mask, int32_t *kv_idx, int32_t *kv_cnt, cudaStream_t st);
 

@@ -158,6 +158,16 @@ sa_status sa_block_scores(const float *qp, const float *kp, int B, int H, int nb
                                           resolve_scale(scale, d), g_wait_ns, (cudaStream_t)stream));
 }
 
+sa_status sa_static_mask(const int32_t *patterns, int B, int H, int nb, uint8_t *mask,
+                         int32_t *kv_idx, int32_t *kv_cnt, void *stream) {
+    if (!patterns || !mask || !kv_idx || !kv_cnt || !shape_ok(B, H, nb)) return SA_ERR_INVALID_ARG;
+    if (!aligned16(kv_idx)) return SA_ERR_INVALID_ARG;
+    int dev;
+    if (!select_device(kv_idx, &dev)) return SA_ERR_INVALID_ARG;
+    return from_cuda(bsa::static_mask(patterns, (long long)B * H, H, nb, mask, kv_idx, kv_cnt,
+                                      (cudaStream_t)stream));
+}
+
 sa_status sa_select_mask_topk_topp(const float *qp, const float *kp, int B, int H, int nb, int d,
                                    int topk, float topp, float scale, uint8_t *mask,
                                    int32_t *kv_idx, int32_t *kv_cnt, void *stream) {

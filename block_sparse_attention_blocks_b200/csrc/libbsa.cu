@@ -2,6 +2,7 @@
 // ptx.cuh, so they are compiled together.
 #include "pool.cu"
 #include "select.cu"
+#include "static.cu"
 #include "attn.cu"
 #include "probe.cu"
 #include "capi.cu"

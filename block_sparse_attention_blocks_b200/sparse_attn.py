@@ -30,6 +30,7 @@ lib.sa_pool_blocks.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]
 lib.sa_select_mask_topk_topp.argtypes = [_P, _P, _I, _I, _I, _I, _I, _F, _F, _P, _P, _P, _P]
 lib.sa_select_from_logits.argtypes = [_P, _I, _I, _I, _I, _F, _P, _P, _P, _P]
 lib.sa_block_scores.argtypes = [_P, _P, _I, _I, _I, _I, _F, _P, _P]
+lib.sa_static_mask.argtypes = [_P, _I, _I, _I, _P, _P, _P, _P]
 lib.sa_pool_select_topk_topp.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _F, _P, _P,
                                          _P, _P]
 _Z = ctypes.c_size_t
@@ -44,7 +45,7 @@ lib.sa_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
 lib.sa_probe_bounded_wait.argtypes = [_P]
 lib.sa_num_blocks.argtypes = [_I, _I]
 for _f in (lib.sa_pool_blocks, lib.sa_select_mask_topk_topp, lib.sa_select_from_logits,
-           lib.sa_pool_select_topk_topp, lib.sa_block_scores,
+           lib.sa_pool_select_topk_topp, lib.sa_block_scores, lib.sa_static_mask,
            lib.sa_block_sparse_attn_fwd, lib.sa_dense_attn_fwd, lib.sa_get_device_error,
            lib.sa_set_wait_limit_ns, lib.sa_probe_bounded_wait, lib.sa_num_blocks):
     _f.restype = _I
@@ -184,6 +185,19 @@ def block_scores(qp, kp, scale: float | None = None, logits=None):
     _check(lib.sa_block_scores(_ptr(qp), _ptr(kp), B, H, nb, d, float(scale or 0.0), _ptr(logits),
                                _stream(qp.device)), "sa_block_scores")
     return logits
+
+
+def static_mask(patterns, B: int, nb: int, device=None, mask=None, kv_idx=None, kv_cnt=None):
+    """Static block patterns -> (mask, kv_idx, kv_cnt) for block_sparse_attn_fwd.
+    patterns: H descriptors (flags, w, p, s): flags 1 = diagonal band |i - j| <= w, 2 = diagonals
+    every p blocks (half-width w), 4 = the first s key blocks; 0 = skipped head."""
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    pat = torch.as_tensor(patterns, dtype=torch.int32).reshape(-1, 4).to(dev)
+    H = pat.shape[0]
+    mask, kv_idx, kv_cnt = _sel_outputs(B, H, nb, dev, mask, kv_idx, kv_cnt)
+    _check(lib.sa_static_mask(_ptr(pat), B, H, nb, _ptr(mask), _ptr(kv_idx), _ptr(kv_cnt),
+                              _stream(dev)), "sa_static_mask")
+    return mask, kv_idx, kv_cnt
 
 
 def select_from_logits(logits, topk: int, topp: float, mask=None, kv_idx=None, kv_cnt=None):

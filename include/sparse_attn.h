@@ -110,6 +110,21 @@ sa_status sa_block_scores(const float *qp, const float *kp, int B, int H, int nb
                           float *logits, void *stream);
 
 /*
+ * Static block patterns (Sparse-vDiT, section 3: diagonal, multi-diagonal and vertical-stripe
+ * heads, and skipped heads) as a mask and kept-block lists for sa_block_sparse_attn_fwd.
+ * patterns : [H, 4] int32 on the device, one {flags, w, p, s} per head, shared by the batch; key
+ *            block j is kept for query block i when any enabled part holds:
+ *              flags & 1: |i - j| <= w                                  (diagonal band)
+ *              flags & 2: i - j within w of a multiple of p, p > 0      (diagonals every p)
+ *              flags & 4: j < s                                         (first s key blocks)
+ *            flags == 0 keeps nothing (skipped head; the attention then writes zeros).
+ * mask, kv_idx, kv_cnt : as for sa_select_mask_topk_topp ([B, H, nb, nb] u8, [B, H, nb, nb] i32
+ *            with the ascending kept ids first, [B, H, nb] i32).
+ */
+sa_status sa_static_mask(const int32_t *patterns, int B, int H, int nb, uint8_t *mask,
+                         int32_t *kv_idx, int32_t *kv_cnt, void *stream);
+
+/*
  * Selection from caller-provided block scores (the second half of sa_select_mask_topk_topp,
  * exposed for tests that feed hand-made rows).  logits: [B, H, nb, nb] fp32 scores already
  * scaled; the row softmax, ranking, top-k union top-p and outputs are as above.  logits may be

@@ -51,9 +51,10 @@ def _load():
     lib.or_select_rows.argtypes = [P, I, I, I, D, P, P, P, P, P, P, P, P]
     lib.or_masked_attention.argtypes = [P, P, P, I, I, I, P, D, P, P, I, P]
     lib.or_dense_attention.argtypes = [P, P, P, I, I, D, P, P, I, P]
+    lib.or_static_mask.argtypes = [P, I, I, P]
     for f in (lib.or_pool_blocks, lib.or_block_probs, lib.or_block_logits, lib.or_softmax_rows,
               lib.or_select_rows,
-              lib.or_masked_attention, lib.or_dense_attention):
+              lib.or_masked_attention, lib.or_dense_attention, lib.or_static_mask):
         f.restype = None
     _lib = lib
     return lib
@@ -165,6 +166,16 @@ def select(qp: np.ndarray, kp: np.ndarray, topk: int, topp: float, scale: float)
     sel = select_from_probs(block_probs(qp, kp, scale), topk, topp)
     sel.logit = block_logits(qp, kp, scale)
     return sel
+
+
+def static_mask(patterns, B: int, nb: int) -> np.ndarray:
+    """Static block pattern mask [B, H, nb, nb] uint8 from per-head descriptors
+    patterns[h] = (flags, w, p, s): diagonal band, multi-diagonal, vertical stripe (see oracle.c)."""
+    pat = np.ascontiguousarray(np.asarray(patterns, np.int32).reshape(-1, 4))
+    H = pat.shape[0]
+    out = np.empty((H, nb, nb), np.uint8)
+    _load().or_static_mask(_ptr(pat), H, nb, _ptr(out))
+    return np.broadcast_to(out, (B, H, nb, nb)).copy()
 
 
 def masked_attention(q_bits, k_bits, v_bits, mask, bs: int, scale: float, sel=None):

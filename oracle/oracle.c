@@ -341,3 +341,34 @@ void or_dense_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v,
         free(qr);
     }
 }
+
+/* ---------------------------------------------------------------------------------------------
+ * Static block patterns.  Sparse-vDiT page ("Sparse-vDiT：動画拡散トランスフォーマの高速化を可能に
+ * するスパースアテンションの解放"), section 3: attention maps of video DiT heads repeat as diagonal,
+ * multi-diagonal and vertical-stripe patterns, fixed per layer and head, and some heads can be
+ * skipped.  Read at block granularity, per head h with pat[h] = {flags, w, p, s}, key block j
+ * is kept for query block i when any enabled part holds:
+ *   flags & 1: |i - j| <= w                                  (diagonal band)
+ *   flags & 2: |(i - j) - m p| <= w for some integer m, p > 0 (diagonals every p blocks)
+ *   flags & 4: j < s                                         (vertical stripe of the first s)
+ * flags == 0 keeps nothing (a skipped head).  mask: [H, nb, nb].
+ * ------------------------------------------------------------------------------------------- */
+void or_static_mask(const int32_t *pat, int64_t H, int64_t nb, uint8_t *mask) {
+    for (int64_t h = 0; h < H; ++h) {
+        const int64_t flags = pat[4 * h], w = pat[4 * h + 1], p = pat[4 * h + 2], s = pat[4 * h + 3];
+        for (int64_t i = 0; i < nb; ++i) {
+            for (int64_t j = 0; j < nb; ++j) {
+                const int64_t diff = i - j;
+                int keep = 0;
+                if ((flags & 1) && llabs(diff) <= w) keep = 1;
+                if ((flags & 2) && p > 0) {
+                    /* every integer m whose diagonal m p can reach within w of diff */
+                    for (int64_t m = -(nb / p) - 1; m <= nb / p + 1 && !keep; ++m)
+                        if (llabs(diff - m * p) <= w) keep = 1;
+                }
+                if ((flags & 4) && j < s) keep = 1;
+                mask[(h * nb + i) * nb + j] = (uint8_t)keep;
+            }
+        }
+    }
+}

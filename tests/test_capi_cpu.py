@@ -189,3 +189,12 @@ def test_bf16_three_way_split_is_exact():
     nz = np.abs(x) > 1e-30
     assert np.all(np.abs(m[nz]) <= np.abs(x[nz]) * 2.0 ** -7)
     assert np.all(np.abs(low[nz]) <= np.abs(x[nz]) * 2.0 ** -14)
+
+
+def test_static_mask_argument_checks(lib):
+    f = lib.sa_static_mask
+    f.argtypes = [ctypes.c_void_p] + [ctypes.c_int] * 3 + [ctypes.c_void_p] * 4
+    assert f(NUL, 1, 1, 16, A, A2, A, S) == 1
+    assert f(A, 1, 1, 16, A, MIS, A, S) == 1
+    assert f(A, 0, 1, 16, A, A2, A, S) == 1
+    assert f(A, 1, 1, 16, NUL, A2, A, S) == 1

@@ -39,6 +39,12 @@ MUTANTS = {
     "dense attention uses the key as value": (
         "const uint16_t *vr = v + (bh * N + sk) * d;\n                for (int64_t c = 0; c < d; ++c) o[c] += e",
         "const uint16_t *vr = k + (bh * N + sk) * d;\n                for (int64_t c = 0; c < d; ++c) o[c] += e"),
+    "static band one block narrower": ("if ((flags & 1) && llabs(diff) <= w) keep = 1;",
+                                       "if ((flags & 1) && llabs(diff) < w) keep = 1;"),
+    "static stripe one block wider": ("if ((flags & 4) && j < s) keep = 1;",
+                                      "if ((flags & 4) && j <= s) keep = 1;"),
+    "static diagonals only on one side": ("for (int64_t m = -(nb / p) - 1; m <= nb / p + 1 && !keep; ++m)",
+                                          "for (int64_t m = 0; m <= nb / p + 1 && !keep; ++m)"),
     "pool reads the wrong channel": ("s += bf16_to_double(x[(bh * N + t) * d + c]);",
                                      "s += bf16_to_double(x[(bh * N + t) * d + (d - 1 - c)]);"),
 }

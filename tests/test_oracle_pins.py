@@ -317,3 +317,68 @@ def test_masked_key_order_invariance(orc):
     perm[64:128] = 64 + rng.permutation(64)
     o2 = orc.masked_attention(q, k[:, perm], v[:, perm], mask, bs, 0.25)
     np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------------------------
+# static block patterns (Sparse-vDiT page, section 3: diagonal, multi-diagonal, vertical stripe)
+# ---------------------------------------------------------------------------------------------
+def _brute_static(flags, w, p, s, nb):
+    """Pure-Python statement of the three patterns on a tiny grid (modular form)."""
+    m = np.zeros((nb, nb), np.uint8)
+    for i in range(nb):
+        for j in range(nb):
+            keep = False
+            if flags & 1 and abs(i - j) <= w:
+                keep = True
+            if flags & 2 and p > 0:
+                r = (i - j) % p
+                if r <= w or p - r <= w:
+                    keep = True
+            if flags & 4 and j < s:
+                keep = True
+            m[i, j] = keep
+    return m
+
+
+def test_static_band_row_counts(orc):
+    nb, w = 37, 3
+    m = orc.static_mask([(1, w, 0, 0)], 1, nb)[0, 0]
+    for i in range(nb):
+        assert m[i].sum() == min(i + w, nb - 1) - max(i - w, 0) + 1
+    assert np.array_equal(m, m.T)
+
+
+def test_static_multidiagonal_special_cases(orc):
+    nb = 29
+    # width 0: exactly the diagonals i - j = m p
+    m = orc.static_mask([(2, 0, 5, 0)], 1, nb)[0, 0]
+    i, j = np.meshgrid(np.arange(nb), np.arange(nb), indexing="ij")
+    assert np.array_equal(m, ((i - j) % 5 == 0).astype(np.uint8))
+    # a period longer than the grid leaves only the main band; period 1 keeps everything
+    assert np.array_equal(orc.static_mask([(2, 2, 4 * nb, 0)], 1, nb),
+                          orc.static_mask([(1, 2, 0, 0)], 1, nb))
+    assert orc.static_mask([(2, 0, 1, 0)], 1, nb).all()
+    mm = orc.static_mask([(2, 1, 7, 0)], 1, nb)[0, 0]
+    assert np.array_equal(mm, mm.T)
+
+
+def test_static_stripe_skip_and_union(orc):
+    nb = 23
+    st = orc.static_mask([(4, 0, 0, 5)], 1, nb)[0, 0]
+    assert st[:, :5].all() and not st[:, 5:].any()
+    assert orc.static_mask([(4, 0, 0, 99)], 1, nb).all()
+    assert not orc.static_mask([(0, 9, 3, 9)], 1, nb).any()
+    both = orc.static_mask([(5, 2, 0, 4)], 1, nb)
+    assert np.array_equal(both, orc.static_mask([(1, 2, 0, 0)], 1, nb) |
+                          orc.static_mask([(4, 0, 0, 4)], 1, nb))
+
+
+def test_static_patterns_against_brute_force(orc):
+    rng = np.random.default_rng(5)
+    pats = [(int(rng.integers(0, 8)), int(rng.integers(0, 4)), int(rng.integers(0, 9)),
+             int(rng.integers(0, 6))) for _ in range(40)]
+    nb = 17
+    got = orc.static_mask(pats, 2, nb)
+    for h, (f, w, p, s) in enumerate(pats):
+        ref = _brute_static(f, w, p, s, nb)
+        assert np.array_equal(got[0, h], ref) and np.array_equal(got[1, h], ref), (f, w, p, s)
