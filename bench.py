@@ -478,6 +478,29 @@ def run_gpu(args, w):
                   "attention_ms": ms_att, "attention_tflops": f_st / (ms_att * 1e-3) / 1e12}
         del ms_, ix_, ct_
 
+    # ---------------------------------------------------------------- SQuad (context)
+    squad = None
+    wsz = int(w.grid[1] * w.grid[2])  # tokens of one latent frame
+    if not args.no_squad and rank == 0 and N % wsz == 0:
+        osq = torch.empty_like(q)
+        bsa.squad_attn_fwd(q, k, v, wsz, o=osq)
+        torch.cuda.synchronize(dev)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 3
+        s0.record(stream)
+        for _ in range(reps):
+            bsa.squad_attn_fwd(q, k, v, wsz, o=osq)
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_sq = s0.elapsed_time(s1) / reps
+        # each query meets the wsz keys of its window, then the N / wsz keys at its position
+        f_sq = 4.0 * d * N * (wsz + N // wsz) * B * H
+        squad = {"window_tokens": wsz, "windows": N // wsz, "ms": ms_sq,
+                 "tflops": f_sq / (ms_sq * 1e-3) / 1e12,
+                 "pattern": "local pass within each latent frame, global pass across frames at "
+                            "each position (SQuad, w = tokens of one frame)"}
+        del osq
+
     peaks, peak_src = load_peaks()
     peak_tc = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     peak_hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
@@ -526,6 +549,8 @@ def run_gpu(args, w):
         line["dense_control"] = dense
     if static:
         line["static_pattern"] = static
+    if squad:
+        line["squad"] = squad
 
     # ---------------------------------------------------------------- oracle on the host
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -561,6 +586,7 @@ def main():
     ap.add_argument("--dense-steps", type=int, default=3)
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-static", action="store_true", help="skip the static-pattern timing")
+    ap.add_argument("--no-squad", action="store_true", help="skip the SQuad timing")
     ap.add_argument("--heads", type=int, default=None,
                     help="run only the first H heads (small cases for profiling; not a bench line)")
     args = ap.parse_args()

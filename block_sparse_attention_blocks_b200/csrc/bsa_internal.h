@@ -18,6 +18,9 @@ cudaError_t block_scores_tc(const float *qp, const float *kp, float *logits, lon
 cudaError_t static_mask(const int32_t *patterns, long long BH, int H, int nb, uint8_t *mask,
                         int32_t *kv_idx, int32_t *kv_cnt, cudaStream_t st);
 
+cudaError_t permute_tokens(const void *src, void *dst, long long G, long long A, long long R,
+                           int d, int num_sms, cudaStream_t st);
+
 cudaError_t select_rows(const float *logits, long long rows, int nb, int topk, float topp,
                         uint8_t *mask, int32_t *kv_idx, int32_t *kv_cnt, cudaStream_t st);
 

@@ -7,4 +7,5 @@
 #include "probe.cu"
 #include "capi.cu"
 #include "pipeline.cu"
+#include "squad.cu"
 #include "noalloc.cu"

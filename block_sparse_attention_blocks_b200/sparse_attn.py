@@ -34,6 +34,9 @@ lib.sa_static_mask.argtypes = [_P, _I, _I, _I, _P, _P, _P, _P]
 lib.sa_pool_select_topk_topp.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _F, _P, _P,
                                          _P, _P]
 _Z = ctypes.c_size_t
+lib.sa_squad_workspace_bytes.argtypes = [_I, _I, _I, _I]
+lib.sa_squad_workspace_bytes.restype = _Z
+lib.sa_squad_attn_fwd.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _Z, _P]
 lib.sa_block_sparse_attn_fwd.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _Z, _P]
 lib.sa_dense_attn_fwd.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _Z, _P]
 lib.sa_attn_workspace_bytes.argtypes = []
@@ -46,6 +49,7 @@ lib.sa_probe_bounded_wait.argtypes = [_P]
 lib.sa_num_blocks.argtypes = [_I, _I]
 for _f in (lib.sa_pool_blocks, lib.sa_select_mask_topk_topp, lib.sa_select_from_logits,
            lib.sa_pool_select_topk_topp, lib.sa_block_scores, lib.sa_static_mask,
+           lib.sa_squad_attn_fwd,
            lib.sa_block_sparse_attn_fwd, lib.sa_dense_attn_fwd, lib.sa_get_device_error,
            lib.sa_set_wait_limit_ns, lib.sa_probe_bounded_wait, lib.sa_num_blocks):
     _f.restype = _I
@@ -238,6 +242,22 @@ def dense_attn_fwd(q, k, v, scale: float | None = None, o=None):
     _check(lib.sa_dense_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d,
                                  float(scale or 0.0), _ptr(ws), ws.numel(), _stream(q.device)),
            "sa_dense_attn_fwd")
+    return o
+
+
+def squad_attn_fwd(q, k, v, w: int, scale: float | None = None, o=None):
+    """SQuad attention: softmax attention within windows of w tokens, then across windows at
+    each position with the local outputs as values -> O [B, H, N, d] bf16 (N a multiple of w)."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, torch.bfloat16, 4)
+    B, H, N, d = q.shape
+    o = o if o is not None else torch.empty_like(q)
+    _need(o, "o", torch.bfloat16, 4)
+    nbytes = int(lib.sa_squad_workspace_bytes(B, H, N, d))
+    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    _check(lib.sa_squad_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d, int(w),
+                                 float(scale or 0.0), _ptr(ws), ws.numel(), _stream(q.device)),
+           "sa_squad_attn_fwd")
     return o
 
 

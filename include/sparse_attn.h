@@ -125,6 +125,24 @@ sa_status sa_static_mask(const int32_t *patterns, int B, int H, int nb, uint8_t 
                          int32_t *kv_idx, int32_t *kv_cnt, void *stream);
 
 /*
+ * SQuad attention (SQuad: Sub-Quadratic Attention Distillation, method section 1): a local pass
+ * of softmax attention within fixed windows of w tokens, then a global pass of softmax attention
+ * among the tokens at the same position of every window, whose values are the local outputs.
+ * With N = W w and token t = a w + r (window a, position r):
+ *   Y[a w + r] = sum_{r'} softmax_{r'}(scale q[a w + r] . k[a w + r']) v[a w + r']
+ *   O[a w + r] = sum_{a'} softmax_{a'}(scale q[a w + r] . k[a' w + r]) Y[a' w + r]
+ * Runs as two dense attention calls with token regrouping between them (Y is held in bf16).
+ * q, k, v, o : [B, H, N, d] bf16, d in {64, 128}; N must be a multiple of w, and w and N / w
+ *              at most 131072.  scale <= 0 selects 1/sqrt(d) (both passes).
+ * workspace  : at least sa_squad_workspace_bytes(B, H, N, d) bytes of device memory, 16-byte
+ *              aligned, owned by the caller (four regrouped tensors and the work counter).
+ */
+size_t sa_squad_workspace_bytes(int B, int H, int N, int d);
+sa_status sa_squad_attn_fwd(const void *q, const void *k, const void *v, void *o, int B, int H,
+                            int N, int d, int w, float scale, void *workspace,
+                            size_t workspace_bytes, void *stream);
+
+/*
  * Selection from caller-provided block scores (the second half of sa_select_mask_topk_topp,
  * exposed for tests that feed hand-made rows).  logits: [B, H, nb, nb] fp32 scores already
  * scaled; the row softmax, ranking, top-k union top-p and outputs are as above.  logits may be

@@ -52,9 +52,11 @@ def _load():
     lib.or_masked_attention.argtypes = [P, P, P, I, I, I, P, D, P, P, I, P]
     lib.or_dense_attention.argtypes = [P, P, P, I, I, D, P, P, I, P]
     lib.or_static_mask.argtypes = [P, I, I, P]
+    lib.or_squad_attention.argtypes = [P, P, P, I, I, I, I, D, P]
     for f in (lib.or_pool_blocks, lib.or_block_probs, lib.or_block_logits, lib.or_softmax_rows,
               lib.or_select_rows,
-              lib.or_masked_attention, lib.or_dense_attention, lib.or_static_mask):
+              lib.or_masked_attention, lib.or_dense_attention, lib.or_static_mask,
+              lib.or_squad_attention):
         f.restype = None
     _lib = lib
     return lib
@@ -176,6 +178,19 @@ def static_mask(patterns, B: int, nb: int) -> np.ndarray:
     out = np.empty((H, nb, nb), np.uint8)
     _load().or_static_mask(_ptr(pat), H, nb, _ptr(out))
     return np.broadcast_to(out, (B, H, nb, nb)).copy()
+
+
+def squad_attention(q_bits, k_bits, v_bits, w: int, scale: float) -> np.ndarray:
+    """SQuad attention (local pass in windows of w tokens, global pass across windows at each
+    position with the local outputs as values).  q/k/v_bits: [BH, N, d] uint16, N a multiple of
+    w.  Returns [BH, N, d] float64."""
+    q, k, v = _bits(q_bits), _bits(k_bits), _bits(v_bits)
+    BH, N, d = q.shape
+    if N % w:
+        raise ValueError("N must be a multiple of w")
+    out = np.empty((BH, N, d), np.float64)
+    _load().or_squad_attention(_ptr(q), _ptr(k), _ptr(v), BH, N, d, w, float(scale), _ptr(out))
+    return out
 
 
 def masked_attention(q_bits, k_bits, v_bits, mask, bs: int, scale: float, sel=None):

@@ -372,3 +372,68 @@ void or_static_mask(const int32_t *pat, int64_t H, int64_t nb, uint8_t *mask) {
         }
     }
 }
+
+/* ---------------------------------------------------------------------------------------------
+ * SQuad attention.  SQuad page ("SQuad: Sub-Quadratic Attention Distillation for Efficient
+ * Video Generation"), method section 1, the SQuad attention operator: full attention is split
+ * into a local pass, softmax attention among the tokens of each fixed window of w tokens, and a
+ * global pass, softmax attention among the tokens at the same relative position in every window,
+ * whose values are the local pass's outputs.  With n = W w tokens, token t = a w + r (window a,
+ * position r):
+ *   Y[a w + r] = sum_{r'} softmax_{r'}(scale q[a w + r] . k[a w + r']) v[a w + r']
+ *   O[a w + r] = sum_{a'} softmax_{a'}(scale q[a w + r] . k[a' w + r]) Y[a' w + r]
+ * q, k, v: [BH, n, d] bf16 bits; out: [BH, n, d].  n must be a multiple of w.
+ * ------------------------------------------------------------------------------------------- */
+static void softmax_mix(const double *qr, const uint16_t *k, const double *vd, const uint16_t *vb,
+                        const int64_t *rows, int64_t m, int64_t d, double scale, double *w,
+                        double *o) {
+    /* o = sum over the m rows listed of softmax(scale qr . k[row]) * value[row]; the values are
+       vd (double) when given, else vb (bf16 bits) */
+    double mx = -INFINITY;
+    for (int64_t x = 0; x < m; ++x) {
+        const uint16_t *kr = k + rows[x] * d;
+        double s = 0.0;
+        for (int64_t c = 0; c < d; ++c) s += qr[c] * bf16_to_double(kr[c]);
+        w[x] = s * scale;
+        if (w[x] > mx) mx = w[x];
+    }
+    double z = 0.0;
+    for (int64_t c = 0; c < d; ++c) o[c] = 0.0;
+    for (int64_t x = 0; x < m; ++x) {
+        const double e = exp(w[x] - mx);
+        z += e;
+        for (int64_t c = 0; c < d; ++c)
+            o[c] += e * (vd ? vd[rows[x] * d + c] : bf16_to_double(vb[rows[x] * d + c]));
+    }
+    for (int64_t c = 0; c < d; ++c) o[c] /= z;
+}
+
+void or_squad_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t BH,
+                        int64_t n, int64_t d, int64_t win, double scale, double *out) {
+    const int64_t W = n / win;
+    double *y = (double *)malloc(sizeof(double) * (size_t)(n * d));
+    double *qr = (double *)malloc(sizeof(double) * (size_t)d);
+    double *wt = (double *)malloc(sizeof(double) * (size_t)(win > W ? win : W));
+    int64_t *rows = (int64_t *)malloc(sizeof(int64_t) * (size_t)(win > W ? win : W));
+    for (int64_t bh = 0; bh < BH; ++bh) {
+        const uint16_t *qb = q + bh * n * d, *kb = k + bh * n * d, *vb = v + bh * n * d;
+        /* local pass: the tokens of window a */
+        for (int64_t t = 0; t < n; ++t) {
+            const int64_t a = t / win;
+            for (int64_t x = 0; x < win; ++x) rows[x] = a * win + x;
+            for (int64_t c = 0; c < d; ++c) qr[c] = bf16_to_double(qb[t * d + c]);
+            softmax_mix(qr, kb, NULL, vb, rows, win, d, scale, wt, y + t * d);
+        }
+        /* global pass: the tokens at position r of every window, values from the local pass */
+        for (int64_t t = 0; t < n; ++t) {
+            const int64_t r = t % win;
+            for (int64_t x = 0; x < W; ++x) rows[x] = x * win + r;
+            for (int64_t c = 0; c < d; ++c) qr[c] = bf16_to_double(qb[t * d + c]);
+            softmax_mix(qr, kb, y, NULL, rows, W, d, scale, wt, out + (bh * n + t) * d);
+        }
+    }
+    free(y);
+    free(qr);
+    free(wt);
+    free(rows);
+}

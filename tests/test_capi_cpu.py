@@ -198,3 +198,19 @@ def test_static_mask_argument_checks(lib):
     assert f(A, 1, 1, 16, A, MIS, A, S) == 1
     assert f(A, 0, 1, 16, A, A2, A, S) == 1
     assert f(A, 1, 1, 16, NUL, A2, A, S) == 1
+
+
+def test_squad_argument_checks(lib):
+    lib.sa_squad_workspace_bytes.restype = ctypes.c_size_t
+    lib.sa_squad_workspace_bytes.argtypes = [ctypes.c_int] * 4
+    W = lib.sa_squad_workspace_bytes(1, 2, 512, 64)
+    assert W >= 4 * 2 * 512 * 64 * 2
+    f = lib.sa_squad_attn_fwd
+    f.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 5 + [ctypes.c_float, ctypes.c_void_p,
+                                                                ctypes.c_size_t, ctypes.c_void_p]
+    assert f(NUL, A, A, A, 1, 2, 512, 64, 64, 0.0, A2, W, S) == 1
+    assert f(A, A, A, A, 1, 2, 512, 96, 64, 0.0, A2, W, S) == 2
+    assert f(A, A, A, A, 1, 2, 512, 64, 100, 0.0, A2, W, S) == 1   # N not a multiple of w
+    assert f(A, A, A, A, 1, 2, 512, 64, 0, 0.0, A2, W, S) == 1
+    assert f(A, A, A, A, 1, 2, 512, 64, 64, 0.0, A2, W - 1, S) == 1
+    assert f(A, A, A, A, 1, 2, 512, 64, 64, float("nan"), A2, W, S) == 1

@@ -45,6 +45,11 @@ MUTANTS = {
                                       "if ((flags & 4) && j <= s) keep = 1;"),
     "static diagonals only on one side": ("for (int64_t m = -(nb / p) - 1; m <= nb / p + 1 && !keep; ++m)",
                                           "for (int64_t m = 0; m <= nb / p + 1 && !keep; ++m)"),
+    "squad global pass takes v, not the local outputs": (
+        "softmax_mix(qr, kb, y, NULL, rows, W, d, scale, wt, out + (bh * n + t) * d);",
+        "softmax_mix(qr, kb, NULL, vb, rows, W, d, scale, wt, out + (bh * n + t) * d);"),
+    "squad local pass over the wrong window": ("for (int64_t x = 0; x < win; ++x) rows[x] = a * win + x;",
+                                               "for (int64_t x = 0; x < win; ++x) rows[x] = ((a + 1) % W) * win + x;"),
     "pool reads the wrong channel": ("s += bf16_to_double(x[(bh * N + t) * d + c]);",
                                      "s += bf16_to_double(x[(bh * N + t) * d + (d - 1 - c)]);"),
 }

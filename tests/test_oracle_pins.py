@@ -382,3 +382,45 @@ def test_static_patterns_against_brute_force(orc):
     for h, (f, w, p, s) in enumerate(pats):
         ref = _brute_static(f, w, p, s, nb)
         assert np.array_equal(got[0, h], ref) and np.array_equal(got[1, h], ref), (f, w, p, s)
+
+
+# ---------------------------------------------------------------------------------------------
+# SQuad local + global attention (SQuad page, method section 1)
+# ---------------------------------------------------------------------------------------------
+def _squad_inputs(seed, BH=2, N=24, d=8):
+    rng = np.random.default_rng(seed)
+    return [f32_to_bf16_bits(rng.standard_normal((BH, N, d)).astype(np.float32)) for _ in range(3)]
+
+
+def test_squad_single_window_and_unit_window_are_dense(orc):
+    # one window of all n tokens: the global groups have one member, O = the local (dense)
+    # attention; windows of one token: the local pass returns v, the global pass is dense
+    q, k, v = _squad_inputs(1)
+    dense = orc.dense_attention(q, k, v, 0.35).reshape(q.shape)
+    assert np.abs(orc.squad_attention(q, k, v, 24, 0.35) - dense).max() < 1e-12
+    assert np.abs(orc.squad_attention(q, k, v, 1, 0.35) - dense).max() < 1e-12
+
+
+def test_squad_constant_values(orc):
+    q, k, _ = _squad_inputs(2)
+    v = np.broadcast_to(f32_to_bf16_bits(np.float32([[0.5, -1.25, 2.0, 0.0, 1.0, 3.0, -2.0, 0.25]])),
+                        q.shape).copy()
+    o = orc.squad_attention(q, k, v, 6, 0.35)
+    assert np.abs(o - bf16_bits_to_f32(v[0, 0]).astype(np.float64)).max() < 1e-12
+
+
+def test_squad_against_torch_reshape(orc):
+    # the same operator by reshapes and fp64 softmax attention in torch
+    import torch
+
+    q, k, v = _squad_inputs(3, BH=3, N=30, d=8)
+    w, scale = 5, 0.3
+    BH, N, d = q.shape
+    W = N // w
+    tq, tk, tv = (torch.from_numpy(bf16_bits_to_f32(x).astype(np.float64)).reshape(BH, W, w, d)
+                  for x in (q, k, v))
+    y = torch.softmax(tq @ tk.transpose(-1, -2) * scale, dim=-1) @ tv          # within windows
+    gq, gk, gy = (x.transpose(1, 2) for x in (tq, tk, y))                    # [BH, w, W, d]
+    o = torch.softmax(gq @ gk.transpose(-1, -2) * scale, dim=-1) @ gy        # across windows
+    ref = o.transpose(1, 2).reshape(BH, N, d).numpy()
+    assert np.abs(orc.squad_attention(q, k, v, w, scale) - ref).max() < 1e-12
