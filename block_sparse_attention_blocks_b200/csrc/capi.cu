@@ -17,6 +17,8 @@ unsigned long long g_wait_ns = kDefaultWaitNs;
 unsigned int *g_progress = nullptr;  // host-mapped stage words of the attention kernel, or null
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// int32 / fp32 buffers read and written element by element
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 bool shape_ok(int B, int H, int N) {
     if (B < 1 || H < 1 || N < 1) return false;
@@ -139,7 +141,7 @@ sa_status sa_select_from_logits(const float *logits, int B, int H, int nb, int t
     if (!logits || !mask || !kv_idx || !kv_cnt || !shape_ok(B, H, nb)) return SA_ERR_INVALID_ARG;
     if (topk < 0 || !(topp >= 0.f && topp <= 1.f)) return SA_ERR_INVALID_ARG;
     if (nb > 1024) return SA_ERR_UNSUPPORTED;
-    if (!aligned16(logits) || !aligned16(kv_idx)) return SA_ERR_INVALID_ARG;
+    if (!aligned4(logits) || !aligned4(kv_idx)) return SA_ERR_INVALID_ARG;
     int dev;
     if (!select_device(kv_idx, &dev)) return SA_ERR_INVALID_ARG;
     return from_cuda(bsa::select_rows(logits, (long long)B * H * nb, nb, topk, topp, mask, kv_idx,
@@ -151,7 +153,7 @@ sa_status sa_block_scores(const float *qp, const float *kp, int B, int H, int nb
     if (!qp || !kp || !logits || !shape_ok(B, H, nb)) return SA_ERR_INVALID_ARG;
     if (isnan(scale)) return SA_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return SA_ERR_UNSUPPORTED;
-    if (!aligned16(qp) || !aligned16(kp) || !aligned16(logits)) return SA_ERR_INVALID_ARG;
+    if (!aligned16(qp) || !aligned16(kp) || !aligned4(logits)) return SA_ERR_INVALID_ARG;
     int dev;
     if (!select_device(logits, &dev)) return SA_ERR_INVALID_ARG;
     return from_cuda(bsa::block_scores_tc(qp, kp, logits, (long long)B * H, nb, d,
@@ -161,7 +163,7 @@ sa_status sa_block_scores(const float *qp, const float *kp, int B, int H, int nb
 sa_status sa_static_mask(const int32_t *patterns, int B, int H, int nb, uint8_t *mask,
                          int32_t *kv_idx, int32_t *kv_cnt, void *stream) {
     if (!patterns || !mask || !kv_idx || !kv_cnt || !shape_ok(B, H, nb)) return SA_ERR_INVALID_ARG;
-    if (!aligned16(kv_idx)) return SA_ERR_INVALID_ARG;
+    if (!aligned4(kv_idx)) return SA_ERR_INVALID_ARG;
     int dev;
     if (!select_device(kv_idx, &dev)) return SA_ERR_INVALID_ARG;
     return from_cuda(bsa::static_mask(patterns, (long long)B * H, H, nb, mask, kv_idx, kv_cnt,
@@ -175,7 +177,7 @@ sa_status sa_select_mask_topk_topp(const float *qp, const float *kp, int B, int 
     if (topk < 0 || !(topp >= 0.f && topp <= 1.f) || isnan(scale)) return SA_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return SA_ERR_UNSUPPORTED;
     if (nb > 1024) return SA_ERR_UNSUPPORTED;
-    if (!aligned16(qp) || !aligned16(kp) || !aligned16(kv_idx)) return SA_ERR_INVALID_ARG;
+    if (!aligned16(qp) || !aligned16(kp) || !aligned4(kv_idx)) return SA_ERR_INVALID_ARG;
     int dev;
     if (!select_device(kv_idx, &dev)) return SA_ERR_INVALID_ARG;
     const long long BH = (long long)B * H;

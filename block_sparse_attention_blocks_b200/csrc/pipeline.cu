@@ -14,7 +14,7 @@ extern "C" sa_status sa_pool_select_topk_topp(const void *q, const void *k, floa
     if (!dims_supported(d, bs)) return SA_ERR_UNSUPPORTED;
     const int nb = sa_num_blocks(N, bs);
     if (nb > 1024) return SA_ERR_UNSUPPORTED;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(qp) || !aligned16(kp) || !aligned16(kv_idx))
+    if (!aligned16(q) || !aligned16(k) || !aligned16(qp) || !aligned16(kp) || !aligned4(kv_idx))
         return SA_ERR_INVALID_ARG;
     int dev;
     if (!select_device(kv_idx, &dev)) return SA_ERR_INVALID_ARG;

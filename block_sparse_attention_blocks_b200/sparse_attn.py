@@ -160,8 +160,8 @@ def select_mask_topk_topp(qp, kp, topk: int, topp: float, scale: float | None = 
 
 def pool_select_topk_topp(q, k, bs: int, topk: int, topp: float, scale: float | None = None,
                           qp=None, kp=None, mask=None, kv_idx=None, kv_cnt=None):
-    """Pooling and selection in one call (selection overlapped with pooling) ->
-    (qp, kp, mask, kv_idx, kv_cnt), the same values pool_blocks + select_mask_topk_topp give."""
+    """Pooling and selection in one call -> (qp, kp, mask, kv_idx, kv_cnt), the same values
+    pool_blocks + select_mask_topk_topp give."""
     for n, t in (("q", q), ("k", k)):
         _need(t, n, torch.bfloat16, 4)
     B, H, N, d = q.shape
@@ -261,23 +261,77 @@ def squad_attn_fwd(q, k, v, w: int, scale: float | None = None, o=None):
     return o
 
 
+def _host_pipeline(q, k, v, bs, topk, topp, scale, dev, out, chunks):
+    """Host inputs: the heads go through in chunks so that copies and kernels overlap.  Chunk c
+    is copied in on one stream, pooled, selected and attended on the current stream, and copied
+    out on a third; the next chunk's copy in and the previous chunk's copy out run meanwhile."""
+    B, H, N, d = q.shape
+    BH = B * H
+    nb = num_blocks(N, bs)
+    qf, kf, vf = (t.reshape(BH, N, d) for t in (q, k, v))
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=q.is_pinned())
+    of = out.reshape(BH, N, d)
+    qd, kd, vd = (torch.empty((BH, N, d), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    od = torch.empty((BH, N, d), dtype=torch.bfloat16, device=dev)
+    qp = torch.empty((1, BH, nb, d), dtype=torch.float32, device=dev)
+    kp = torch.empty_like(qp)
+    mask = torch.empty((1, BH, nb, nb), dtype=torch.uint8, device=dev)
+    kv_idx = torch.empty((1, BH, nb, nb), dtype=torch.int32, device=dev)
+    kv_cnt = torch.empty((1, BH, nb), dtype=torch.int32, device=dev)
+    main = torch.cuda.current_stream(dev)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    s_in.wait_stream(main)
+    s_out.wait_stream(main)
+    per = -(-BH // chunks)
+    for h0 in range(0, BH, per):
+        h1 = min(BH, h0 + per)
+        with torch.cuda.stream(s_in):
+            for dst, src in ((qd, qf), (kd, kf), (vd, vf)):
+                dst[h0:h1].copy_(src[h0:h1], non_blocking=True)
+            ev_in = torch.cuda.Event()
+            ev_in.record(s_in)
+        main.wait_event(ev_in)
+        sl = lambda t: t[:, h0:h1] if t.dim() == 4 else t[h0:h1].unsqueeze(0)
+        pool_select_topk_topp(sl(qd), sl(kd), bs, topk, topp, scale, qp=sl(qp), kp=sl(kp),
+                              mask=sl(mask), kv_idx=sl(kv_idx), kv_cnt=kv_cnt[:, h0:h1])
+        block_sparse_attn_fwd(sl(qd), sl(kd), sl(vd), sl(kv_idx), kv_cnt[:, h0:h1], bs, scale,
+                              o=sl(od))
+        ev_done = torch.cuda.Event()
+        ev_done.record(main)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_done)
+            of[h0:h1].copy_(od[h0:h1], non_blocking=True)
+    main.wait_stream(s_out)
+    # the device buffers stay in use by the side streams until their copies end
+    for t in (qd, kd, vd, od):
+        t.record_stream(s_in)
+        t.record_stream(s_out)
+    main.synchronize()  # O is on the host when the call returns
+    sel = (mask.reshape(B, H, nb, nb), kv_idx.reshape(B, H, nb, nb), kv_cnt.reshape(B, H, nb))
+    return out, sel
+
+
 def sparse_attention(q, k, v, bs: int, topk: int, topp: float, scale: float | None = None,
-                     device=None, return_selection: bool = False):
+                     device=None, return_selection: bool = False, out=None, chunks: int = 8):
     """The whole path: pool -> select -> block-sparse attention.
 
-    q, k, v may live on the host (ideally pinned) or on a CUDA device.  Host inputs are copied
-    to `device` (default: the current CUDA device) on the current stream and O is copied back
-    to the host; device inputs return a device O.
+    q, k, v may live on the host (ideally pinned) or on a CUDA device.  Device inputs return a
+    device O.  Host inputs are processed in `chunks` groups of heads on `device` (default: the
+    current CUDA device), with the copies of one group overlapping the kernels of another; O is
+    written to `out` (a host tensor of q's shape, ideally pinned) or to a new host tensor, and is
+    complete when the call returns.
     """
-    on_host = not q.is_cuda
-    if on_host:
+    if not q.is_cuda:
         dev = torch.device(device) if device is not None else torch.device("cuda",
                                                                            torch.cuda.current_device())
-        q, k, v = (t.to(dev, non_blocking=True) for t in (q, k, v))
+        for n, t in (("q", q), ("k", k), ("v", v)):
+            if t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_contiguous():
+                raise SAError(f"{n}: expected a contiguous 4-D bfloat16 tensor")
+        o, sel = _host_pipeline(q, k, v, bs, topk, topp, scale, dev, out, max(1, int(chunks)))
+        return (o, sel) if return_selection else o
     _, _, mask, kv_idx, kv_cnt = pool_select_topk_topp(q, k, bs, topk, topp, scale)
-    o = block_sparse_attn_fwd(q, k, v, kv_idx, kv_cnt, bs, scale)
-    if on_host:
-        o = o.to("cpu")
+    o = block_sparse_attn_fwd(q, k, v, kv_idx, kv_cnt, bs, scale, o=out)
     if return_selection:
         return o, (mask, kv_idx, kv_cnt)
     return o

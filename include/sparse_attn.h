@@ -31,7 +31,9 @@
  *     entry points take a small caller-owned device workspace (sa_attn_workspace_bytes()) that
  *     holds their work counter; calls that may overlap on the GPU need separate workspaces.
  *   - Tensors are dense and row-major with the last dimension contiguous.  bf16 tensors are
- *     passed as void*; their base addresses must be 16-byte aligned, fp32 tensors too.
+ *     passed as void*; their base addresses, and those of the pooled fp32 tensors and of
+ *     workspaces, must be 16-byte aligned.  int32 lists and counts, uint8 masks and fp32 block
+ *     scores are accessed element by element and need only their natural alignment.
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  The call
  *     runs on the device that owns the output pointer.
  *   - Supported shapes: d in {64, 128}, bs in {64, 128}, N >= 1 (any N; a tail block shorter

@@ -63,6 +63,7 @@ def test_num_blocks(lib):
 A = ctypes.c_void_p(0x10000)
 A2 = ctypes.c_void_p(0x20000)
 MIS = ctypes.c_void_p(0x10008)
+MIS4 = ctypes.c_void_p(0x10002)  # not even 4-byte aligned (int32 / fp32 element buffers)
 NUL = ctypes.c_void_p(0)
 S = ctypes.c_void_p(0)
 
@@ -97,7 +98,7 @@ def test_select_argument_checks(lib):
     assert call(s=float("nan")) == 1
     assert call(d=80) == 2
     assert call(nb=1025) == 2
-    assert call(idx=MIS) == 1
+    assert call(idx=MIS4) == 1
     g = lib.sa_select_from_logits
     g.argtypes = [ctypes.c_void_p] + [ctypes.c_int] * 4 + [ctypes.c_float] + [ctypes.c_void_p] * 4
     assert g(NUL, 1, 1, 16, 2, 0.5, A, A, A, S) == 1
@@ -124,7 +125,7 @@ def test_pool_select_argument_checks(lib):
     assert call(bs=32) == 2
     assert call(N=128 * 1025) == 2
     assert call(qp=MIS) == 1
-    assert call(idx=MIS) == 1
+    assert call(idx=MIS4) == 1
 
 
 def test_attention_argument_checks(lib):
@@ -163,7 +164,8 @@ def test_block_scores_argument_checks(lib):
     assert f(NUL, A, 1, 1, 16, 128, 0.0, A2, S) == 1
     assert f(A, A, 1, 1, 16, 96, 0.0, A2, S) == 2
     assert f(A, A, 1, 1, 16, 128, float("nan"), A2, S) == 1
-    assert f(A, A, 1, 1, 16, 128, 0.0, MIS, S) == 1
+    assert f(A, A, 1, 1, 16, 128, 0.0, MIS4, S) == 1
+    assert f(MIS, A, 1, 1, 16, 128, 0.0, A2, S) == 1
     assert f(A, A, 0, 1, 16, 128, 0.0, A2, S) == 1
 
 
@@ -195,7 +197,7 @@ def test_static_mask_argument_checks(lib):
     f = lib.sa_static_mask
     f.argtypes = [ctypes.c_void_p] + [ctypes.c_int] * 3 + [ctypes.c_void_p] * 4
     assert f(NUL, 1, 1, 16, A, A2, A, S) == 1
-    assert f(A, 1, 1, 16, A, MIS, A, S) == 1
+    assert f(A, 1, 1, 16, A, MIS4, A, S) == 1
     assert f(A, 0, 1, 16, A, A2, A, S) == 1
     assert f(A, 1, 1, 16, NUL, A2, A, S) == 1
 

@@ -300,3 +300,22 @@ def test_exp2_polynomial_against_cuda_exp2():
     assert rel < 1e-4, rel
     tiny = bsa.sparse_attn.exp2_poly(torch.tensor([-float("inf"), -300.0, -125.7], device=DEV))
     assert (tiny >= 0).all() and tiny.max() < 2e-38
+
+
+def test_host_pipeline_matches_device_path():
+    # host inputs go through in head chunks with overlapped copies; the result must be the
+    # device path's, bit for bit (the same kernels per head).  nb = 5: a chunk's kv_idx slice
+    # starts 4 bytes off a 16-byte boundary for odd first heads.
+    rng = np.random.default_rng(16)
+    B, H, N, d, bs = 2, 3, 600, 128, 128
+    q, k, v = (rand_bits(rng, (B, H, N, d)) for _ in range(3))
+    qh, kh, vh = (torch.from_numpy(x).view(torch.bfloat16).pin_memory() for x in (q, k, v))
+    out = torch.empty(qh.shape, dtype=torch.bfloat16).pin_memory()
+    oh, (mh, ih, ch) = bsa.sparse_attention(qh, kh, vh, bs, 2, 0.7, out=out, chunks=4,
+                                            return_selection=True)
+    assert oh.data_ptr() == out.data_ptr() and not oh.is_cuda
+    od, (md, idd, cd) = bsa.sparse_attention(qh.to(DEV), kh.to(DEV), vh.to(DEV), bs, 2, 0.7,
+                                             return_selection=True)
+    torch.cuda.synchronize()
+    assert torch.equal(oh.view(torch.int16), od.cpu().view(torch.int16))
+    assert torch.equal(mh.cpu(), md.cpu()) and torch.equal(ch.cpu(), cd.cpu())
