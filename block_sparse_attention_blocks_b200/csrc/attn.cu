@@ -3,8 +3,9 @@
 //
 // For each query block i and each kept key block j, S = Q_i K_j^T is a dense 128 x BS x d
 // contraction and O_i += P V_j a dense 128 x d x BS one, so both run on the tcgen05 tensor cores
-// with fp32 accumulators in tensor memory; softmax is online (running max and sum, O rescaled
-// when the max grows by more than 2^8), as in FlashAttention.  The key-block walk is what Sparse
+// with fp32 accumulators in tensor memory; softmax is online as in FlashAttention (a reference
+// max per row from the first kept block, P allowed to reach 2^30 before the reference moves and
+// O and the row sum are rescaled).  The key-block walk is what Sparse
 // VideoGen2 (section 2.C) describes: dense compute on a contiguous query tile, sparse loads of
 // the kept key/value blocks.  Keys at or beyond N are masked; query rows at or beyond N (and,
 // for BS = 64, rows of the next query block inside the 128-row tile) are computed but not
