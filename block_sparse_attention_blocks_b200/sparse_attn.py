@@ -2,8 +2,10 @@
 
 Every step of the path runs in the library's sm_100a kernels; this module checks tensor
 properties, allocates outputs through PyTorch (which owns device memory and streams here) and
-passes raw pointers and the current CUDA stream through ctypes.  There is no fallback: if the
-library is missing, importing this module raises.
+passes raw pointers and the current CUDA stream through ctypes.  For host inputs,
+`sparse_attention` also stages the tensors through device memory in chunks of heads, with the
+copies on side streams (plumbing only: no arithmetic runs on the host).  There is no fallback:
+if the library is missing, importing this module raises.
 """
 from __future__ import annotations
 
