@@ -53,10 +53,14 @@ def _load():
     lib.or_dense_attention.argtypes = [P, P, P, I, I, D, P, P, I, P]
     lib.or_static_mask.argtypes = [P, I, I, P]
     lib.or_squad_attention.argtypes = [P, P, P, I, I, I, I, D, P]
+    lib.or_kmeans.argtypes = [P, I, I, I, I, P, P]
+    lib.or_centroid_topp.argtypes = [P, P, P, I, I, I, D, D, P]
+    lib.or_cluster_attention.argtypes = [P, P, P, I, I, P, P, P, I, D, P]
     for f in (lib.or_pool_blocks, lib.or_block_probs, lib.or_block_logits, lib.or_softmax_rows,
               lib.or_select_rows,
               lib.or_masked_attention, lib.or_dense_attention, lib.or_static_mask,
-              lib.or_squad_attention):
+              lib.or_squad_attention, lib.or_kmeans, lib.or_centroid_topp,
+              lib.or_cluster_attention):
         f.restype = None
     _lib = lib
     return lib
@@ -191,6 +195,65 @@ def squad_attention(q_bits, k_bits, v_bits, w: int, scale: float) -> np.ndarray:
     out = np.empty((BH, N, d), np.float64)
     _load().or_squad_attention(_ptr(q), _ptr(k), _ptr(v), BH, N, d, w, float(scale), _ptr(out))
     return out
+
+
+def _bf16_values(bits) -> np.ndarray:
+    """The values of bf16 bit patterns (the top half of an IEEE binary32), as float64."""
+    b = np.ascontiguousarray(_bits(bits)).astype(np.uint32) << np.uint32(16)
+    return b.view(np.float32).astype(np.float64)
+
+
+def kmeans(x: np.ndarray, init: np.ndarray, iters: int):
+    """Lloyd k-means of the rows of x [n, d] from the centroids init [C, d] (SVG2 method A/C).
+    Returns (centroids [C, d] float64, assignment [n] int32)."""
+    x = np.ascontiguousarray(x, np.float64)
+    cent = np.ascontiguousarray(init, np.float64).copy()
+    n, d = x.shape
+    assign = np.empty(n, np.int32)
+    _load().or_kmeans(_ptr(x), n, d, cent.shape[0], int(iters), _ptr(cent), _ptr(assign))
+    return cent, assign
+
+
+def centroid_topp(cq: np.ndarray, ck: np.ndarray, size_k: np.ndarray, scale: float,
+                  p: float) -> np.ndarray:
+    """SVG2 centroid top-p (method B): sel [Cq, Ck] 0/1, key clusters taken by estimated score
+    size * exp(scale cq . ck) normalised per query cluster, until the cumulative score reaches p."""
+    cq = np.ascontiguousarray(cq, np.float64)
+    ck = np.ascontiguousarray(ck, np.float64)
+    size = np.ascontiguousarray(size_k, np.int64)
+    Cq, d = cq.shape
+    Ck = ck.shape[0]
+    sel = np.empty((Cq, Ck), np.uint8)
+    _load().or_centroid_topp(_ptr(cq), _ptr(ck), _ptr(size), Cq, Ck, d, float(scale), float(p),
+                             _ptr(sel))
+    return sel
+
+
+def cluster_attention(q_bits, k_bits, v_bits, assign_q, assign_k, sel, scale: float) -> np.ndarray:
+    """Attention of each query token over the keys of the clusters its cluster selected (one
+    head; q/k/v_bits [n, d] uint16).  Returns [n, d] float64."""
+    q, k, v = _bits(q_bits), _bits(k_bits), _bits(v_bits)
+    n, d = q.shape
+    aq = np.ascontiguousarray(assign_q, np.int32)
+    ak = np.ascontiguousarray(assign_k, np.int32)
+    s = np.ascontiguousarray(sel, np.uint8)
+    out = np.empty((n, d), np.float64)
+    _load().or_cluster_attention(_ptr(q), _ptr(k), _ptr(v), n, d, _ptr(aq), _ptr(ak), _ptr(s),
+                                 s.shape[1], float(scale), _ptr(out))
+    return out
+
+
+def svg2_attention(q_bits, k_bits, v_bits, init_q, init_k, iters: int, p: float, scale: float):
+    """The SVG2 path for one head: k-means of Q and of K (from the given, e.g. cached,
+    centroids), centroid top-p, attention over the selected clusters.  Returns (out [n, d],
+    assign_q, assign_k, cent_q, cent_k, sel)."""
+    qd, kd = _bf16_values(q_bits), _bf16_values(k_bits)
+    cent_q, aq = kmeans(qd, init_q, iters)
+    cent_k, ak = kmeans(kd, init_k, iters)
+    size_k = np.bincount(ak, minlength=cent_k.shape[0]).astype(np.int64)
+    sel = centroid_topp(cent_q, cent_k, size_k, scale, p)
+    out = cluster_attention(q_bits, k_bits, v_bits, aq, ak, sel, scale)
+    return out, aq, ak, cent_q, cent_k, sel
 
 
 def masked_attention(q_bits, k_bits, v_bits, mask, bs: int, scale: float, sel=None):

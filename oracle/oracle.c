@@ -437,3 +437,125 @@ void or_squad_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v,
     free(wt);
     free(rows);
 }
+
+/* ---------------------------------------------------------------------------------------------
+ * Sparse VideoGen2 semantic-aware permutation with centroid top-p.  SVG2 page ("Sparse
+ * VideoGen2: Accelerate Video Generation with Sparse Attention via Semantic-Aware Permutation"),
+ * method A (Q and K clustered separately by k-means into Cq and Ck groups, tokens reordered so
+ * that a cluster is contiguous; the permutations leave the result equal to attention in token
+ * order), B (scores between cluster centroids, clusters taken in order of the estimated score
+ * until the cumulative score reaches p) and C (k-means warm-started from cached centroids).
+ * ------------------------------------------------------------------------------------------- */
+
+/* k-means (Lloyd): `iters` rounds of assigning every row of x [n, d] to its nearest centroid
+ * (squared Euclidean distance, the lower index on a tie) and moving every centroid to the mean of
+ * its rows (a centroid without rows stays where it is), then a final assignment.  cent [C, d]
+ * holds the starting centroids on entry and the final ones on return; assign [n]. */
+void or_kmeans(const double *x, int64_t n, int64_t d, int64_t C, int64_t iters, double *cent,
+               int32_t *assign) {
+    double *sum = (double *)malloc(sizeof(double) * (size_t)(C * d));
+    int64_t *cnt = (int64_t *)malloc(sizeof(int64_t) * (size_t)C);
+    for (int64_t it = 0; it <= iters; ++it) {
+        for (int64_t t = 0; t < n; ++t) {
+            double best = INFINITY;
+            int64_t arg = 0;
+            for (int64_t c = 0; c < C; ++c) {
+                double dist = 0.0;
+                for (int64_t e = 0; e < d; ++e) {
+                    const double diff = x[t * d + e] - cent[c * d + e];
+                    dist += diff * diff;
+                }
+                if (dist < best) {
+                    best = dist;
+                    arg = c;
+                }
+            }
+            assign[t] = (int32_t)arg;
+        }
+        if (it == iters) break;
+        for (int64_t i = 0; i < C * d; ++i) sum[i] = 0.0;
+        for (int64_t c = 0; c < C; ++c) cnt[c] = 0;
+        for (int64_t t = 0; t < n; ++t) {
+            const int64_t c = assign[t];
+            cnt[c] += 1;
+            for (int64_t e = 0; e < d; ++e) sum[c * d + e] += x[t * d + e];
+        }
+        for (int64_t c = 0; c < C; ++c)
+            if (cnt[c] > 0)
+                for (int64_t e = 0; e < d; ++e) cent[c * d + e] = sum[c * d + e] / (double)cnt[c];
+    }
+    free(sum);
+    free(cnt);
+}
+
+/* Centroid top-p: for query cluster a, key cluster j is estimated to receive
+ *   w[a, j] = size_k[j] exp(scale cq[a] . ck[j]) / sum_j' size_k[j'] exp(scale cq[a] . ck[j'])
+ * of the attention (every key of a cluster stands in for by its centroid).  Key clusters are
+ * taken in order of w descending (the lower id first on a tie) until the cumulative w reaches p
+ * (p <= 0 takes none, p >= 1 takes every cluster with keys).  sel [Cq, Ck] 0/1. */
+void or_centroid_topp(const double *cq, const double *ck, const int64_t *size_k, int64_t Cq,
+                      int64_t Ck, int64_t d, double scale, double p, uint8_t *sel) {
+    ranked_t *ord = (ranked_t *)malloc(sizeof(ranked_t) * (size_t)Ck);
+    double *logit = (double *)malloc(sizeof(double) * (size_t)Ck);
+    for (int64_t a = 0; a < Cq; ++a) {
+        double mx = -INFINITY;
+        for (int64_t j = 0; j < Ck; ++j) {
+            double s = 0.0;
+            for (int64_t e = 0; e < d; ++e) s += cq[a * d + e] * ck[j * d + e];
+            logit[j] = s * scale;
+            if (size_k[j] > 0 && logit[j] > mx) mx = logit[j];
+        }
+        double z = 0.0;
+        for (int64_t j = 0; j < Ck; ++j) {
+            ord[j].p = size_k[j] > 0 ? (double)size_k[j] * exp(logit[j] - mx) : 0.0;
+            ord[j].j = (int32_t)j;
+            z += ord[j].p;
+        }
+        for (int64_t j = 0; j < Ck; ++j) ord[j].p /= z;
+        qsort(ord, (size_t)Ck, sizeof(ranked_t), ranked_cmp);
+        uint8_t *row = sel + a * Ck;
+        for (int64_t j = 0; j < Ck; ++j) row[j] = 0;
+        if (p <= 0.0) continue;
+        double cum = 0.0;
+        for (int64_t q = 0; q < Ck; ++q) {
+            if (ord[q].p <= 0.0) break;  /* clusters without keys are never taken */
+            row[ord[q].j] = 1;
+            cum += ord[q].p;
+            if (p < 1.0 && cum >= p) break;
+        }
+    }
+    free(ord);
+    free(logit);
+}
+
+/* Attention of every query token over the keys of the clusters its cluster selected:
+ *   O[t] = sum_{s : sel[aq[t], ak[s]]} softmax_s(scale q[t] . k[s]) v[s]
+ * (zero when the selection is empty).  q, k, v: [n, d] bf16 bits of one head; out [n, d]. */
+void or_cluster_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t n,
+                          int64_t d, const int32_t *aq, const int32_t *ak, const uint8_t *sel,
+                          int64_t Ck, double scale, double *out) {
+    double *w = (double *)malloc(sizeof(double) * (size_t)n);
+    for (int64_t t = 0; t < n; ++t) {
+        const uint8_t *row = sel + (int64_t)aq[t] * Ck;
+        double mx = -INFINITY;
+        for (int64_t s = 0; s < n; ++s) {
+            if (!row[ak[s]]) continue;
+            double x = 0.0;
+            for (int64_t c = 0; c < d; ++c) x += bf16_to_double(q[t * d + c]) * bf16_to_double(k[s * d + c]);
+            w[s] = x * scale;
+            if (w[s] > mx) mx = w[s];
+        }
+        double z = 0.0;
+        double *o = out + t * d;
+        for (int64_t c = 0; c < d; ++c) o[c] = 0.0;
+        for (int64_t s = 0; s < n; ++s) {
+            if (!row[ak[s]]) continue;
+            const double e = exp(w[s] - mx);
+            z += e;
+            for (int64_t c = 0; c < d; ++c) o[c] += e * bf16_to_double(v[s * d + c]);
+        }
+        if (z > 0.0)
+            for (int64_t c = 0; c < d; ++c) o[c] /= z;
+    }
+    free(w);
+}

@@ -50,6 +50,14 @@ MUTANTS = {
         "softmax_mix(qr, kb, NULL, vb, rows, W, d, scale, wt, out + (bh * n + t) * d);"),
     "squad local pass over the wrong window": ("for (int64_t x = 0; x < win; ++x) rows[x] = a * win + x;",
                                                "for (int64_t x = 0; x < win; ++x) rows[x] = ((a + 1) % W) * win + x;"),
+    "centroid top-p ignores the cluster sizes": (
+        "ord[j].p = size_k[j] > 0 ? (double)size_k[j] * exp(logit[j] - mx) : 0.0;",
+        "ord[j].p = size_k[j] > 0 ? exp(logit[j] - mx) : 0.0;"),
+    "k-means keeps the starting centroids": (
+        "cent[c * d + e] = sum[c * d + e] / (double)cnt[c];",
+        "cent[c * d + e] = cent[c * d + e];"),
+    "cluster attention reads the first query cluster's selection": (
+        "const uint8_t *row = sel + (int64_t)aq[t] * Ck;", "const uint8_t *row = sel;"),
     "pool reads the wrong channel": ("s += bf16_to_double(x[(bh * N + t) * d + c]);",
                                      "s += bf16_to_double(x[(bh * N + t) * d + (d - 1 - c)]);"),
 }

@@ -424,3 +424,100 @@ def test_squad_against_torch_reshape(orc):
     o = torch.softmax(gq @ gk.transpose(-1, -2) * scale, dim=-1) @ gy        # across windows
     ref = o.transpose(1, 2).reshape(BH, N, d).numpy()
     assert np.abs(orc.squad_attention(q, k, v, w, scale) - ref).max() < 1e-12
+
+
+# ---------------------------------------------------------------------------------------------
+# SVG2 semantic-aware permutation with centroid top-p (SVG2 page, method A, B and C)
+# ---------------------------------------------------------------------------------------------
+def _lloyd_numpy(x, init, iters):
+    """Plain vectorised Lloyd's algorithm (an independent statement of the oracle's k-means)."""
+    cent = init.astype(np.float64).copy()
+    for it in range(iters + 1):
+        dist = ((x[:, None, :] - cent[None, :, :]) ** 2).sum(-1)
+        assign = dist.argmin(1)              # the lower index on a tie
+        if it == iters:
+            break
+        for c in range(cent.shape[0]):
+            if (assign == c).any():
+                cent[c] = x[assign == c].mean(0)
+    return cent, assign
+
+
+def test_kmeans_separated_blobs_and_fixed_points(orc):
+    rng = np.random.default_rng(21)
+    centres = np.eye(4) * 6.0
+    x = np.concatenate([rng.standard_normal((15, 4)) * 0.2 + c for c in centres[:3]])
+    cent, assign = orc.kmeans(x, x[[0, 15, 30]], 6)
+    assert np.array_equal(assign, np.repeat(np.arange(3), 15))
+    for c in range(3):
+        assert np.abs(cent[c] - x[assign == c].mean(0)).max() < 1e-12
+    # a converged state does not move; one cluster per point keeps every point as its centroid
+    cent2, assign2 = orc.kmeans(x, cent, 3)
+    assert np.array_equal(assign2, assign) and np.abs(cent2 - cent).max() < 1e-12
+    cent3, assign3 = orc.kmeans(x, x, 2)
+    assert np.array_equal(assign3, np.arange(len(x))) and np.abs(cent3 - x).max() < 1e-12
+
+
+def test_kmeans_against_numpy_lloyd(orc):
+    rng = np.random.default_rng(22)
+    x = rng.standard_normal((60, 5))
+    init = x[rng.choice(60, 7, replace=False)]
+    cent, assign = orc.kmeans(x, init, 4)
+    ref_c, ref_a = _lloyd_numpy(x, init, 4)
+    assert np.array_equal(assign, ref_a) and np.abs(cent - ref_c).max() < 1e-12
+
+
+def test_centroid_topp_worked_example_and_limits(orc):
+    # one query centroid at the origin gives equal logits, so the estimate is the cluster size
+    # share: sizes (5, 3, 2, 0) -> (0.5, 0.3, 0.2, 0); p = 0.6 takes clusters 0 and 1
+    cq = np.zeros((1, 3))
+    ck = np.arange(12, dtype=np.float64).reshape(4, 3)
+    size = np.array([5, 3, 2, 0])
+    assert orc.centroid_topp(cq, ck, size, 1.0, 0.6).tolist() == [[1, 1, 0, 0]]
+    assert orc.centroid_topp(cq, ck, size, 1.0, 0.5).tolist() == [[1, 0, 0, 0]]
+    assert orc.centroid_topp(cq, ck, size, 1.0, 1.0).tolist() == [[1, 1, 1, 0]]   # not the empty one
+    assert orc.centroid_topp(cq, ck, size, 1.0, 0.0).tolist() == [[0, 0, 0, 0]]
+    # unit-size clusters: the estimate is the softmax of the query centroid's scores
+    rng = np.random.default_rng(23)
+    cq = rng.standard_normal((2, 4))
+    ck = rng.standard_normal((6, 4))
+    for a in range(2):
+        w = np.exp(0.5 * ck @ cq[a])
+        w /= w.sum()
+        order = sorted(range(6), key=lambda j: (-w[j], j))
+        cum, take = 0.0, []
+        for j in order:
+            take.append(j)
+            cum += w[j]
+            if cum >= 0.7:
+                break
+        sel = orc.centroid_topp(cq, ck, np.ones(6, np.int64), 0.5, 0.7)[a]
+        assert sorted(np.flatnonzero(sel).tolist()) == sorted(take)
+
+
+def test_cluster_attention_reduces_to_dense_and_block_sparse(orc):
+    rng = np.random.default_rng(24)
+    n, d, bs = 48, 8, 16
+    q, k, v = (f32_to_bf16_bits(rng.standard_normal((n, d)).astype(np.float32)) for _ in range(3))
+    dense = orc.dense_attention(q[None], k[None], v[None], 0.3).reshape(n, d)
+    one = np.zeros(n, np.int32)
+    assert np.abs(orc.cluster_attention(q, k, v, one, one, np.ones((1, 1), np.uint8), 0.3)
+                  - dense).max() < 1e-12
+    # clusters = contiguous blocks: the selection is a block mask
+    blocks = (np.arange(n) // bs).astype(np.int32)
+    mask = np.array([[1, 0, 1], [0, 1, 0], [1, 1, 1]], np.uint8)
+    got = orc.cluster_attention(q, k, v, blocks, blocks, mask, 0.3)
+    ref = orc.masked_attention(q[None], k[None], v[None], mask[None], bs, 0.3).reshape(n, d)
+    assert np.abs(got - ref).max() < 1e-12
+
+
+def test_svg2_one_key_per_cluster_and_full_p_is_dense(orc):
+    rng = np.random.default_rng(25)
+    n, d = 32, 8
+    q, k, v = (f32_to_bf16_bits(rng.standard_normal((n, d)).astype(np.float32)) for _ in range(3))
+    kd = bf16_bits_to_f32(k).astype(np.float64)
+    qd = bf16_bits_to_f32(q).astype(np.float64)
+    out, aq, ak, cq, ck, sel = orc.svg2_attention(q, k, v, qd[:4], kd, 3, 1.0, 0.3)
+    assert np.array_equal(ak, np.arange(n)) and sel.all()
+    dense = orc.dense_attention(q[None], k[None], v[None], 0.3).reshape(n, d)
+    assert np.abs(out - dense).max() < 1e-12
