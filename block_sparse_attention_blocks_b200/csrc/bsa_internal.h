@@ -29,6 +29,35 @@ cudaError_t attn_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtenso
                      int d, int bs, float scale, unsigned long long wait_ns, int num_sms,
                      unsigned int *progress, unsigned int *workspace, cudaStream_t st);
 
+cudaError_t attn_varlen_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                            const int2 *units, int units_per_head, const int32_t *tiles,
+                            const int32_t *tcnt, int tstride, const int32_t *perm_q, void *o,
+                            long long BH, int N, int Cq, int d, float scale,
+                            unsigned long long wait_ns, int num_sms, unsigned int *workspace,
+                            cudaStream_t st);
+
+cudaError_t kmeans_lloyd(const void *x, float *cent, int32_t *assign, int32_t *perm,
+                         int32_t *cstart, int32_t *csize, long long BH, int N, int d, int C,
+                         int iters, cudaStream_t st);
+
+cudaError_t cluster_sort(const int32_t *assign, long long BH, int N, int C, int32_t *perm,
+                         int32_t *cstart, int32_t *csize, cudaStream_t st);
+
+cudaError_t centroid_logits(const float *cq, const float *ck, const int32_t *size_k,
+                            float *logits, long long BH, int Cq, int Ck, int d, float scale,
+                            cudaStream_t st);
+
+cudaError_t prune_empty(uint8_t *sel, const int32_t *size_k, long long BH, int Cq, int Ck,
+                        int num_sms, cudaStream_t st);
+
+cudaError_t build_cluster_tables(const uint8_t *sel, const int32_t *qstart, const int32_t *qsize,
+                                 const int32_t *kstart, const int32_t *ksize, long long BH,
+                                 int Cq, int Ck, int U, int tstride, int2 *units, int32_t *tiles,
+                                 int32_t *tcnt, cudaStream_t st);
+
+cudaError_t gather_rows(const void *src, const int32_t *perm, void *dst, long long BH, int N,
+                        int d, int num_sms, cudaStream_t st);
+
 cudaError_t bounded_wait_probe(unsigned long long wait_ns, cudaStream_t st);
 
 cudaError_t exp2_poly_eval(const float *x, float *y, int n, cudaStream_t st);

@@ -4,8 +4,10 @@
 #include "select.cu"
 #include "static.cu"
 #include "attn.cu"
+#include "attn_varlen.cu"
 #include "probe.cu"
 #include "capi.cu"
 #include "pipeline.cu"
 #include "squad.cu"
+#include "svg2.cu"
 #include "noalloc.cu"

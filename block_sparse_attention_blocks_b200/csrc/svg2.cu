@@ -1,0 +1,713 @@
+// Semantic-aware permutation with centroid top-p (page "Sparse VideoGen2: Accelerate Video
+// Generation with Sparse Attention via Semantic-Aware Permutation", method sections A, B and C).
+//
+//   A. k-means (Lloyd) of the Q rows and, separately, of the K rows of every head into Cq and Ck
+//      clusters, started from the caller's centroids (the centroid cache of section C); tokens
+//      are then reordered so that every cluster is a contiguous range.
+//   B. The score of key cluster j for query cluster a is estimated from the centroids, every key
+//      standing in for by its centroid: |j| exp(scale mu_q[a] . mu_k[j]), normalised over j.
+//      Key clusters are taken in descending order of it until the cumulative score reaches p.
+//   C. Attention of each query token over the keys of the clusters its cluster selected, on the
+//      permuted tensors (dense query tiles, key tiles of variable length), written back in the
+//      original token order.
+//
+// Kernels here: the assignment step (nearest centroid, squared Euclidean distance, the lower
+// index on a tie), a stable counting sort of the assignment (the permutation and each cluster's
+// range), the update step (the mean of each cluster's rows, summed in token order), the
+// centroid scores, the tables of query tiles and key tiles, and the row gather.  Selection runs
+// on the top-p kernel of the block path (top-k = 0) over the scores log|j| + scale mu_q . mu_k,
+// whose softmax is the estimate above; the attention is attn_varlen.cu.
+#include "bsa_internal.h"
+#include "sparse_attn.h"
+
+namespace bsa {
+
+constexpr int kMaxClusters = 1024;   // Cq, Ck: one selection row per warp, sort counters in smem
+constexpr int kMaxVarlenN = 1 << 24; // key tile entries pack (first row << 7) into 31 bits
+
+// ------------------------------------------------------------------------------------------
+// k-means assignment: thread per token, its row in registers; centroids staged 32 at a time in
+// shared memory with their squared norms; |x - c|^2 - |x|^2 = |c|^2 - 2 x . c in fp32.
+// ------------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) kmeans_assign_kernel(const __nv_bfloat16 *__restrict__ x,
+                                                            const float *__restrict__ cent,
+                                                            int32_t *__restrict__ assign, int N,
+                                                            int C) {
+    constexpr int CH = 32;
+    __shared__ __align__(16) float cs[CH * D];
+    __shared__ float cn[CH];
+    const int bh = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n = blockIdx.x * 256 + threadIdx.x;
+    const bool ok = n < N;
+    float xr[D];
+    {
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + ((size_t)bh * N + (ok ? n : 0)) * D);
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+            const uint4 w = src[c];
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                xr[8 * c + 2 * h] = __uint_as_float(ws[h] << 16);
+                xr[8 * c + 2 * h + 1] = __uint_as_float(ws[h] & 0xFFFF0000u);
+            }
+        }
+    }
+    const float *cb = cent + (size_t)bh * C * D;
+    float best = INFINITY;
+    int arg = 0;
+    for (int c0 = 0; c0 < C; c0 += CH) {
+        __syncthreads();  // every thread is done with the previous chunk
+        for (int i = threadIdx.x; i < CH * D / 4; i += 256) {
+            const int cc = i / (D / 4);
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (c0 + cc < C) v = reinterpret_cast<const float4 *>(cb + (size_t)(c0 + cc) * D)[i % (D / 4)];
+            reinterpret_cast<float4 *>(cs)[i] = v;
+        }
+        __syncthreads();
+        for (int cc = warp; cc < CH; cc += 8) {
+            float s = 0.f;
+            for (int e = lane; e < D; e += 32) s = fmaf(cs[cc * D + e], cs[cc * D + e], s);
+            s = warp_sum(s);
+            if (lane == 0) cn[cc] = c0 + cc < C ? s : INFINITY;  // padding is never nearest
+        }
+        __syncthreads();
+        const int m = min(CH, C - c0);
+        for (int cc = 0; cc < m; cc += 4) {
+            float a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int e = 0; e < D; e += 4) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float4 c4 = *reinterpret_cast<const float4 *>(&cs[(cc + j) * D + e]);
+                    a[j] = fmaf(xr[e], c4.x, a[j]);
+                    a[j] = fmaf(xr[e + 1], c4.y, a[j]);
+                    a[j] = fmaf(xr[e + 2], c4.z, a[j]);
+                    a[j] = fmaf(xr[e + 3], c4.w, a[j]);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float dist = fmaf(-2.f, a[j], cn[cc + j]);
+                if (dist < best) {  // strict: the lower index keeps a tie
+                    best = dist;
+                    arg = c0 + cc + j;
+                }
+            }
+        }
+    }
+    if (ok) assign[(size_t)bh * N + n] = arg;
+}
+
+// ------------------------------------------------------------------------------------------
+// Stable counting sort of one head's assignment (one CTA of 8 warps per head).  Warp w owns a
+// contiguous eighth of the tokens: it counts its tokens per cluster, the counts are scanned in
+// (cluster, warp) order, and each warp then places its tokens in token order (lanes of a 32-token
+// step that share a cluster are ranked with match.any).  Cluster c occupies
+// perm[cstart[c] .. cstart[c] + csize[c]) with its tokens ascending.
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) cluster_sort_kernel(const int32_t *__restrict__ assign,
+                                                           int N, int C, int32_t *__restrict__ perm,
+                                                           int32_t *__restrict__ cstart,
+                                                           int32_t *__restrict__ csize) {
+    extern __shared__ int32_t sm_sort[];
+    int32_t *cnt = sm_sort;           // [8][C]: count, then the warp's next free position
+    int32_t *start = sm_sort + 8 * C; // [C]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long bh = blockIdx.x;
+    const int32_t *as = assign + bh * N;
+    for (int i = threadIdx.x; i < 8 * C; i += 256) cnt[i] = 0;
+    __syncthreads();
+    const int per = (N + 7) / 8;
+    const int lo = min(N, warp * per), hi = min(N, lo + per);
+    bool bad = false;
+    for (int s = lo; s < hi; s += 32) {
+        const int n = s + lane;
+        if (n < hi) {
+            int a = as[n];
+            if (a < 0 || a >= C) {
+                bad = true;
+                a = a < 0 ? 0 : C - 1;
+            }
+            atomicAdd(&cnt[warp * C + a], 1);
+        }
+    }
+    if (bad) atomicOr(&g_bsa_device_error, BSA_DEVERR_BOUNDS);
+    __syncthreads();
+    for (int c = threadIdx.x; c < C; c += 256) {
+        int t = 0;
+        for (int w = 0; w < 8; ++w) t += cnt[w * C + c];
+        start[c] = t;
+    }
+    __syncthreads();
+    if (warp == 0) {  // exclusive scan of the cluster sizes
+        int run = 0;
+        for (int c0 = 0; c0 < C; c0 += 32) {
+            const int c = c0 + lane;
+            const int v = c < C ? start[c] : 0;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            if (c < C) start[c] = run + incl - v;
+            run += __shfl_sync(0xffffffffu, incl, 31);
+        }
+    }
+    __syncthreads();
+    for (int c = threadIdx.x; c < C; c += 256) {
+        int run = start[c];
+        cstart[bh * C + c] = run;
+        for (int w = 0; w < 8; ++w) {
+            const int t = cnt[w * C + c];
+            cnt[w * C + c] = run;
+            run += t;
+        }
+        csize[bh * C + c] = run - start[c];
+    }
+    __syncthreads();
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int s = lo; s < hi; s += 32) {  // warp-uniform bounds
+        const int n = s + lane;
+        const bool v = n < hi;
+        int a = -1;
+        if (v) a = min(max(as[n], 0), C - 1);
+        const uint32_t peers = __match_any_sync(0xffffffffu, a);
+        const int rank = __popc(peers & lt);
+        if (v) perm[bh * N + cnt[warp * C + a] + rank] = n;
+        __syncwarp();
+        if (v && rank == 0) cnt[warp * C + a] += __popc(peers);
+        __syncwarp();
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// k-means update: one CTA per (cluster, head).  Column pairs x token lanes; each lane sums its
+// tokens in permuted (= token) order, the lanes are added in lane order, so the result does not
+// depend on scheduling.  A cluster without tokens keeps its centroid.
+// ------------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(512) kmeans_update_kernel(const __nv_bfloat16 *__restrict__ x,
+                                                            const int32_t *__restrict__ perm,
+                                                            const int32_t *__restrict__ cstart,
+                                                            const int32_t *__restrict__ csize,
+                                                            float *__restrict__ cent, int N, int C) {
+    constexpr int P = D / 2;    // bf16 pairs per row
+    constexpr int G = 512 / P;  // token lanes
+    __shared__ float2 part[G][P];
+    const int c = blockIdx.x;
+    const long long bh = blockIdx.y;
+    const int pr = threadIdx.x % P, g = threadIdx.x / P;
+    const int sz = csize[bh * C + c];
+    if (sz <= 0) return;  // the whole CTA leaves together
+    const int32_t *pm = perm + bh * N + cstart[bh * C + c];
+    const uint32_t *xb = reinterpret_cast<const uint32_t *>(x) + (size_t)bh * N * P;
+    float sx = 0.f, sy = 0.f;
+#pragma unroll 4
+    for (int s = g; s < sz; s += G) {
+        const int n = min(max(pm[s], 0), N - 1);
+        const uint32_t w = xb[(size_t)n * P + pr];
+        sx += __uint_as_float(w << 16);
+        sy += __uint_as_float(w & 0xFFFF0000u);
+    }
+    part[g][pr] = make_float2(sx, sy);
+    __syncthreads();
+    if (g == 0) {
+        float tx = 0.f, ty = 0.f;
+        for (int i = 0; i < G; ++i) {
+            tx += part[i][pr].x;
+            ty += part[i][pr].y;
+        }
+        float *dst = cent + (bh * C + c) * D + 2 * pr;
+        dst[0] = tx / (float)sz;
+        dst[1] = ty / (float)sz;
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// Centroid scores: logits[a, j] = log|j| + scale mu_q[a] . mu_k[j], -inf for an empty key
+// cluster, so that softmax_j(logits[a, :]) is the estimated score of section B.  One warp per
+// query centroid, one lane per key centroid of a 32-wide chunk staged in shared memory.
+// ------------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) centroid_logits_kernel(const float *__restrict__ cq,
+                                                              const float *__restrict__ ck,
+                                                              const int32_t *__restrict__ size_k,
+                                                              float *__restrict__ logits, int Cq,
+                                                              int Ck, float scale) {
+    __shared__ float qs[8][D];
+    __shared__ float ks[32][D + 1];  // +1: lane j reads row j, conflict-free
+    __shared__ float lns[32];
+    __shared__ int nonempty[32];
+    const long long bh = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int a = blockIdx.x * 8 + warp;
+    for (int i = threadIdx.x; i < 8 * D; i += 256) {
+        const int w = i / D, e = i % D;
+        const int aa = blockIdx.x * 8 + w;
+        qs[w][e] = aa < Cq ? cq[(bh * Cq + aa) * D + e] : 0.f;
+    }
+    for (int j0 = 0; j0 < Ck; j0 += 32) {
+        __syncthreads();
+        for (int i = threadIdx.x; i < 32 * D; i += 256) {
+            const int jj = i / D, e = i % D;
+            ks[jj][e] = j0 + jj < Ck ? ck[(bh * Ck + j0 + jj) * D + e] : 0.f;
+        }
+        if (threadIdx.x < 32) {
+            const int j = j0 + threadIdx.x;
+            const int sz = j < Ck ? size_k[bh * Ck + j] : 0;
+            nonempty[threadIdx.x] = sz > 0;
+            lns[threadIdx.x] = sz > 0 ? logf((float)sz) : 0.f;
+        }
+        __syncthreads();
+        const int j = j0 + lane;
+        if (a < Cq && j < Ck) {
+            float s = 0.f;
+#pragma unroll 8
+            for (int e = 0; e < D; ++e) s = fmaf(qs[warp][e], ks[lane][e], s);
+            logits[(bh * Cq + a) * Ck + j] = nonempty[lane] ? fmaf(s, scale, lns[lane]) : -INFINITY;
+        }
+    }
+}
+
+// A selected key cluster without keys is dropped from the selection.
+__global__ void __launch_bounds__(256) prune_empty_kernel(uint8_t *__restrict__ sel,
+                                                          const int32_t *__restrict__ size_k,
+                                                          long long rows, int Cq, int Ck) {
+    const long long total = rows * Ck;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const long long row = i / Ck;
+        const int j = (int)(i - row * Ck);
+        if (size_k[(row / Cq) * Ck + j] <= 0) sel[i] = 0;
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// Query tiles of a head (one warp per head): cluster a's rows [qstart, qstart + qsize) are cut
+// into tiles of up to 128 rows, in cluster order; unused slots up to U get q_rows = 0.
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) build_units_kernel(const int32_t *__restrict__ qstart,
+                                                          const int32_t *__restrict__ qsize,
+                                                          long long BH, int Cq, int U,
+                                                          int2 *__restrict__ units) {
+    const int lane = threadIdx.x & 31;
+    const long long bh = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (bh >= BH) return;
+    int2 *ub = units + bh * U;
+    int base = 0;
+    bool bad = false;
+    for (int a0 = 0; a0 < Cq; a0 += 32) {
+        const int a = a0 + lane;
+        const int sz = a < Cq ? max(qsize[bh * Cq + a], 0) : 0;
+        const int st = a < Cq ? qstart[bh * Cq + a] : 0;
+        const int nt = (sz + 127) >> 7;
+        int incl = nt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        const int off = base + incl - nt;
+        for (int t = 0; t < nt; ++t) {
+            const int u = off + t;
+            if (u < U)
+                ub[u] = make_int2(st + 128 * t, (min(128, sz - 128 * t) << 16) | a);
+            else
+                bad = true;
+        }
+        base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    for (int u = base + lane; u < U; u += 32) ub[u] = make_int2(0, 0);
+    if (bad) atomicOr(&g_bsa_device_error, BSA_DEVERR_BOUNDS);
+}
+
+// ------------------------------------------------------------------------------------------
+// Key tiles of each (head, query cluster) row (one warp per row): the selected non-empty key
+// clusters in id order; clusters that are adjacent in the permuted order (nothing but empty
+// clusters between them) merge into one run, and each run is cut into tiles of up to 128 keys,
+// so only the last tile of a run is partial.  Entry = (first row << 7) | (valid keys - 1).
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) build_key_tiles_kernel(
+    const uint8_t *__restrict__ sel, const int32_t *__restrict__ kstart,
+    const int32_t *__restrict__ ksize, long long rows, int Cq, int Ck, int tstride,
+    int32_t *__restrict__ tiles, int32_t *__restrict__ tcnt) {
+    const int lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (row >= rows) return;
+    const long long bh = row / Cq;
+    const uint8_t *sr = sel + row * Ck;
+    int32_t *out = tiles + row * tstride;
+    int pos = 0, rs = 0, re = 0;  // the open run of keys [rs, re)
+    bool overflow = false;
+    auto flush = [&]() {
+        if (re > rs) {
+            const int nt = (re - rs + 127) >> 7;
+            for (int t = lane; t < nt; t += 32) {
+                const int r0 = rs + 128 * t;
+                if (pos + t < tstride) out[pos + t] = (r0 << 7) | (min(128, re - r0) - 1);
+            }
+            if (pos + nt > tstride) overflow = true;
+            pos = min(pos + nt, tstride);
+        }
+    };
+    for (int j0 = 0; j0 < Ck; j0 += 32) {
+        const int j = j0 + lane;
+        int st = 0, sz = 0;
+        if (j < Ck && sr[j]) {
+            st = kstart[bh * Ck + j];
+            sz = ksize[bh * Ck + j];
+        }
+        uint32_t b = __ballot_sync(0xffffffffu, sz > 0);
+        while (b) {  // warp-uniform
+            const int src = __ffs(b) - 1;
+            b &= b - 1;
+            const int s = __shfl_sync(0xffffffffu, st, src);
+            const int len = __shfl_sync(0xffffffffu, sz, src);
+            if (re > rs && s == re) {
+                re += len;
+            } else {
+                flush();
+                rs = s;
+                re = s + len;
+            }
+        }
+    }
+    flush();
+    if (lane == 0) {
+        tcnt[row] = pos;
+        if (overflow) atomicOr(&g_bsa_device_error, BSA_DEVERR_BOUNDS);
+    }
+}
+
+// dst[bh, s, :] = src[bh, perm[bh, s], :], token rows moved as 16-byte vectors.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4 *__restrict__ src,
+                                                          uint4 *__restrict__ dst,
+                                                          const int32_t *__restrict__ perm,
+                                                          long long rows, int N, int vec) {
+    const long long total = rows * vec;
+    for (long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x; x < total;
+         x += (long long)gridDim.x * blockDim.x) {
+        const long long row = x / vec;
+        const int c = (int)(x - row * vec);
+        const long long bh = row / N;
+        const int n = min(max(perm[row], 0), N - 1);
+        dst[x] = src[(bh * N + n) * vec + c];
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// host side
+// ------------------------------------------------------------------------------------------
+static unsigned grid_for(long long work, int per_block, int num_sms) {
+    long long g = (work + per_block - 1) / per_block;
+    const long long cap = (long long)num_sms * 16;
+    if (g > cap) g = cap;
+    return (unsigned)(g > 0 ? g : 1);
+}
+
+cudaError_t kmeans_lloyd(const void *x, float *cent, int32_t *assign, int32_t *perm,
+                         int32_t *cstart, int32_t *csize, long long BH, int N, int d, int C,
+                         int iters, cudaStream_t st) {
+    const dim3 ga((unsigned)((N + 255) / 256), (unsigned)BH);
+    const dim3 gu((unsigned)C, (unsigned)BH);
+    const size_t sort_smem = (size_t)9 * C * sizeof(int32_t);
+    const auto *xb = reinterpret_cast<const __nv_bfloat16 *>(x);
+    for (int it = 0;; ++it) {
+        if (d == 128)
+            kmeans_assign_kernel<128><<<ga, 256, 0, st>>>(xb, cent, assign, N, C);
+        else
+            kmeans_assign_kernel<64><<<ga, 256, 0, st>>>(xb, cent, assign, N, C);
+        cluster_sort_kernel<<<(unsigned)BH, 256, sort_smem, st>>>(assign, N, C, perm, cstart, csize);
+        if (it == iters) break;
+        if (d == 128)
+            kmeans_update_kernel<128><<<gu, 512, 0, st>>>(xb, perm, cstart, csize, cent, N, C);
+        else
+            kmeans_update_kernel<64><<<gu, 512, 0, st>>>(xb, perm, cstart, csize, cent, N, C);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t cluster_sort(const int32_t *assign, long long BH, int N, int C, int32_t *perm,
+                         int32_t *cstart, int32_t *csize, cudaStream_t st) {
+    cluster_sort_kernel<<<(unsigned)BH, 256, (size_t)9 * C * sizeof(int32_t), st>>>(
+        assign, N, C, perm, cstart, csize);
+    return cudaGetLastError();
+}
+
+cudaError_t centroid_logits(const float *cq, const float *ck, const int32_t *size_k,
+                            float *logits, long long BH, int Cq, int Ck, int d, float scale,
+                            cudaStream_t st) {
+    const dim3 g((unsigned)((Cq + 7) / 8), (unsigned)BH);
+    if (d == 128)
+        centroid_logits_kernel<128><<<g, 256, 0, st>>>(cq, ck, size_k, logits, Cq, Ck, scale);
+    else
+        centroid_logits_kernel<64><<<g, 256, 0, st>>>(cq, ck, size_k, logits, Cq, Ck, scale);
+    return cudaGetLastError();
+}
+
+cudaError_t prune_empty(uint8_t *sel, const int32_t *size_k, long long BH, int Cq, int Ck,
+                        int num_sms, cudaStream_t st) {
+    const long long rows = BH * Cq;
+    prune_empty_kernel<<<grid_for(rows * Ck, 256, num_sms), 256, 0, st>>>(sel, size_k, rows, Cq, Ck);
+    return cudaGetLastError();
+}
+
+cudaError_t build_cluster_tables(const uint8_t *sel, const int32_t *qstart, const int32_t *qsize,
+                                 const int32_t *kstart, const int32_t *ksize, long long BH,
+                                 int Cq, int Ck, int U, int tstride, int2 *units, int32_t *tiles,
+                                 int32_t *tcnt, cudaStream_t st) {
+    build_units_kernel<<<(unsigned)((BH + 7) / 8), 256, 0, st>>>(qstart, qsize, BH, Cq, U, units);
+    const long long rows = BH * Cq;
+    build_key_tiles_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(sel, kstart, ksize, rows, Cq,
+                                                                       Ck, tstride, tiles, tcnt);
+    return cudaGetLastError();
+}
+
+cudaError_t gather_rows(const void *src, const int32_t *perm, void *dst, long long BH, int N,
+                        int d, int num_sms, cudaStream_t st) {
+    const int vec = d / 8;
+    const long long rows = BH * N;
+    gather_rows_kernel<<<grid_for(rows * vec, 256, num_sms), 256, 0, st>>>(
+        reinterpret_cast<const uint4 *>(src), reinterpret_cast<uint4 *>(dst), perm, rows, N, vec);
+    return cudaGetLastError();
+}
+
+}  // namespace bsa
+
+// ------------------------------------------------------------------------------------------
+// C ABI
+// ------------------------------------------------------------------------------------------
+namespace {
+
+size_t round256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+// Carves the caller's workspace.  Every region starts on a 256-byte boundary.
+struct ClusterWorkspace {
+    unsigned int *counter;
+    int32_t *perm_q, *perm_k, *qstart, *qsize, *kstart, *ksize, *tiles, *tcnt;
+    int2 *units;
+    void *qp, *kp, *vp;
+    // the full path only: assignments, centroid scores (then the selection's id lists) and counts
+    int32_t *assign_q, *assign_k, *sel_cnt;
+    float *logits;
+    int U, tstride;
+};
+
+size_t cluster_workspace(int B, int H, int N, int d, int Cq, int Ck, bool full, void *base,
+                         ClusterWorkspace *w) {
+    const size_t BH = (size_t)B * H;
+    const int nbt = (N + 127) / 128;
+    const int U = nbt + Cq, tstride = nbt + Ck;
+    size_t off = 0;
+    uint8_t *p = reinterpret_cast<uint8_t *>(base);
+    auto take = [&](size_t bytes) -> void * {
+        void *r = p ? p + off : nullptr;
+        off += round256(bytes);
+        return r;
+    };
+    ClusterWorkspace t;
+    t.counter = (unsigned int *)take(kAttnWorkspaceBytes);
+    t.perm_q = (int32_t *)take(BH * N * 4);
+    t.perm_k = (int32_t *)take(BH * N * 4);
+    t.qstart = (int32_t *)take(BH * Cq * 4);
+    t.qsize = (int32_t *)take(BH * Cq * 4);
+    t.kstart = (int32_t *)take(BH * Ck * 4);
+    t.ksize = (int32_t *)take(BH * Ck * 4);
+    t.tiles = (int32_t *)take(BH * Cq * (size_t)tstride * 4);
+    t.tcnt = (int32_t *)take(BH * Cq * 4);
+    t.units = (int2 *)take(BH * (size_t)U * 8);
+    t.qp = take(BH * N * (size_t)d * 2);
+    t.kp = take(BH * N * (size_t)d * 2);
+    t.vp = take(BH * N * (size_t)d * 2);
+    t.assign_q = t.assign_k = t.sel_cnt = nullptr;
+    t.logits = nullptr;
+    if (full) {
+        t.assign_q = (int32_t *)take(BH * N * 4);
+        t.assign_k = (int32_t *)take(BH * N * 4);
+        t.logits = (float *)take(BH * Cq * (size_t)Ck * 4);
+        t.sel_cnt = (int32_t *)take(BH * Cq * 4);
+    }
+    t.U = U;
+    t.tstride = tstride;
+    if (w) *w = t;
+    return off;
+}
+
+bool clusters_ok(int C) { return C >= 1 && C <= bsa::kMaxClusters; }
+
+// Shape checks shared by the cluster entry points.
+sa_status cluster_shape(int B, int H, int N, int d, int Cq, int Ck) {
+    if (!shape_ok(B, H, N) || !clusters_ok(Cq) || !clusters_ok(Ck)) return SA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return SA_ERR_UNSUPPORTED;
+    if (N >= bsa::kMaxVarlenN) return SA_ERR_UNSUPPORTED;
+    const long long units = (long long)B * H * ((N + 127) / 128 + Cq);
+    if (units > 0x7FFFFFFFLL) return SA_ERR_UNSUPPORTED;
+    return SA_OK;
+}
+
+// Tables, permuted tensors and the attention, from the two permutations and the selection.
+sa_status cluster_attention_tail(const void *q, const void *k, const void *v, void *o,
+                                 const uint8_t *sel, const ClusterWorkspace &w, int B, int H,
+                                 int N, int d, int Cq, int Ck, float scale, int dev,
+                                 cudaStream_t st) {
+    const long long BH = (long long)B * H;
+    const int sms = num_sms(dev);
+    cudaError_t e = bsa::build_cluster_tables(sel, w.qstart, w.qsize, w.kstart, w.ksize, BH, Cq, Ck,
+                                              w.U, w.tstride, w.units, w.tiles, w.tcnt, st);
+    if (e == cudaSuccess) e = bsa::gather_rows(q, w.perm_q, w.qp, BH, N, d, sms, st);
+    if (e == cudaSuccess) e = bsa::gather_rows(k, w.perm_k, w.kp, BH, N, d, sms, st);
+    if (e == cudaSuccess) e = bsa::gather_rows(v, w.perm_k, w.vp, BH, N, d, sms, st);
+    if (e != cudaSuccess) return SA_ERR_CUDA;
+    CUtensorMap tq, tk, tv;
+    if (!make_tmap(&tq, w.qp, BH, N, d, 128) || !make_tmap(&tk, w.kp, BH, N, d, 128) ||
+        !make_tmap(&tv, w.vp, BH, N, d, 128))
+        return SA_ERR_CUDA;
+    return from_cuda(bsa::attn_varlen_fwd(tq, tk, tv, w.units, w.U, w.tiles, w.tcnt, w.tstride,
+                                          w.perm_q, o, BH, N, Cq, d, resolve_scale(scale, d),
+                                          g_wait_ns, sms, w.counter, st));
+}
+
+// Centroid scores, top-p and the removal of empty clusters; logits doubles as the id list.
+cudaError_t centroid_select(const float *cq, const float *ck, const int32_t *size_k, long long BH,
+                            int Cq, int Ck, int d, float topp, float scale, uint8_t *sel,
+                            float *logits, int32_t *sel_cnt, int sms, cudaStream_t st) {
+    cudaError_t e = bsa::centroid_logits(cq, ck, size_k, logits, BH, Cq, Ck, d, scale, st);
+    if (e == cudaSuccess)
+        e = bsa::select_rows(logits, BH * Cq, Ck, 0, topp, sel,
+                             reinterpret_cast<int32_t *>(logits), sel_cnt, st);
+    if (e == cudaSuccess) e = bsa::prune_empty(sel, size_k, BH, Cq, Ck, sms, st);
+    return e;
+}
+
+}  // namespace
+
+extern "C" sa_status sa_kmeans(const void *x, float *cent, int32_t *assign, int32_t *perm,
+                               int32_t *cstart, int32_t *csize, int B, int H, int N, int d, int C,
+                               int iters, void *stream) {
+    if (!x || !cent || !assign || !perm || !cstart || !csize) return SA_ERR_INVALID_ARG;
+    if (!shape_ok(B, H, N) || !clusters_ok(C) || iters < 0) return SA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return SA_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned16(cent) || !aligned4(assign) || !aligned4(perm) ||
+        !aligned4(cstart) || !aligned4(csize))
+        return SA_ERR_INVALID_ARG;
+    int dev;
+    if (!select_device(assign, &dev)) return SA_ERR_INVALID_ARG;
+    return from_cuda(bsa::kmeans_lloyd(x, cent, assign, perm, cstart, csize, (long long)B * H, N, d,
+                                       C, iters, (cudaStream_t)stream));
+}
+
+extern "C" sa_status sa_cluster_sort(const int32_t *assign, int B, int H, int N, int C,
+                                     int32_t *perm, int32_t *cstart, int32_t *csize,
+                                     void *stream) {
+    if (!assign || !perm || !cstart || !csize) return SA_ERR_INVALID_ARG;
+    if (!shape_ok(B, H, N) || !clusters_ok(C)) return SA_ERR_INVALID_ARG;
+    if (!aligned4(assign) || !aligned4(perm) || !aligned4(cstart) || !aligned4(csize))
+        return SA_ERR_INVALID_ARG;
+    int dev;
+    if (!select_device(perm, &dev)) return SA_ERR_INVALID_ARG;
+    return from_cuda(bsa::cluster_sort(assign, (long long)B * H, N, C, perm, cstart, csize,
+                                       (cudaStream_t)stream));
+}
+
+extern "C" size_t sa_centroid_topp_workspace_bytes(int B, int H, int Cq, int Ck) {
+    if (B <= 0 || H <= 0 || Cq <= 0 || Ck <= 0) return 0;
+    const size_t BH = (size_t)B * H;
+    return round256(BH * Cq * (size_t)Ck * 4) + round256(BH * Cq * 4);
+}
+
+extern "C" sa_status sa_centroid_topp(const float *cq, const float *ck, const int32_t *size_k,
+                                      int B, int H, int Cq, int Ck, int d, float topp, float scale,
+                                      uint8_t *sel, void *workspace, size_t workspace_bytes,
+                                      void *stream) {
+    if (!cq || !ck || !size_k || !sel || !workspace) return SA_ERR_INVALID_ARG;
+    if (!shape_ok(B, H, 1) || !clusters_ok(Cq) || !clusters_ok(Ck)) return SA_ERR_INVALID_ARG;
+    if (!(topp >= 0.f && topp <= 1.f) || isnan(scale)) return SA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return SA_ERR_UNSUPPORTED;
+    if (workspace_bytes < sa_centroid_topp_workspace_bytes(B, H, Cq, Ck) || !aligned16(workspace))
+        return SA_ERR_INVALID_ARG;
+    if (!aligned4(cq) || !aligned4(ck) || !aligned4(size_k)) return SA_ERR_INVALID_ARG;
+    int dev;
+    if (!select_device(sel, &dev)) return SA_ERR_INVALID_ARG;
+    const long long BH = (long long)B * H;
+    float *logits = reinterpret_cast<float *>(workspace);
+    int32_t *cnt = reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(workspace) +
+                                               round256((size_t)BH * Cq * Ck * 4));
+    return from_cuda(centroid_select(cq, ck, size_k, BH, Cq, Ck, d, topp, resolve_scale(scale, d),
+                                     sel, logits, cnt, num_sms(dev), (cudaStream_t)stream));
+}
+
+extern "C" size_t sa_cluster_attn_workspace_bytes(int B, int H, int N, int d, int Cq, int Ck) {
+    if (B <= 0 || H <= 0 || N <= 0 || d <= 0 || Cq <= 0 || Ck <= 0) return 0;
+    return cluster_workspace(B, H, N, d, Cq, Ck, false, nullptr, nullptr);
+}
+
+extern "C" sa_status sa_cluster_attn_fwd(const void *q, const void *k, const void *v, void *o,
+                                         const int32_t *assign_q, const int32_t *assign_k,
+                                         const uint8_t *sel, int B, int H, int N, int d, int Cq,
+                                         int Ck, float scale, void *workspace,
+                                         size_t workspace_bytes, void *stream) {
+    if (!q || !k || !v || !o || !assign_q || !assign_k || !sel || !workspace)
+        return SA_ERR_INVALID_ARG;
+    const sa_status s = cluster_shape(B, H, N, d, Cq, Ck);
+    if (s != SA_OK) return s;
+    if (isnan(scale)) return SA_ERR_INVALID_ARG;
+    if (workspace_bytes < sa_cluster_attn_workspace_bytes(B, H, N, d, Cq, Ck) ||
+        !aligned16(workspace))
+        return SA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(assign_q) ||
+        !aligned4(assign_k))
+        return SA_ERR_INVALID_ARG;
+    int dev;
+    if (!select_device(o, &dev)) return SA_ERR_INVALID_ARG;
+    const cudaStream_t st = (cudaStream_t)stream;
+    ClusterWorkspace w;
+    cluster_workspace(B, H, N, d, Cq, Ck, false, workspace, &w);
+    const long long BH = (long long)B * H;
+    cudaError_t e = bsa::cluster_sort(assign_q, BH, N, Cq, w.perm_q, w.qstart, w.qsize, st);
+    if (e == cudaSuccess) e = bsa::cluster_sort(assign_k, BH, N, Ck, w.perm_k, w.kstart, w.ksize, st);
+    if (e != cudaSuccess) return SA_ERR_CUDA;
+    return cluster_attention_tail(q, k, v, o, sel, w, B, H, N, d, Cq, Ck, scale, dev, st);
+}
+
+extern "C" size_t sa_svg2_workspace_bytes(int B, int H, int N, int d, int Cq, int Ck) {
+    if (B <= 0 || H <= 0 || N <= 0 || d <= 0 || Cq <= 0 || Ck <= 0) return 0;
+    return cluster_workspace(B, H, N, d, Cq, Ck, true, nullptr, nullptr);
+}
+
+extern "C" sa_status sa_svg2_attn_fwd(const void *q, const void *k, const void *v, void *o,
+                                      float *cent_q, float *cent_k, int B, int H, int N, int d,
+                                      int Cq, int Ck, int iters, float topp, float scale,
+                                      uint8_t *sel, void *workspace, size_t workspace_bytes,
+                                      void *stream) {
+    if (!q || !k || !v || !o || !cent_q || !cent_k || !sel || !workspace) return SA_ERR_INVALID_ARG;
+    const sa_status s = cluster_shape(B, H, N, d, Cq, Ck);
+    if (s != SA_OK) return s;
+    if (iters < 0 || !(topp >= 0.f && topp <= 1.f) || isnan(scale)) return SA_ERR_INVALID_ARG;
+    if (workspace_bytes < sa_svg2_workspace_bytes(B, H, N, d, Cq, Ck) || !aligned16(workspace))
+        return SA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(cent_q) ||
+        !aligned16(cent_k))
+        return SA_ERR_INVALID_ARG;
+    int dev;
+    if (!select_device(o, &dev)) return SA_ERR_INVALID_ARG;
+    const cudaStream_t st = (cudaStream_t)stream;
+    ClusterWorkspace w;
+    cluster_workspace(B, H, N, d, Cq, Ck, true, workspace, &w);
+    const long long BH = (long long)B * H;
+    cudaError_t e = bsa::kmeans_lloyd(q, cent_q, w.assign_q, w.perm_q, w.qstart, w.qsize, BH, N, d,
+                                      Cq, iters, st);
+    if (e == cudaSuccess)
+        e = bsa::kmeans_lloyd(k, cent_k, w.assign_k, w.perm_k, w.kstart, w.ksize, BH, N, d, Ck,
+                              iters, st);
+    if (e == cudaSuccess)
+        e = centroid_select(cent_q, cent_k, w.ksize, BH, Cq, Ck, d, topp, resolve_scale(scale, d),
+                            sel, w.logits, w.sel_cnt, num_sms(dev), st);
+    if (e != cudaSuccess) return SA_ERR_CUDA;
+    return cluster_attention_tail(q, k, v, o, sel, w, B, H, N, d, Cq, Ck, scale, dev, st);
+}

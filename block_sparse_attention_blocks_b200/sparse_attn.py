@@ -39,6 +39,19 @@ _Z = ctypes.c_size_t
 lib.sa_squad_workspace_bytes.argtypes = [_I, _I, _I, _I]
 lib.sa_squad_workspace_bytes.restype = _Z
 lib.sa_squad_attn_fwd.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _Z, _P]
+lib.sa_kmeans.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]
+lib.sa_cluster_sort.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P, _P]
+lib.sa_centroid_topp_workspace_bytes.argtypes = [_I, _I, _I, _I]
+lib.sa_centroid_topp_workspace_bytes.restype = _Z
+lib.sa_centroid_topp.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _F, _F, _P, _P, _Z, _P]
+lib.sa_cluster_attn_workspace_bytes.argtypes = [_I, _I, _I, _I, _I, _I]
+lib.sa_cluster_attn_workspace_bytes.restype = _Z
+lib.sa_cluster_attn_fwd.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _Z,
+                                    _P]
+lib.sa_svg2_workspace_bytes.argtypes = [_I, _I, _I, _I, _I, _I]
+lib.sa_svg2_workspace_bytes.restype = _Z
+lib.sa_svg2_attn_fwd.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _P, _P,
+                                 _Z, _P]
 lib.sa_block_sparse_attn_fwd.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _Z, _P]
 lib.sa_dense_attn_fwd.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _Z, _P]
 lib.sa_attn_workspace_bytes.argtypes = []
@@ -51,7 +64,8 @@ lib.sa_probe_bounded_wait.argtypes = [_P]
 lib.sa_num_blocks.argtypes = [_I, _I]
 for _f in (lib.sa_pool_blocks, lib.sa_select_mask_topk_topp, lib.sa_select_from_logits,
            lib.sa_pool_select_topk_topp, lib.sa_block_scores, lib.sa_static_mask,
-           lib.sa_squad_attn_fwd,
+           lib.sa_squad_attn_fwd, lib.sa_kmeans, lib.sa_cluster_sort, lib.sa_centroid_topp,
+           lib.sa_cluster_attn_fwd, lib.sa_svg2_attn_fwd,
            lib.sa_block_sparse_attn_fwd, lib.sa_dense_attn_fwd, lib.sa_get_device_error,
            lib.sa_set_wait_limit_ns, lib.sa_probe_bounded_wait, lib.sa_num_blocks):
     _f.restype = _I
@@ -261,6 +275,105 @@ def squad_attn_fwd(q, k, v, w: int, scale: float | None = None, o=None):
                                  float(scale or 0.0), _ptr(ws), ws.numel(), _stream(q.device)),
            "sa_squad_attn_fwd")
     return o
+
+
+def kmeans(x, cent, iters: int):
+    """Lloyd k-means of the token rows of every head, from the centroids `cent` [B, H, C, d]
+    fp32, which are overwritten with the result (SVG2 section A, warm-started from a cache as in
+    section C).  x: [B, H, N, d] bf16.  Returns (assign [B, H, N], perm [B, H, N], cstart
+    [B, H, C], csize [B, H, C]) int32: the final assignment, and the stable order of the tokens
+    by cluster (cluster c is perm[cstart[c] : cstart[c] + csize[c]])."""
+    _need(x, "x", torch.bfloat16, 4)
+    _need(cent, "cent", torch.float32, 4)
+    B, H, N, d = x.shape
+    C = cent.shape[2]
+    if tuple(cent.shape) != (B, H, C, d):
+        raise ValueError("cent must be [B, H, C, d]")
+    assign = torch.empty(B, H, N, device=x.device, dtype=torch.int32)
+    perm = torch.empty_like(assign)
+    cstart = torch.empty(B, H, C, device=x.device, dtype=torch.int32)
+    csize = torch.empty_like(cstart)
+    _check(lib.sa_kmeans(_ptr(x), _ptr(cent), _ptr(assign), _ptr(perm), _ptr(cstart), _ptr(csize),
+                         B, H, N, d, C, int(iters), _stream(x.device)), "sa_kmeans")
+    return assign, perm, cstart, csize
+
+
+def cluster_sort(assign, C: int):
+    """Stable order of the tokens by cluster id: (perm [B, H, N], cstart [B, H, C], csize
+    [B, H, C]) int32 from assign [B, H, N] int32 ids in [0, C)."""
+    _need(assign, "assign", torch.int32, 3)
+    B, H, N = assign.shape
+    perm = torch.empty_like(assign)
+    cstart = torch.empty(B, H, C, device=assign.device, dtype=torch.int32)
+    csize = torch.empty_like(cstart)
+    _check(lib.sa_cluster_sort(_ptr(assign), B, H, N, int(C), _ptr(perm), _ptr(cstart),
+                               _ptr(csize), _stream(assign.device)), "sa_cluster_sort")
+    return perm, cstart, csize
+
+
+def centroid_topp(cq, ck, size_k, topp: float, scale: float | None = None):
+    """Centroid top-p (SVG2 section B): sel [B, H, Cq, Ck] uint8, the key clusters each query
+    cluster takes.  cq [B, H, Cq, d], ck [B, H, Ck, d] fp32 centroids; size_k [B, H, Ck] int32
+    key cluster sizes."""
+    _need(cq, "cq", torch.float32, 4)
+    _need(ck, "ck", torch.float32, 4)
+    _need(size_k, "size_k", torch.int32, 3)
+    B, H, Cq, d = cq.shape
+    Ck = ck.shape[2]
+    sel = torch.empty(B, H, Cq, Ck, device=cq.device, dtype=torch.uint8)
+    nbytes = int(lib.sa_centroid_topp_workspace_bytes(B, H, Cq, Ck))
+    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=cq.device)
+    _check(lib.sa_centroid_topp(_ptr(cq), _ptr(ck), _ptr(size_k), B, H, Cq, Ck, d, float(topp),
+                                float(scale or 0.0), _ptr(sel), _ptr(ws), ws.numel(),
+                                _stream(cq.device)), "sa_centroid_topp")
+    return sel
+
+
+def cluster_attn_fwd(q, k, v, assign_q, assign_k, sel, scale: float | None = None, o=None):
+    """Attention of each query token over the keys of the key clusters its query cluster
+    selected -> O [B, H, N, d] bf16.  assign_q, assign_k [B, H, N] int32 cluster ids; sel
+    [B, H, Cq, Ck] uint8."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, torch.bfloat16, 4)
+    _need(assign_q, "assign_q", torch.int32, 3)
+    _need(assign_k, "assign_k", torch.int32, 3)
+    _need(sel, "sel", torch.uint8, 4)
+    B, H, N, d = q.shape
+    Cq, Ck = sel.shape[2], sel.shape[3]
+    o = o if o is not None else torch.empty_like(q)
+    _need(o, "o", torch.bfloat16, 4)
+    nbytes = int(lib.sa_cluster_attn_workspace_bytes(B, H, N, d, Cq, Ck))
+    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    _check(lib.sa_cluster_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(assign_q),
+                                   _ptr(assign_k), _ptr(sel), B, H, N, d, Cq, Ck,
+                                   float(scale or 0.0), _ptr(ws), ws.numel(), _stream(q.device)),
+           "sa_cluster_attn_fwd")
+    return o
+
+
+def svg2_attn_fwd(q, k, v, cent_q, cent_k, iters: int, topp: float, scale: float | None = None,
+                  o=None, sel=None, workspace=None):
+    """The semantic-aware permutation path of SVG2: k-means of Q and of K from the centroid
+    cache cent_q [B, H, Cq, d] / cent_k [B, H, Ck, d] fp32 (updated in place), centroid top-p,
+    attention over the selected clusters.  Returns (O [B, H, N, d] bf16, sel [B, H, Cq, Ck])."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, torch.bfloat16, 4)
+    _need(cent_q, "cent_q", torch.float32, 4)
+    _need(cent_k, "cent_k", torch.float32, 4)
+    B, H, N, d = q.shape
+    Cq, Ck = cent_q.shape[2], cent_k.shape[2]
+    o = o if o is not None else torch.empty_like(q)
+    sel = sel if sel is not None else torch.empty(B, H, Cq, Ck, device=q.device, dtype=torch.uint8)
+    _need(o, "o", torch.bfloat16, 4)
+    _need(sel, "sel", torch.uint8, 4)
+    nbytes = int(lib.sa_svg2_workspace_bytes(B, H, N, d, Cq, Ck))
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    _check(lib.sa_svg2_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(cent_q), _ptr(cent_k),
+                                B, H, N, d, Cq, Ck, int(iters), float(topp), float(scale or 0.0),
+                                _ptr(sel), _ptr(workspace), workspace.numel(), _stream(q.device)),
+           "sa_svg2_attn_fwd")
+    return o, sel
 
 
 def _host_pipeline(q, k, v, bs, topk, topp, scale, dev, out, chunks):

@@ -145,6 +145,77 @@ sa_status sa_squad_attn_fwd(const void *q, const void *k, const void *v, void *o
                             size_t workspace_bytes, void *stream);
 
 /*
+ * Semantic-aware permutation with centroid top-p (Sparse VideoGen2, method sections A-C).
+ * Cluster counts C, Cq, Ck are in [1, 1024]; d in {64, 128}; N < 2^24 for the attention calls.
+ *
+ * sa_kmeans: Lloyd's algorithm on the token rows of every head of x [B, H, N, d] bf16, from the
+ *   centroids in cent [B, H, C, d] fp32 (16-byte aligned; a centroid cache, overwritten with the
+ *   result).  `iters` update steps, each the mean of the rows assigned to a cluster (a cluster
+ *   with no rows keeps its centroid), then a final assignment to the updated centroids: nearest
+ *   centroid by squared Euclidean distance in fp32, the lower index on a tie.  Outputs (int32):
+ *   assign [B, H, N] the final cluster of each token; perm [B, H, N] the tokens in order of
+ *   cluster, ascending within a cluster; cstart, csize [B, H, C] where each cluster's tokens sit
+ *   in perm.  Cluster sums run in token order, so results repeat bit for bit.
+ */
+sa_status sa_kmeans(const void *x, float *cent, int32_t *assign, int32_t *perm, int32_t *cstart,
+                    int32_t *csize, int B, int H, int N, int d, int C, int iters, void *stream);
+
+/*
+ * The stable order of the tokens by cluster id (the permutation of section A) alone:
+ * assign [B, H, N] int32 ids in [0, C) (others are clamped and flagged in the device error word)
+ * -> perm, cstart, csize as for sa_kmeans.
+ */
+sa_status sa_cluster_sort(const int32_t *assign, int B, int H, int N, int C, int32_t *perm,
+                          int32_t *cstart, int32_t *csize, void *stream);
+
+/*
+ * Centroid top-p (section B).  For query cluster a of head (b, h), key cluster j is estimated to
+ * receive the share  w[a, j] = size_k[j] exp(scale cq[a] . ck[j]) / sum_j' (same)  of the
+ * attention (each key stands in for by its centroid).  Key clusters are ranked by w descending
+ * (the lower id first on a tie) and taken until the cumulative share reaches topp; topp <= 0
+ * takes none, topp >= 1 every cluster with keys; a cluster with size_k = 0 is never taken.
+ * The decision runs in fp32 (the top-p kernel of the block path), so clusters whose share lies
+ * within ~1e-5 of the cut may differ from an exact evaluation.
+ * cq [B, H, Cq, d], ck [B, H, Ck, d] fp32; size_k [B, H, Ck] int32; sel [B, H, Cq, Ck] uint8
+ * 0/1, written.  workspace: sa_centroid_topp_workspace_bytes() bytes, 16-byte aligned.
+ */
+size_t sa_centroid_topp_workspace_bytes(int B, int H, int Cq, int Ck);
+sa_status sa_centroid_topp(const float *cq, const float *ck, const int32_t *size_k, int B, int H,
+                           int Cq, int Ck, int d, float topp, float scale, uint8_t *sel,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Attention over selected clusters (section C):
+ *   O[b,h,t,:] = sum over keys s with sel[b,h,assign_q[t],assign_k[s]] != 0 of
+ *                softmax_s(scale Q[t] . K[s]) V[s];   zero when the selection is empty.
+ * Q is permuted by query cluster and K, V by key cluster (each cluster contiguous); every query
+ * tile of up to 128 rows of one cluster runs over key tiles of up to 128 consecutive permuted
+ * keys covering exactly the selected clusters (adjacent clusters share tiles), on the tensor
+ * cores; outputs go straight back to the original token positions.
+ * q, k, v, o : [B, H, N, d] bf16.  assign_q, assign_k : [B, H, N] int32 in [0, Cq) / [0, Ck).
+ * sel : [B, H, Cq, Ck] uint8, nonzero = selected.  scale <= 0 selects 1/sqrt(d).
+ * workspace : sa_cluster_attn_workspace_bytes() bytes, 16-byte aligned (the permuted tensors,
+ *             the permutations and the tile tables).
+ */
+size_t sa_cluster_attn_workspace_bytes(int B, int H, int N, int d, int Cq, int Ck);
+sa_status sa_cluster_attn_fwd(const void *q, const void *k, const void *v, void *o,
+                              const int32_t *assign_q, const int32_t *assign_k,
+                              const uint8_t *sel, int B, int H, int N, int d, int Cq, int Ck,
+                              float scale, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * The whole SVG2 path: sa_kmeans of Q (into cent_q [B, H, Cq, d]) and of K (into cent_k
+ * [B, H, Ck, d]) with `iters` update steps from the caller's centroid cache, sa_centroid_topp on
+ * the resulting centroids and key cluster sizes (sel [B, H, Cq, Ck] uint8, written), then the
+ * attention of sa_cluster_attn_fwd.  workspace: sa_svg2_workspace_bytes() bytes, 16-byte aligned.
+ */
+size_t sa_svg2_workspace_bytes(int B, int H, int N, int d, int Cq, int Ck);
+sa_status sa_svg2_attn_fwd(const void *q, const void *k, const void *v, void *o, float *cent_q,
+                           float *cent_k, int B, int H, int N, int d, int Cq, int Ck, int iters,
+                           float topp, float scale, uint8_t *sel, void *workspace,
+                           size_t workspace_bytes, void *stream);
+
+/*
  * Selection from caller-provided block scores (the second half of sa_select_mask_topk_topp,
  * exposed for tests that feed hand-made rows).  logits: [B, H, nb, nb] fp32 scores already
  * scaled; the row softmax, ranking, top-k union top-p and outputs are as above.  logits may be

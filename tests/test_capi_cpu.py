@@ -216,3 +216,60 @@ def test_squad_argument_checks(lib):
     assert f(A, A, A, A, 1, 2, 512, 64, 0, 0.0, A2, W, S) == 1
     assert f(A, A, A, A, 1, 2, 512, 64, 64, 0.0, A2, W - 1, S) == 1
     assert f(A, A, A, A, 1, 2, 512, 64, 64, float("nan"), A2, W, S) == 1
+
+
+def test_cluster_entry_point_argument_checks(lib):
+    I, P, F, Z = ctypes.c_int, ctypes.c_void_p, ctypes.c_float, ctypes.c_size_t
+    km = lib.sa_kmeans
+    km.argtypes = [P] * 6 + [I] * 6 + [P]
+    assert km(NUL, A, A, A, A, A, 1, 2, 100, 64, 8, 2, S) == 1
+    assert km(A, A, A, A, A, A, 1, 2, 100, 96, 8, 2, S) == 2          # d
+    assert km(A, A, A, A, A, A, 1, 2, 100, 64, 0, 2, S) == 1          # C < 1
+    assert km(A, A, A, A, A, A, 1, 2, 100, 64, 1025, 2, S) == 1       # C > 1024
+    assert km(A, A, A, A, A, A, 1, 2, 100, 64, 8, -1, S) == 1         # iters
+    assert km(A, MIS, A, A, A, A, 1, 2, 100, 64, 8, 2, S) == 1        # centroids need 16 B
+    cs = lib.sa_cluster_sort
+    cs.argtypes = [P] + [I] * 4 + [P] * 4
+    assert cs(NUL, 1, 1, 10, 4, A, A, A, S) == 1
+    assert cs(A, 1, 1, 10, 4, MIS4, A, A, S) == 1
+
+    lib.sa_centroid_topp_workspace_bytes.restype = Z
+    lib.sa_centroid_topp_workspace_bytes.argtypes = [I] * 4
+    Wt = lib.sa_centroid_topp_workspace_bytes(1, 2, 16, 40)
+    assert Wt >= 2 * 16 * 40 * 4 + 2 * 16 * 4
+    assert lib.sa_centroid_topp_workspace_bytes(0, 2, 16, 40) == 0
+    ct = lib.sa_centroid_topp
+    ct.argtypes = [P] * 3 + [I] * 5 + [F, F, P, P, Z, P]
+    assert ct(NUL, A, A, 1, 2, 16, 40, 64, 0.9, 0.0, A2, A, Wt, S) == 1
+    assert ct(A, A, A, 1, 2, 16, 40, 80, 0.9, 0.0, A2, A, Wt, S) == 2
+    assert ct(A, A, A, 1, 2, 16, 40, 64, 1.5, 0.0, A2, A, Wt, S) == 1
+    assert ct(A, A, A, 1, 2, 16, 40, 64, 0.9, float("nan"), A2, A, Wt, S) == 1
+    assert ct(A, A, A, 1, 2, 16, 40, 64, 0.9, 0.0, A2, A, Wt - 1, S) == 1
+    assert ct(A, A, A, 1, 2, 16, 2000, 64, 0.9, 0.0, A2, A, Wt, S) == 1
+
+    for name in ("sa_cluster_attn_workspace_bytes", "sa_svg2_workspace_bytes"):
+        getattr(lib, name).restype = Z
+        getattr(lib, name).argtypes = [I] * 6
+    Wc = lib.sa_cluster_attn_workspace_bytes(1, 2, 1000, 64, 16, 40)
+    Ws = lib.sa_svg2_workspace_bytes(1, 2, 1000, 64, 16, 40)
+    # three permuted tensors, two permutations, tile tables; the full path adds the assignments
+    # and the centroid scores
+    assert Wc >= 3 * 2 * 1000 * 64 * 2 + 2 * 2 * 1000 * 4 + 2 * 16 * (8 + 40) * 4
+    assert Ws >= Wc + 2 * 2 * 1000 * 4 + 2 * 16 * 40 * 4
+    ca = lib.sa_cluster_attn_fwd
+    ca.argtypes = [P] * 7 + [I] * 6 + [F, P, Z, P]
+    assert ca(NUL, A, A, A, A, A, A, 1, 2, 1000, 64, 16, 40, 0.0, A2, Wc, S) == 1
+    assert ca(A, A, A, A, A, A, A, 1, 2, 1000, 96, 16, 40, 0.0, A2, Wc, S) == 2
+    assert ca(A, A, A, A, A, A, A, 1, 2, 1 << 24, 64, 16, 40, 0.0, A2, Wc, S) == 2  # N limit
+    assert ca(A, A, A, A, A, A, A, 1, 2, 1000, 64, 0, 40, 0.0, A2, Wc, S) == 1
+    assert ca(A, A, A, A, A, A, A, 1, 2, 1000, 64, 16, 40, 0.0, A2, Wc - 1, S) == 1
+    assert ca(A, A, A, A, MIS4, A, A, 1, 2, 1000, 64, 16, 40, 0.0, A2, Wc, S) == 1
+    assert ca(MIS, A, A, A, A, A, A, 1, 2, 1000, 64, 16, 40, 0.0, A2, Wc, S) == 1
+    sv = lib.sa_svg2_attn_fwd
+    sv.argtypes = [P] * 6 + [I] * 7 + [F, F, P, P, Z, P]
+    assert sv(A, A, A, A, A, NUL, 1, 2, 1000, 64, 16, 40, 2, 0.9, 0.0, A, A2, Ws, S) == 1
+    assert sv(A, A, A, A, A, A, 1, 2, 1000, 128, 16, 40, -1, 0.9, 0.0, A, A2, Ws, S) == 1
+    assert sv(A, A, A, A, A, A, 1, 2, 1000, 64, 16, 40, 2, -0.1, 0.0, A, A2, Ws, S) == 1
+    assert sv(A, A, A, A, A, A, 1, 2, 1000, 64, 16, 40, 2, 0.9, 0.0, A, A2, Wc, S) == 1
+    assert sv(A, A, A, A, MIS, A, 1, 2, 1000, 64, 16, 40, 2, 0.9, 0.0, A, A2, Ws, S) == 1
+    assert sv(A, A, A, A, A, A, 1, 2, 1000, 32, 16, 40, 2, 0.9, 0.0, A, A2, Ws, S) == 2
