@@ -499,6 +499,49 @@ def run_gpu(args, w):
                             "each position (SQuad, w = tokens of one frame)"}
         del osq
 
+    # ---------------------------------------------------------------- SVG2 (context, opt-in)
+    svg2 = None
+    if args.svg2 and rank == 0:
+        Cq, Ck = args.svg2_clusters
+        # first centroid cache: the tokens at evenly spaced positions of each head; every later
+        # call starts from the previous call's centroids (the cache of SVG2 section C)
+        cq = q[:, :, torch.linspace(0, N - 1, Cq, device=dev).long(), :].float().contiguous()
+        ck = k[:, :, torch.linspace(0, N - 1, Ck, device=dev).long(), :].float().contiguous()
+        osv = torch.empty_like(q)
+        ws = torch.empty(int(bsa.lib.sa_svg2_workspace_bytes(B, H, N, d, Cq, Ck)),
+                         dtype=torch.uint8, device=dev)
+        _, sel = bsa.svg2_attn_fwd(q, k, v, cq, ck, args.svg2_iters, w.topp, o=osv, workspace=ws)
+        torch.cuda.synchronize(dev)
+        s0, s1, s2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        reps = 5
+        s0.record(stream)
+        for _ in range(reps):
+            bsa.svg2_attn_fwd(q, k, v, cq, ck, args.svg2_iters, w.topp, o=osv, sel=sel,
+                              workspace=ws)
+        s1.record(stream)
+        for _ in range(reps):  # the two k-means alone, from copies of the cache
+            bsa.kmeans(q, cq.clone(), args.svg2_iters)
+            bsa.kmeans(k, ck.clone(), args.svg2_iters)
+        s2.record(stream)
+        torch.cuda.synchronize(dev)
+        err = bsa.device_error()
+        if err:
+            raise RuntimeError(f"device error {err} in the SVG2 timing")
+        # the last call's clusters: its final assignment is the nearest centroid of the cache
+        _, _, _, qsz = bsa.kmeans(q, cq.clone(), 0)
+        _, _, _, ksz = bsa.kmeans(k, ck.clone(), 0)
+        qsz, ksz = qsz.double(), ksz.double()
+        pairs_sv = float(torch.einsum("bha,bhaj,bhj->", qsz, sel.double(), ksz))
+        ms_sv = s0.elapsed_time(s1) / reps
+        f_sv = 4.0 * d * pairs_sv
+        svg2 = {"query_clusters": Cq, "key_clusters": Ck, "kmeans_iters": args.svg2_iters,
+                "topp": w.topp, "ms": ms_sv, "kmeans_ms": s1.elapsed_time(s2) / reps,
+                "density": pairs_sv / float(B * H * N * N),
+                "tflops": f_sv / (ms_sv * 1e-3) / 1e12,
+                "pattern": "k-means of Q and K warm-started from the previous call's centroids, "
+                           "centroid top-p, attention over the selected clusters (SVG2)"}
+        del osv, ws, sel
+
     peaks, peak_src = load_peaks()
     peak_tc = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     peak_hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
@@ -549,6 +592,8 @@ def run_gpu(args, w):
         line["static_pattern"] = static
     if squad:
         line["squad"] = squad
+    if svg2:
+        line["svg2"] = svg2
 
     # ---------------------------------------------------------------- oracle on the host
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -585,6 +630,11 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-static", action="store_true", help="skip the static-pattern timing")
     ap.add_argument("--no-squad", action="store_true", help="skip the SQuad timing")
+    ap.add_argument("--svg2", action="store_true",
+                    help="also time the SVG2 path (k-means, centroid top-p, cluster attention)")
+    ap.add_argument("--svg2-clusters", type=lambda s: tuple(int(x) for x in s.split(",")),
+                    default=(128, 256), help="query,key cluster counts for --svg2")
+    ap.add_argument("--svg2-iters", type=int, default=2, help="k-means update steps for --svg2")
     ap.add_argument("--heads", type=int, default=None,
                     help="run only the first H heads (small cases for profiling; not a bench line)")
     args = ap.parse_args()
