@@ -5,8 +5,9 @@ CPU-baseline leg may import this module.  The CUDA path never imports it, and it
 the CUDA path: the two share nothing but the seeded input generator.
 
 The arithmetic lives in ``oracle.c`` (plain fp64 loops, OpenMP over rows).  This module only
-compiles it, loads it with ctypes and marshals numpy arrays.  Each function cites the passage it
-follows in its C definition.
+compiles it, loads it with ctypes and marshals numpy arrays; each of those functions cites the
+passage it follows in its C definition.  The one exception is the probe-fitted correction at the
+end of this file, whose steps are numpy library calls (SVD, least squares) written out here.
 """
 from __future__ import annotations
 
@@ -294,3 +295,54 @@ def dense_attention(q_bits, k_bits, v_bits, scale: float, rows=None):
     _load().or_dense_attention(_ptr(q), _ptr(k), _ptr(v), N, d, float(scale), _ptr(sb), _ptr(st),
                                len(rows), _ptr(out))
     return out
+
+
+# ---------------------------------------------------------------------------------------------
+# Probe-fitted residual reconstruction (page "Partition the Support, Reconstruct the Residual:
+# Training-Free Sparse Attention for Video Generation and World Models", the abstract and the
+# summary's section 3).  The page gives this step in one sentence: a few exact query rows
+# calibrate, for each call, an affine correction computed from the sparse output, confined to
+# the output subspace the probe residuals span.  The steps below are the plainest reading of it;
+# their library steps are numpy's SVD and least squares.
+# ---------------------------------------------------------------------------------------------
+def probe_fit_correction(o_sparse, probes, exact, rtol: float = 1e-9):
+    """One head of one call.  o_sparse [n, d]: the sparse attention output; probes [m]: probe
+    query rows; exact [m, d]: their exact (dense) attention outputs.
+
+      R  = exact - o_sparse[probes]                the probe residuals
+      Bs = orthonormal basis [d, r] of the row space of R (right singular vectors whose singular
+           value exceeds rtol times the largest)   the observed output subspace
+      A  = argmin || [o_sparse[probes], 1] A - R Bs ||   over A [(d + 1), r]; the minimum-norm
+           solution when the probes leave it underdetermined
+      o  = o_sparse + [o_sparse, 1] A Bs^T         applied to every row
+
+    Returns (o [n, d], Bs [d, r], A [d + 1, r]), float64."""
+    Os = np.asarray(o_sparse, np.float64)
+    n, d = Os.shape
+    P = np.asarray(probes, np.int64).reshape(-1)
+    E = np.asarray(exact, np.float64).reshape(len(P), d)
+    R = E - Os[P]
+    if len(P) == 0 or not np.any(R):
+        return Os.copy(), np.zeros((d, 0)), np.zeros((d + 1, 0))
+    _, s, vt = np.linalg.svd(R, full_matrices=False)
+    r = int(np.count_nonzero(s > rtol * s[0]))
+    Bs = vt[:r].T
+    X = np.hstack([Os[P], np.ones((len(P), 1))])
+    A = np.linalg.lstsq(X, R @ Bs, rcond=None)[0]
+    return Os + np.hstack([Os, np.ones((n, 1))]) @ A @ Bs.T, Bs, A
+
+
+def sparsepr_attention(q_bits, k_bits, v_bits, mask, bs: int, scale: float, probes):
+    """Block-sparse attention of one head (q/k/v_bits [N, d], mask [nb, nb]) followed by the
+    probe-fitted correction with the exact outputs of the given probe rows.  Returns
+    (o_corrected [N, d], o_sparse [N, d])."""
+    q, k, v = _bits(q_bits), _bits(k_bits), _bits(v_bits)
+    N, d = q.shape
+    nb = (N + bs - 1) // bs
+    blocks = masked_attention(q[None], k[None], v[None], np.asarray(mask).reshape(1, nb, nb), bs,
+                              scale)
+    o_sparse = blocks.reshape(nb * bs, d)[:N]
+    P = np.asarray(probes, np.int64).reshape(-1)
+    exact = dense_attention(q[None], k[None], v[None], scale, rows=[(0, int(t)) for t in P])
+    o, _, _ = probe_fit_correction(o_sparse, P, exact)
+    return o, o_sparse

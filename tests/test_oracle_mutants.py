@@ -1,7 +1,8 @@
 """The pins must have teeth: plant plausible slips in a copy of the oracle and watch them fail.
 
-Each mutant is a one-line textual change to a temporary copy of oracle/oracle.c, compiled into
-its own library and loaded as a separate module.  The whole pin suite runs against it and at
+Each mutant is a one-line textual change to a temporary copy of oracle/oracle.c (or, for the
+numpy steps, of oracle/__init__.py), compiled into its own library and loaded as a separate
+module.  The whole pin suite runs against it and at
 least one pin has to fail.  The real oracle is never modified.
 """
 import importlib.util
@@ -60,6 +61,16 @@ MUTANTS = {
         "const uint8_t *row = sel + (int64_t)aq[t] * Ck;", "const uint8_t *row = sel;"),
     "pool reads the wrong channel": ("s += bf16_to_double(x[(bh * N + t) * d + c]);",
                                      "s += bf16_to_double(x[(bh * N + t) * d + (d - 1 - c)]);"),
+    # the probe-fitted correction is numpy code in the module itself
+    "probe fit without the affine offset": (
+        "X = np.hstack([Os[P], np.ones((len(P), 1))])",
+        "X = np.hstack([Os[P], np.zeros((len(P), 1))])", "__init__.py"),
+    "probe residual with the wrong sign": ("R = E - Os[P]", "R = Os[P] - E", "__init__.py"),
+    "probe fit keeps one residual direction": (
+        "r = int(np.count_nonzero(s > rtol * s[0]))", "r = 1", "__init__.py"),
+    "probe rows misaligned with their exact outputs": (
+        "o, _, _ = probe_fit_correction(o_sparse, P, exact)",
+        "o, _, _ = probe_fit_correction(o_sparse, (P + 1) % N, exact)", "__init__.py"),
 }
 
 
@@ -77,13 +88,13 @@ def _pin_calls():
     return calls
 
 
-def _build_mutant(tmp_path, tag, old, new):
+def _build_mutant(tmp_path, tag, old, new, fname="oracle.c"):
     src_dir = os.path.join(ROOT, "oracle")
     dst = tmp_path / f"oracle_mut_{tag}"
     shutil.copytree(src_dir, dst, ignore=shutil.ignore_patterns("*.so", "__pycache__"))
-    c = (dst / "oracle.c").read_text()
+    c = (dst / fname).read_text()
     assert c.count(old) >= 1, f"mutation anchor not found: {old!r}"
-    (dst / "oracle.c").write_text(c.replace(old, new, 1))
+    (dst / fname).write_text(c.replace(old, new, 1))
     name = f"oracle_mut_{tag}"
     spec = importlib.util.spec_from_file_location(name, dst / "__init__.py")
     mod = importlib.util.module_from_spec(spec)
@@ -95,9 +106,9 @@ def _build_mutant(tmp_path, tag, old, new):
 
 @pytest.mark.parametrize("label", sorted(MUTANTS))
 def test_pins_catch_mutant(tmp_path, label):
-    old, new = MUTANTS[label]
+    old, new, *fname = MUTANTS[label]
     tag = "".join(ch if ch.isalnum() else "_" for ch in label)[:40]
-    mod = _build_mutant(tmp_path, tag, old, new)
+    mod = _build_mutant(tmp_path, tag, old, new, *fname)
     failed = []
     for name, fn, kw in _pin_calls():
         try:

@@ -521,3 +521,64 @@ def test_svg2_one_key_per_cluster_and_full_p_is_dense(orc):
     assert np.array_equal(ak, np.arange(n)) and sel.all()
     dense = orc.dense_attention(q[None], k[None], v[None], 0.3).reshape(n, d)
     assert np.abs(out - dense).max() < 1e-12
+
+
+# ---------------------------------------------------------------------------------------------
+# SparsePR probe-fitted residual reconstruction (page "Partition the Support, Reconstruct the
+# Residual", abstract and summary section 3)
+# ---------------------------------------------------------------------------------------------
+def test_probe_fit_recovers_a_planted_affine_residual(orc):
+    # residual = [o, 1] A0 B0^T exactly, with enough probes: the fit finds the subspace of B0 and
+    # the map, and the corrected output is exact on every row, not only on the probes
+    rng = np.random.default_rng(31)
+    n, d, r0 = 120, 8, 3
+    Os = rng.standard_normal((n, d))
+    A0 = rng.standard_normal((d + 1, r0))
+    B0 = np.linalg.qr(rng.standard_normal((d, r0)))[0]
+    exact_all = Os + np.hstack([Os, np.ones((n, 1))]) @ A0 @ B0.T
+    P = rng.choice(n, 30, replace=False)
+    o, Bs, A = orc.probe_fit_correction(Os, P, exact_all[P])
+    assert Bs.shape == (d, r0)
+    assert np.abs(Bs @ Bs.T - B0 @ B0.T).max() < 1e-9
+    assert np.abs(o - exact_all).max() < 1e-9
+
+
+def test_probe_fit_interpolates_few_probes_within_the_residual_subspace(orc):
+    rng = np.random.default_rng(32)
+    n, d = 60, 16
+    Os = rng.standard_normal((n, d))
+    P = np.array([3, 17, 40, 41, 59])
+    E = rng.standard_normal((5, d))
+    o, Bs, A = orc.probe_fit_correction(Os, P, E)
+    # fewer probes than affine features: the least-squares fit matches every probe
+    assert np.abs(o[P] - E).max() < 1e-9
+    proj = np.eye(d) - Bs @ Bs.T
+    assert np.abs((E - Os[P]) @ proj).max() < 1e-9     # the basis spans the residuals
+    assert np.abs((o - Os) @ proj).max() < 1e-9        # and holds the whole correction
+    # minimum norm: A lies in the row space of the probe features
+    X = np.hstack([Os[P], np.ones((5, 1))])
+    row_space = X.T @ np.linalg.solve(X @ X.T, X)
+    assert np.abs(A - row_space @ A).max() < 1e-9
+    # the order of the probes does not matter
+    perm = np.array([4, 2, 0, 1, 3])
+    o2, _, _ = orc.probe_fit_correction(Os, P[perm], E[perm])
+    assert np.abs(o2 - o).max() < 1e-9
+
+
+def test_sparsepr_attention_exact_cases(orc):
+    rng = np.random.default_rng(33)
+    N, d, bs, scale = 40, 8, 16, 0.3
+    q, k, v = (f32_to_bf16_bits(rng.standard_normal((N, d)).astype(np.float32)) for _ in range(3))
+    dense = orc.dense_attention(q[None], k[None], v[None], scale).reshape(N, d)
+    # a full mask: the sparse output is already exact and nothing is corrected
+    o, o_sparse = orc.sparsepr_attention(q, k, v, np.ones((3, 3), np.uint8), bs, scale, [0, 7, 39])
+    assert np.abs(o_sparse - dense).max() < 1e-12 and np.abs(o - dense).max() < 1e-12
+    # a diagonal mask with fewer probes than d + 1: the probe rows come out exact, the sparse
+    # output is the block-masked attention
+    mask = np.eye(3, dtype=np.uint8)
+    P = [2, 20, 33]
+    o, o_sparse = orc.sparsepr_attention(q, k, v, mask, bs, scale, P)
+    ref_sparse = orc.masked_attention(q[None], k[None], v[None], mask[None], bs, scale)
+    assert np.abs(o_sparse - ref_sparse.reshape(3 * bs, d)[:N]).max() < 1e-12
+    assert np.abs(o[P] - dense[P]).max() < 1e-9
+    assert np.abs(o_sparse[P] - dense[P]).max() > 1e-3   # the mask did drop something
