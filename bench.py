@@ -314,11 +314,15 @@ def run_reference(args, w):
 
 
 def config_dict(w, extra):
+    tensor_mb = w.B * w.H * w.N * w.d * 2 / 1e6
     c = {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "block": w.bs,
          "topk": w.topk, "topp": w.topp,
          "latent_grid": list(w.grid),
-         "l2": f"inputs larger than L2: Q, K, V are {w.B * w.H * w.N * w.d * 2 / 1e6:.0f} MB "
-               f"each (L2 {L2_BYTES / 2**20:.0f} MiB); pooling streams Q and K every step"}
+         "l2": (f"inputs larger than L2: Q, K, V are {tensor_mb:.0f} MB each (L2 "
+                f"{L2_BYTES / 2**20:.0f} MiB); pooling streams Q and K every step"
+                if tensor_mb * 1e6 > L2_BYTES else
+                f"inputs fit in L2 ({tensor_mb:.1f} MB per tensor): a parity-size case, not the "
+                f"bench line")}
     if extra:
         c.update(extra)
     return c
