@@ -305,16 +305,21 @@ def dense_attention(q_bits, k_bits, v_bits, scale: float, rows=None):
 # the output subspace the probe residuals span.  The steps below are the plainest reading of it;
 # their library steps are numpy's SVD and least squares.
 # ---------------------------------------------------------------------------------------------
-def probe_fit_correction(o_sparse, probes, exact, rtol: float = 1e-9):
+def probe_fit_correction(o_sparse, probes, exact, rtol: float = 1e-9, rank=None):
     """One head of one call.  o_sparse [n, d]: the sparse attention output; probes [m]: probe
     query rows; exact [m, d]: their exact (dense) attention outputs.
 
       R  = exact - o_sparse[probes]                the probe residuals
-      Bs = orthonormal basis [d, r] of the row space of R (right singular vectors whose singular
-           value exceeds rtol times the largest)   the observed output subspace
+      Bs = orthonormal basis [d, r] of the observed output subspace: the right singular vectors
+           of R whose singular value exceeds rtol times the largest (its numerical row space),
+           or only the leading `rank` of them when rank is given
       A  = argmin || [o_sparse[probes], 1] A - R Bs ||   over A [(d + 1), r]; the minimum-norm
            solution when the probes leave it underdetermined
       o  = o_sparse + [o_sparse, 1] A Bs^T         applied to every row
+
+    With the whole numerical row space (rank None) the correction equals the minimum-norm
+    least-squares fit of the residuals themselves, [o, 1] X^+ R with X = [o_sparse[probes], 1]:
+    that fit is already a combination of the rows of R.  A smaller rank confines it further.
 
     Returns (o [n, d], Bs [d, r], A [d + 1, r]), float64."""
     Os = np.asarray(o_sparse, np.float64)
@@ -326,6 +331,8 @@ def probe_fit_correction(o_sparse, probes, exact, rtol: float = 1e-9):
         return Os.copy(), np.zeros((d, 0)), np.zeros((d + 1, 0))
     _, s, vt = np.linalg.svd(R, full_matrices=False)
     r = int(np.count_nonzero(s > rtol * s[0]))
+    if rank is not None:
+        r = min(r, int(rank))
     Bs = vt[:r].T
     X = np.hstack([Os[P], np.ones((len(P), 1))])
     A = np.linalg.lstsq(X, R @ Bs, rcond=None)[0]

@@ -582,3 +582,27 @@ def test_sparsepr_attention_exact_cases(orc):
     assert np.abs(o_sparse - ref_sparse.reshape(3 * bs, d)[:N]).max() < 1e-12
     assert np.abs(o[P] - dense[P]).max() < 1e-9
     assert np.abs(o_sparse[P] - dense[P]).max() > 1e-3   # the mask did drop something
+
+
+def test_probe_fit_full_subspace_is_the_least_squares_fit_of_the_residuals(orc):
+    # at the full numerical rank the subspace step changes nothing: the correction is the
+    # minimum-norm least-squares map of the residuals (pseudo-inverse, another numpy route)
+    rng = np.random.default_rng(34)
+    n, d = 80, 12
+    Os = rng.standard_normal((n, d))
+    for m in (6, 40):
+        P = rng.choice(n, m, replace=False)
+        E = Os[P] + rng.standard_normal((m, d))
+        o, Bs, _ = orc.probe_fit_correction(Os, P, E)
+        X = np.hstack([Os[P], np.ones((m, 1))])
+        W = np.linalg.pinv(X) @ (E - Os[P])
+        assert np.abs(o - (Os + np.hstack([Os, np.ones((n, 1))]) @ W)).max() < 1e-9
+    # a lower rank keeps the leading residual directions only
+    P = rng.choice(n, 40, replace=False)
+    E = Os[P] + rng.standard_normal((40, d))
+    o2, B2, _ = orc.probe_fit_correction(Os, P, E, rank=2)
+    _, _, vt = np.linalg.svd(E - Os[P])
+    assert B2.shape == (d, 2)
+    assert np.abs(B2 @ B2.T - vt[:2].T @ vt[:2]).max() < 1e-9
+    proj = np.eye(d) - B2 @ B2.T
+    assert np.abs((o2 - Os) @ proj).max() < 1e-9
