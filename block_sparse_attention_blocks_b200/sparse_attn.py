@@ -111,6 +111,27 @@ def _need(t: torch.Tensor, name: str, dtype, ndim: int):
         raise ValueError(f"{name} must be a contiguous {ndim}-d tensor, got shape {tuple(t.shape)}")
 
 
+def _shape(t: torch.Tensor, name: str, shape):
+    """Buffers are passed to the library as bare pointers, so their sizes are checked here."""
+    if tuple(t.shape) != tuple(int(s) for s in shape):
+        raise ValueError(f"{name} must have shape {tuple(int(s) for s in shape)}, "
+                         f"got {tuple(t.shape)}")
+
+
+def _cuda_device(device) -> torch.device:
+    """A CUDA device with its index ("cuda" alone means the current device)."""
+    dev = torch.device(device) if device is not None else torch.device("cuda")
+    if dev.type == "cuda" and dev.index is None:
+        dev = torch.device("cuda", torch.cuda.current_device())
+    return dev
+
+
+def _same_device(ref: torch.Tensor, **tensors):
+    for name, t in tensors.items():
+        if t.device != ref.device:
+            raise ValueError(f"{name} is on {t.device}, expected {ref.device}")
+
+
 _WORKSPACES = {}
 
 
@@ -143,6 +164,9 @@ def pool_blocks(q: torch.Tensor, k: torch.Tensor, bs: int, qp=None, kp=None):
     kp = kp if kp is not None else torch.empty(B, H, nb, d, device=q.device, dtype=torch.float32)
     _need(qp, "qp", torch.float32, 4)
     _need(kp, "kp", torch.float32, 4)
+    _shape(qp, "qp", (B, H, nb, d))
+    _shape(kp, "kp", (B, H, nb, d))
+    _same_device(q, k=k, qp=qp, kp=kp)
     _check(lib.sa_pool_blocks(_ptr(q), _ptr(k), _ptr(qp), _ptr(kp), B, H, N, d, bs,
                               _stream(q.device)), "sa_pool_blocks")
     return qp, kp
@@ -157,6 +181,13 @@ def _sel_outputs(B, H, nb, device, mask, kv_idx, kv_cnt):
     _need(mask, "mask", torch.uint8, 4)
     _need(kv_idx, "kv_idx", torch.int32, 4)
     _need(kv_cnt, "kv_cnt", torch.int32, 3)
+    _shape(mask, "mask", (B, H, nb, nb))
+    _shape(kv_idx, "kv_idx", (B, H, nb, nb))
+    _shape(kv_cnt, "kv_cnt", (B, H, nb))
+    dev = _cuda_device(device)
+    for n, t in (("mask", mask), ("kv_idx", kv_idx), ("kv_cnt", kv_cnt)):
+        if t.device != dev:
+            raise ValueError(f"{n} is on {t.device}, expected {dev}")
     return mask, kv_idx, kv_cnt
 
 
@@ -166,6 +197,8 @@ def select_mask_topk_topp(qp, kp, topk: int, topp: float, scale: float | None = 
     _need(qp, "qp", torch.float32, 4)
     _need(kp, "kp", torch.float32, 4)
     B, H, nb, d = qp.shape
+    _shape(kp, "kp", qp.shape)
+    _same_device(qp, kp=kp)
     mask, kv_idx, kv_cnt = _sel_outputs(B, H, nb, qp.device, mask, kv_idx, kv_cnt)
     _check(lib.sa_select_mask_topk_topp(_ptr(qp), _ptr(kp), B, H, nb, d, int(topk), float(topp),
                                         float(scale or 0.0), _ptr(mask), _ptr(kv_idx),
@@ -186,6 +219,10 @@ def pool_select_topk_topp(q, k, bs: int, topk: int, topp: float, scale: float | 
     kp = kp if kp is not None else torch.empty(B, H, nb, d, dtype=torch.float32, device=q.device)
     _need(qp, "qp", torch.float32, 4)
     _need(kp, "kp", torch.float32, 4)
+    _shape(k, "k", q.shape)
+    _shape(qp, "qp", (B, H, nb, d))
+    _shape(kp, "kp", (B, H, nb, d))
+    _same_device(q, k=k, qp=qp, kp=kp)
     mask, kv_idx, kv_cnt = _sel_outputs(B, H, nb, q.device, mask, kv_idx, kv_cnt)
     _check(lib.sa_pool_select_topk_topp(_ptr(q), _ptr(k), _ptr(qp), _ptr(kp), B, H, N, d, bs,
                                         int(topk), float(topp), float(scale or 0.0), _ptr(mask),
@@ -202,6 +239,9 @@ def block_scores(qp, kp, scale: float | None = None, logits=None):
     logits = logits if logits is not None else torch.empty(B, H, nb, nb, dtype=torch.float32,
                                                            device=qp.device)
     _need(logits, "logits", torch.float32, 4)
+    _shape(kp, "kp", qp.shape)
+    _shape(logits, "logits", (B, H, nb, nb))
+    _same_device(qp, kp=kp, logits=logits)
     _check(lib.sa_block_scores(_ptr(qp), _ptr(kp), B, H, nb, d, float(scale or 0.0), _ptr(logits),
                                _stream(qp.device)), "sa_block_scores")
     return logits
@@ -211,7 +251,7 @@ def static_mask(patterns, B: int, nb: int, device=None, mask=None, kv_idx=None, 
     """Static block patterns -> (mask, kv_idx, kv_cnt) for block_sparse_attn_fwd.
     patterns: H descriptors (flags, w, p, s): flags 1 = diagonal band |i - j| <= w, 2 = diagonals
     every p blocks (half-width w), 4 = the first s key blocks; 0 = skipped head."""
-    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    dev = _cuda_device(device)
     pat = torch.as_tensor(patterns, dtype=torch.int32).reshape(-1, 4).to(dev)
     H = pat.shape[0]
     mask, kv_idx, kv_cnt = _sel_outputs(B, H, nb, dev, mask, kv_idx, kv_cnt)
@@ -224,6 +264,7 @@ def select_from_logits(logits, topk: int, topp: float, mask=None, kv_idx=None, k
     """Selection from given block scores [B, H, nb, nb] fp32 -> (mask, kv_idx, kv_cnt)."""
     _need(logits, "logits", torch.float32, 4)
     B, H, nb, _ = logits.shape
+    _shape(logits, "logits", (B, H, nb, nb))
     mask, kv_idx, kv_cnt = _sel_outputs(B, H, nb, logits.device, mask, kv_idx, kv_cnt)
     _check(lib.sa_select_from_logits(_ptr(logits), B, H, nb, int(topk), float(topp), _ptr(mask),
                                      _ptr(kv_idx), _ptr(kv_cnt), _stream(logits.device)),
@@ -238,8 +279,14 @@ def block_sparse_attn_fwd(q, k, v, kv_idx, kv_cnt, bs: int, scale: float | None 
     _need(kv_idx, "kv_idx", torch.int32, 4)
     _need(kv_cnt, "kv_cnt", torch.int32, 3)
     B, H, N, d = q.shape
+    nb = num_blocks(N, bs)
     o = o if o is not None else torch.empty_like(q)
     _need(o, "o", torch.bfloat16, 4)
+    for n, t in (("k", k), ("v", v), ("o", o)):
+        _shape(t, n, q.shape)
+    _shape(kv_idx, "kv_idx", (B, H, nb, nb))
+    _shape(kv_cnt, "kv_cnt", (B, H, nb))
+    _same_device(q, k=k, v=v, o=o, kv_idx=kv_idx, kv_cnt=kv_cnt)
     ws = _workspace(q.device)
     _check(lib.sa_block_sparse_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_idx), _ptr(kv_cnt),
                                         _ptr(o), B, H, N, d, bs, float(scale or 0.0), _ptr(ws),
@@ -254,6 +301,9 @@ def dense_attn_fwd(q, k, v, scale: float | None = None, o=None):
     B, H, N, d = q.shape
     o = o if o is not None else torch.empty_like(q)
     _need(o, "o", torch.bfloat16, 4)
+    for n, t in (("k", k), ("v", v), ("o", o)):
+        _shape(t, n, q.shape)
+    _same_device(q, k=k, v=v, o=o)
     ws = _workspace(q.device)
     _check(lib.sa_dense_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d,
                                  float(scale or 0.0), _ptr(ws), ws.numel(), _stream(q.device)),
@@ -269,6 +319,9 @@ def squad_attn_fwd(q, k, v, w: int, scale: float | None = None, o=None):
     B, H, N, d = q.shape
     o = o if o is not None else torch.empty_like(q)
     _need(o, "o", torch.bfloat16, 4)
+    for n, t in (("k", k), ("v", v), ("o", o)):
+        _shape(t, n, q.shape)
+    _same_device(q, k=k, v=v, o=o)
     nbytes = int(lib.sa_squad_workspace_bytes(B, H, N, d))
     ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
     _check(lib.sa_squad_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d, int(w),
@@ -287,8 +340,8 @@ def kmeans(x, cent, iters: int):
     _need(cent, "cent", torch.float32, 4)
     B, H, N, d = x.shape
     C = cent.shape[2]
-    if tuple(cent.shape) != (B, H, C, d):
-        raise ValueError("cent must be [B, H, C, d]")
+    _shape(cent, "cent", (B, H, C, d))
+    _same_device(x, cent=cent)
     assign = torch.empty(B, H, N, device=x.device, dtype=torch.int32)
     perm = torch.empty_like(assign)
     cstart = torch.empty(B, H, C, device=x.device, dtype=torch.int32)
@@ -320,6 +373,9 @@ def centroid_topp(cq, ck, size_k, topp: float, scale: float | None = None):
     _need(size_k, "size_k", torch.int32, 3)
     B, H, Cq, d = cq.shape
     Ck = ck.shape[2]
+    _shape(ck, "ck", (B, H, Ck, d))
+    _shape(size_k, "size_k", (B, H, Ck))
+    _same_device(cq, ck=ck, size_k=size_k)
     sel = torch.empty(B, H, Cq, Ck, device=cq.device, dtype=torch.uint8)
     nbytes = int(lib.sa_centroid_topp_workspace_bytes(B, H, Cq, Ck))
     ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=cq.device)
@@ -342,6 +398,12 @@ def cluster_attn_fwd(q, k, v, assign_q, assign_k, sel, scale: float | None = Non
     Cq, Ck = sel.shape[2], sel.shape[3]
     o = o if o is not None else torch.empty_like(q)
     _need(o, "o", torch.bfloat16, 4)
+    for n, t in (("k", k), ("v", v), ("o", o)):
+        _shape(t, n, q.shape)
+    _shape(assign_q, "assign_q", (B, H, N))
+    _shape(assign_k, "assign_k", (B, H, N))
+    _shape(sel, "sel", (B, H, Cq, Ck))
+    _same_device(q, k=k, v=v, o=o, assign_q=assign_q, assign_k=assign_k, sel=sel)
     nbytes = int(lib.sa_cluster_attn_workspace_bytes(B, H, N, d, Cq, Ck))
     ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
     _check(lib.sa_cluster_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(assign_q),
@@ -366,8 +428,15 @@ def svg2_attn_fwd(q, k, v, cent_q, cent_k, iters: int, topp: float, scale: float
     sel = sel if sel is not None else torch.empty(B, H, Cq, Ck, device=q.device, dtype=torch.uint8)
     _need(o, "o", torch.bfloat16, 4)
     _need(sel, "sel", torch.uint8, 4)
+    for n, t in (("k", k), ("v", v), ("o", o)):
+        _shape(t, n, q.shape)
+    _shape(cent_q, "cent_q", (B, H, Cq, d))
+    _shape(cent_k, "cent_k", (B, H, Ck, d))
+    _shape(sel, "sel", (B, H, Cq, Ck))
+    _same_device(q, k=k, v=v, o=o, cent_q=cent_q, cent_k=cent_k, sel=sel)
     nbytes = int(lib.sa_svg2_workspace_bytes(B, H, N, d, Cq, Ck))
-    if workspace is None or workspace.numel() < nbytes:
+    if (workspace is None or workspace.numel() < nbytes or workspace.dtype != torch.uint8
+            or workspace.device != q.device):
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
     _check(lib.sa_svg2_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(cent_q), _ptr(cent_k),
                                 B, H, N, d, Cq, Ck, int(iters), float(topp), float(scale or 0.0),
@@ -438,11 +507,16 @@ def sparse_attention(q, k, v, bs: int, topk: int, topp: float, scale: float | No
     complete when the call returns.
     """
     if not q.is_cuda:
-        dev = torch.device(device) if device is not None else torch.device("cuda",
-                                                                           torch.cuda.current_device())
         for n, t in (("q", q), ("k", k), ("v", v)):
             if t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_contiguous():
-                raise SAError(f"{n}: expected a contiguous 4-D bfloat16 tensor")
+                raise TypeError(f"{n}: expected a contiguous 4-D bfloat16 tensor")
+            if t.shape != q.shape or t.is_cuda:
+                raise ValueError(f"{n}: expected a host tensor of shape {tuple(q.shape)}")
+        if out is not None and (out.shape != q.shape or out.dtype != torch.bfloat16
+                                or out.is_cuda or not out.is_contiguous()):
+            raise ValueError(f"out: expected a contiguous host bfloat16 tensor of shape "
+                             f"{tuple(q.shape)}")
+        dev = _cuda_device(device)
         o, sel = _host_pipeline(q, k, v, bs, topk, topp, scale, dev, out, max(1, int(chunks)))
         return (o, sel) if return_selection else o
     _, _, mask, kv_idx, kv_cnt = pool_select_topk_topp(q, k, bs, topk, topp, scale)

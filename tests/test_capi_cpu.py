@@ -273,3 +273,20 @@ def test_cluster_entry_point_argument_checks(lib):
     assert sv(A, A, A, A, A, A, 1, 2, 1000, 64, 16, 40, 2, 0.9, 0.0, A, A2, Wc, S) == 1
     assert sv(A, A, A, A, MIS, A, 1, 2, 1000, 64, 16, 40, 2, 0.9, 0.0, A, A2, Ws, S) == 1
     assert sv(A, A, A, A, A, A, 1, 2, 1000, 32, 16, 40, 2, 0.9, 0.0, A, A2, Ws, S) == 2
+
+
+def test_host_inputs_are_checked_before_any_device_work():
+    import torch
+
+    from block_sparse_attention_blocks_b200 import sparse_attn as s
+
+    q = torch.empty(1, 2, 100, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        s.sparse_attention(q, q[:, :1].contiguous(), q, 64, 2, 0.9)       # k of another shape
+    with pytest.raises(TypeError):
+        s.sparse_attention(q, q.float(), q, 64, 2, 0.9)                   # v not bf16
+    with pytest.raises(ValueError):
+        s.sparse_attention(q, q, q, 64, 2, 0.9, out=torch.empty(1, 2, 99, 64,
+                                                                 dtype=torch.bfloat16))
+    with pytest.raises(TypeError):
+        s.sparse_attention(q, q, q.transpose(2, 3), 64, 2, 0.9)           # not contiguous
