@@ -5,7 +5,7 @@
 //      clusters, started from the caller's centroids (the centroid cache of section C); tokens
 //      are then reordered so that every cluster is a contiguous range.
 //   B. The score of key cluster j for query cluster a is estimated from the centroids, every key
-//      standing in for by its centroid: |j| exp(scale mu_q[a] . mu_k[j]), normalised over j.
+//      represented by its centroid: |j| exp(scale mu_q[a] . mu_k[j]), normalised over j.
 //      Key clusters are taken in descending order of it until the cumulative score reaches p.
 //   C. Attention of each query token over the keys of the clusters its cluster selected, on the
 //      permuted tensors (dense query tiles, key tiles of variable length), written back in the

@@ -171,7 +171,7 @@ sa_status sa_cluster_sort(const int32_t *assign, int B, int H, int N, int C, int
 /*
  * Centroid top-p (section B).  For query cluster a of head (b, h), key cluster j is estimated to
  * receive the share  w[a, j] = size_k[j] exp(scale cq[a] . ck[j]) / sum_j' (same)  of the
- * attention (each key stands in for by its centroid).  Key clusters are ranked by w descending
+ * attention (each key represented by its centroid).  Key clusters are ranked by w descending
  * (the lower id first on a tie) and taken until the cumulative share reaches topp; topp <= 0
  * takes none, topp >= 1 every cluster with keys; a cluster with size_k = 0 is never taken.
  * The decision runs in fp32 (the top-p kernel of the block path), so clusters whose share lies

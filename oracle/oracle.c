@@ -490,7 +490,7 @@ void or_kmeans(const double *x, int64_t n, int64_t d, int64_t C, int64_t iters, 
 
 /* Centroid top-p: for query cluster a, key cluster j is estimated to receive
  *   w[a, j] = size_k[j] exp(scale cq[a] . ck[j]) / sum_j' size_k[j'] exp(scale cq[a] . ck[j'])
- * of the attention (every key of a cluster stands in for by its centroid).  Key clusters are
+ * of the attention (every key of a cluster represented by its centroid).  Key clusters are
  * taken in order of w descending (the lower id first on a tie) until the cumulative w reaches p
  * (p <= 0 takes none, p >= 1 takes every cluster with keys).  sel [Cq, Ck] 0/1. */
 void or_centroid_topp(const double *cq, const double *ck, const int64_t *size_k, int64_t Cq,
