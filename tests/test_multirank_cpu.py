@@ -38,7 +38,7 @@ def _worker(rank, world, port, out):
 def test_two_ranks_share_inputs_and_max_time():
     world = 2
     port = _free_port()
-    with mp.Manager() as man:
+    with mp.get_context("spawn").Manager() as man:  # no fork of this threaded process
         out = man.dict()
         mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)
