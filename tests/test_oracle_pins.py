@@ -606,3 +606,25 @@ def test_probe_fit_full_subspace_is_the_least_squares_fit_of_the_residuals(orc):
     assert np.abs(B2 @ B2.T - vt[:2].T @ vt[:2]).max() < 1e-9
     proj = np.eye(d) - B2 @ B2.T
     assert np.abs((o2 - Os) @ proj).max() < 1e-9
+
+
+def test_cluster_attention_against_torch_masked_sdpa(orc):
+    # random clusters and selection: the same as fp64 torch attention with the token mask
+    # M[t, s] = sel[aq[t], ak[s]] (rows whose mask is empty are zero)
+    import torch
+
+    rng = np.random.default_rng(26)
+    n, d, Cq, Ck = 70, 8, 5, 6
+    q, k, v = (f32_to_bf16_bits(rng.standard_normal((n, d)).astype(np.float32)) for _ in range(3))
+    aq = rng.integers(0, Cq, n).astype(np.int32)
+    ak = rng.integers(0, Ck, n).astype(np.int32)
+    sel = (rng.random((Cq, Ck)) < 0.4).astype(np.uint8)
+    sel[0] = 0
+    got = orc.cluster_attention(q, k, v, aq, ak, sel, 0.35)
+    M = torch.from_numpy(sel[aq][:, ak].astype(bool))
+    t = lambda b: torch.from_numpy(widen(b))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        t(q)[None], t(k)[None], t(v)[None], attn_mask=M[None], scale=0.35)[0].numpy()
+    empty = ~M.numpy().any(1)
+    ref[empty] = 0.0
+    assert np.abs(got - ref).max() < 1e-12
