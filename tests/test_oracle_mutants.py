@@ -68,6 +68,9 @@ MUTANTS = {
     "probe residual with the wrong sign": ("R = E - Os[P]", "R = Os[P] - E", "__init__.py"),
     "probe fit keeps one residual direction": (
         "r = int(np.count_nonzero(s > rtol * s[0]))", "r = 1", "__init__.py"),
+    "SVG2 cluster sizes from the query assignment": (
+        "size_k = np.bincount(ak, minlength=cent_k.shape[0])",
+        "size_k = np.bincount(aq, minlength=cent_k.shape[0])[:cent_k.shape[0]]", "__init__.py"),
     "probe rows misaligned with their exact outputs": (
         "o, _, _ = probe_fit_correction(o_sparse, P, exact)",
         "o, _, _ = probe_fit_correction(o_sparse, (P + 1) % N, exact)", "__init__.py"),

@@ -628,3 +628,40 @@ def test_cluster_attention_against_torch_masked_sdpa(orc):
     empty = ~M.numpy().any(1)
     ref[empty] = 0.0
     assert np.abs(got - ref).max() < 1e-12
+
+
+def test_svg2_composition_against_numpy_and_torch(orc):
+    # the whole path written independently: numpy Lloyd for Q and K, the size-weighted centroid
+    # shares ranked and cut in plain Python, fp64 torch attention under the token mask
+    import torch
+
+    rng = np.random.default_rng(27)
+    n, d, Cq, Ck, iters, p, scale = 90, 6, 4, 7, 2, 0.8, 0.4
+    q, k, v = (f32_to_bf16_bits(rng.standard_normal((n, d)).astype(np.float32)) for _ in range(3))
+    qd, kd = widen(q), widen(k)
+    iq = qd[rng.choice(n, Cq, replace=False)]
+    ik = kd[rng.choice(n, Ck, replace=False)]
+    out, aq, ak, cq, ck, sel = orc.svg2_attention(q, k, v, iq, ik, iters, p, scale)
+    ref_cq, ref_aq = _lloyd_numpy(qd, iq, iters)
+    ref_ck, ref_ak = _lloyd_numpy(kd, ik, iters)
+    assert np.array_equal(aq, ref_aq) and np.array_equal(ak, ref_ak)
+    assert np.abs(cq - ref_cq).max() < 1e-12 and np.abs(ck - ref_ck).max() < 1e-12
+    size = np.bincount(ref_ak, minlength=Ck)
+    ref_sel = np.zeros((Cq, Ck), np.uint8)
+    for a in range(Cq):
+        lg = scale * (ref_ck @ ref_cq[a])
+        w = np.where(size > 0, size * np.exp(lg - lg[size > 0].max()), 0.0)
+        w /= w.sum()
+        cum = 0.0
+        for j in sorted(range(Ck), key=lambda j: (-w[j], j)):
+            if w[j] <= 0 or cum >= p:
+                break
+            ref_sel[a, j] = 1
+            cum += w[j]
+    assert np.array_equal(sel, ref_sel)
+    M = torch.from_numpy(ref_sel[ref_aq][:, ref_ak].astype(bool))
+    t = lambda b: torch.from_numpy(widen(b))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        t(q)[None], t(k)[None], t(v)[None], attn_mask=M[None], scale=scale)[0].numpy()
+    ref[~M.numpy().any(1)] = 0.0
+    assert np.abs(out - ref).max() < 1e-12
