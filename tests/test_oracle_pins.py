@@ -665,3 +665,28 @@ def test_svg2_composition_against_numpy_and_torch(orc):
         t(q)[None], t(k)[None], t(v)[None], attn_mask=M[None], scale=scale)[0].numpy()
     ref[~M.numpy().any(1)] = 0.0
     assert np.abs(out - ref).max() < 1e-12
+
+
+def test_sparsepr_composition_against_torch_and_pinv(orc):
+    # block-masked and exact attention by fp64 torch, the fit by the pseudo-inverse of the
+    # probe features: the oracle's SparsePR path must agree (more probes than features here)
+    import torch
+
+    rng = np.random.default_rng(35)
+    N, d, bs, scale = 96, 4, 16, 0.5
+    nb = N // bs
+    q, k, v = (f32_to_bf16_bits(rng.standard_normal((N, d)).astype(np.float32)) for _ in range(3))
+    mask = (rng.random((nb, nb)) < 0.4).astype(np.uint8)
+    mask[:, 0] = 1
+    P = np.sort(rng.choice(N, 20, replace=False))
+    o, o_sparse = orc.sparsepr_attention(q, k, v, mask, bs, scale, P)
+    t = lambda b: torch.from_numpy(widen(b))
+    tok = torch.from_numpy(np.kron(mask, np.ones((bs, bs), np.uint8)).astype(bool))
+    sp = torch.nn.functional.scaled_dot_product_attention(
+        t(q)[None], t(k)[None], t(v)[None], attn_mask=tok[None], scale=scale)[0].numpy()
+    ex = torch.nn.functional.scaled_dot_product_attention(
+        t(q)[None], t(k)[None], t(v)[None], scale=scale)[0].numpy()
+    assert np.abs(o_sparse - sp).max() < 1e-12
+    X = np.hstack([sp[P], np.ones((len(P), 1))])
+    W = np.linalg.pinv(X) @ (ex[P] - sp[P])
+    assert np.abs(o - (sp + np.hstack([sp, np.ones((N, 1))]) @ W)).max() < 1e-9
