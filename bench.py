@@ -503,6 +503,40 @@ def run_gpu(args, w):
                             "each position (SQuad, w = tokens of one frame)"}
         del osq
 
+    # ---------------------------------------------------------------- (k, p) sweep (opt-in)
+    sweep = None
+    if args.sweep and rank == 0 and w.sweep:
+        peaks_s, _ = load_peaks()
+        peak_s = peaks_s.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+        sweep = []
+        for topk, topp in w.sweep:
+            sm_, si_, sc_ = (torch.empty_like(t) for t in (mask, kv_idx, kv_cnt))
+            bsa.pool_select_topk_topp(q, k, bs, topk, topp, qp=qp, kp=kp, mask=sm_, kv_idx=si_,
+                                      kv_cnt=sc_)
+            bsa.block_sparse_attn_fwd(q, k, v, si_, sc_, bs, o=o)
+            torch.cuda.synchronize(dev)
+            s0, s1, s2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            reps = 5
+            s0.record(stream)
+            for _ in range(reps):
+                bsa.pool_select_topk_topp(q, k, bs, topk, topp, qp=qp, kp=kp, mask=sm_,
+                                          kv_idx=si_, kv_cnt=sc_)
+            s1.record(stream)
+            for _ in range(reps):
+                bsa.block_sparse_attn_fwd(q, k, v, si_, sc_, bs, o=o)
+            s2.record(stream)
+            torch.cuda.synchronize(dev)
+            f_s, p_s = executed_flops(sc_, sm_, N, d, bs)
+            ms_a = s1.elapsed_time(s2) / reps
+            tf = f_s / (ms_a * 1e-3) / 1e12
+            sweep.append({"topk": topk, "topp": topp, "density": p_s / float(B * H * nb * nb),
+                          "pool_select_ms": s0.elapsed_time(s1) / reps, "attention_ms": ms_a,
+                          "attention_tflops": tf, "frac_of_sustained": tf / peak_s})
+            del sm_, si_, sc_
+        err = bsa.device_error()
+        if err:
+            raise RuntimeError(f"device error {err} in the sweep")
+
     # ---------------------------------------------------------------- SVG2 (context, opt-in)
     svg2 = None
     if args.svg2 and rank == 0:
@@ -598,6 +632,8 @@ def run_gpu(args, w):
         line["squad"] = squad
     if svg2:
         line["svg2"] = svg2
+    if sweep:
+        line["sweep"] = sweep
 
     # ---------------------------------------------------------------- oracle on the host
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -634,6 +670,9 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-static", action="store_true", help="skip the static-pattern timing")
     ap.add_argument("--no-squad", action="store_true", help="skip the SQuad timing")
+    ap.add_argument("--sweep", action="store_true",
+                    help="also time pool+select and attention at every (k, p) point of the "
+                         "workload's sweep")
     ap.add_argument("--svg2", action="store_true",
                     help="also time the SVG2 path (k-means, centroid top-p, cluster attention)")
     ap.add_argument("--svg2-clusters", type=lambda s: tuple(int(x) for x in s.split(",")),
