@@ -86,6 +86,18 @@ sa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SA_OK : SA_ERR_CU
 
 constexpr size_t kAttnWorkspaceBytes = 256;
 
+// Host-side argument checks of the block-sparse attention entry points (no device work).
+sa_status check_sparse_attn_args(const void *q, const void *k, const void *v,
+                                 const int32_t *kv_idx, const int32_t *kv_cnt, const void *o,
+                                 int B, int H, int N, int d, int bs, float scale) {
+    if (!q || !k || !v || !kv_idx || !kv_cnt || !o || !shape_ok(B, H, N)) return SA_ERR_INVALID_ARG;
+    if (!dims_supported(d, bs)) return SA_ERR_UNSUPPORTED;
+    if (sa_num_blocks(N, bs) > 1024) return SA_ERR_UNSUPPORTED;
+    if (isnan(scale)) return SA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SA_ERR_INVALID_ARG;
+    return SA_OK;
+}
+
 sa_status run_attention(const void *q, const void *k, const void *v, const int32_t *kv_idx,
                         const int32_t *kv_cnt, void *o, int B, int H, int N, int d, int bs,
                         float scale, void *workspace, void *stream) {
@@ -193,13 +205,10 @@ sa_status sa_block_sparse_attn_fwd(const void *q, const void *k, const void *v,
                                    const int32_t *kv_idx, const int32_t *kv_cnt, void *o, int B,
                                    int H, int N, int d, int bs, float scale, void *workspace,
                                    size_t workspace_bytes, void *stream) {
-    if (!q || !k || !v || !kv_idx || !kv_cnt || !o || !shape_ok(B, H, N)) return SA_ERR_INVALID_ARG;
+    const sa_status a = check_sparse_attn_args(q, k, v, kv_idx, kv_cnt, o, B, H, N, d, bs, scale);
+    if (a != SA_OK) return a;
     if (!workspace || workspace_bytes < kAttnWorkspaceBytes || !aligned16(workspace))
         return SA_ERR_INVALID_ARG;
-    if (!dims_supported(d, bs)) return SA_ERR_UNSUPPORTED;
-    if (sa_num_blocks(N, bs) > 1024) return SA_ERR_UNSUPPORTED;
-    if (isnan(scale)) return SA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SA_ERR_INVALID_ARG;
     return run_attention(q, k, v, kv_idx, kv_cnt, o, B, H, N, d, bs, scale, workspace, stream);
 }
 

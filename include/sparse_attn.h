@@ -263,7 +263,10 @@ size_t sa_attn_workspace_bytes(void);
  * library's device image, which every GPU that loads the library holds until the process exits.
  * Arguments, layouts and results are those of sa_block_sparse_attn_fwd without the workspace.
  * - The first call on a device resolves the array's device address (cudaGetSymbolAddress, with
- *   that device current) and caches it; make that first call before any stream capture.
+ *   that device current) and caches it; make that first call before any stream capture.  The
+ *   cache is keyed on the device context's unique id: after cudaDeviceReset (or any other end
+ *   of the context) the next call resolves the address again in the new context, and that
+ *   call, too, should come before any stream capture.
  * - Every call shares the one array, which keeps the last call's contents; each call zeroes
  *   the counter on `stream` before its kernel.  Calls that overlap on the GPU (different
  *   streams, or several host threads) race on the array and must be serialised by the caller.

@@ -151,6 +151,26 @@ def test_attention_argument_checks(lib):
     assert g(A, A, A, A, 1, 1, 256, 128, 0.0, NUL, W, S) == 1
 
 
+def test_noalloc_attention_argument_checks(lib):
+    # the allocation-free entry point rejects what the workspace entry point rejects, on the host
+    # and before it resolves its scratch array: null pointers, unsupported sizes, a NaN scale,
+    # misaligned buffers, and an output that is not device memory
+    f = lib.sa_block_sparse_attn_fwd_noalloc
+    f.argtypes = [ctypes.c_void_p] * 6 + [ctypes.c_int] * 5 + [ctypes.c_float, ctypes.c_void_p]
+    assert f(A, A, A, A, A, NUL, 1, 1, 256, 128, 128, 0.0, S) == 1   # null o
+    assert f(NUL, A, A, A, A, A, 1, 1, 256, 128, 128, 0.0, S) == 1   # null q
+    assert f(A, A, A, A, NUL, A, 1, 1, 256, 128, 128, 0.0, S) == 1   # null kv_cnt
+    assert f(A, A, A, A, A, A, 1, 1, 256, 96, 128, 0.0, S) == 2      # unsupported d
+    assert f(A, A, A, A, A, A, 1, 1, 256, 128, 32, 0.0, S) == 2      # unsupported bs
+    assert f(A, A, A, A, A, A, 1, 1, 128 * 1025, 128, 128, 0.0, S) == 2
+    assert f(A, A, A, A, A, A, 1, 1, 256, 128, 128, float("nan"), S) == 1
+    assert f(A, A, A, A, A, MIS, 1, 1, 256, 128, 128, 0.0, S) == 1
+    assert f(A, A, A, A, A, A, 0, 1, 256, 128, 128, 0.0, S) == 1
+    host = ctypes.create_string_buffer(256 * 128 * 2 + 16)
+    o_host = ctypes.c_void_p((ctypes.addressof(host) + 15) // 16 * 16)
+    assert f(A, A, A, A, A, o_host, 1, 1, 256, 128, 128, 0.0, S) == 1  # o not device memory
+
+
 def test_python_binding_imports():
     import block_sparse_attention_blocks_b200 as pkg
 

@@ -13,7 +13,8 @@ import pytest
 import torch
 
 from block_sparse_attention_blocks_b200 import workloads as W
-from tests.parity import compare_attention, compare_masks, list_from_mask
+from tests.parity import (compare_attention, compare_masks, list_from_mask, pool_error_bound,
+                          score_error_bound)
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -80,12 +81,18 @@ def test_workload_parity(orc, name):
     if name == "stress_mixed":
         points.append((nb, w.topp))  # dense control: k = all blocks
     oracle_mask = None
+    # rule (b) of the mask parity: the proven error of the GPU's fp32 pooled scores
+    err = score_error_bound(oq, ok_, w.scale, pool_error_bound(orc, qb.reshape(BH, N, d), bs),
+                            pool_error_bound(orc, kb.reshape(BH, N, d), bs))
     for topk, topp in points:
         mask, idx, cnt = bsa.select_mask_topk_topp(qp, kp, topk, topp)
         torch.cuda.synchronize()
         sel = orc.select(oq, ok_, topk, topp, w.scale)
-        st = compare_masks(mask.cpu().numpy(), idx.cpu().numpy(), cnt.cpu().numpy(), sel)
+        st = compare_masks(mask.cpu().numpy(), idx.cpu().numpy(), cnt.cpu().numpy(), sel, err)
+        allowed = st.pop("allowed")
         print(f"{name} k={topk} p={topp}: density {sel.cnt.mean() / nb:.4f} {st}")
+        for a in allowed:
+            print(f"  allowed mismatch (row, block, reason, |P_j - P_tau| / P_tau): {a}")
         if (topk, topp) == (w.topk, w.topp):
             oracle_mask = sel.mask.reshape(w.B, w.H, nb, nb)
         if topk >= nb:
