@@ -51,16 +51,28 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                  : "memory");
 }
 
-// One poll of the barrier; a thread that finds the phase incomplete may be suspended for at most
-// ~20 us (explicit hint), so that the bounded waits below see the clock often.
+// One poll of the barrier.  The test form returns at once; the try form lets a thread that finds
+// the phase incomplete be suspended for a short, system-defined time (a suspend-time hint costs
+// ~150 cycles per call even when the phase is already complete, so none is given).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"(20000u)
+        : "r"(bar), "r"(parity)
         : "memory");
     return ok != 0;
 }
@@ -70,7 +82,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns,
                                           volatile int *abort_flag, uint32_t tag = 0,
                                           uint32_t detail = 0) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_test_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     uint32_t spins = 0;
     while (true) {
@@ -97,6 +109,7 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_
                                           volatile int *abort_flag, uint32_t tag = 0,
                                           uint32_t detail = 0) {
     const bool leader = (threadIdx.x & 31) == 0;
+    if (__all_sync(0xffffffffu, mbar_test_wait(bar, parity))) return true;  // usual case: done
     uint64_t t0 = 0;
     uint32_t spins = 0;
     while (true) {
