@@ -180,12 +180,35 @@ def max_over_ranks(x: float, device=None) -> float:
     return float(t.item())
 
 
-def make_inputs(w, rank, world):
-    """Seeded inputs; rank 0 generates them once and shares them through /dev/shm."""
+def shard_heads(n: int, rank: int, world: int):
+    """The flat (batch, head) indices rank `rank` of `world` computes when the heads of one call
+    are split across ranks: a contiguous slice, sizes differing by at most one."""
+    lo = rank * n // world
+    hi = (rank + 1) * n // world
+    return list(range(lo, hi))
+
+
+def sum_over_ranks(x: float, device=None) -> float:
+    """The sum of x over all ranks (identity on one process)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def make_inputs(w, rank, world, split_heads=False):
+    """Seeded inputs; rank 0 generates them once and shares them through /dev/shm.  With
+    split_heads every rank generates only its own slice of the heads (shard_heads)."""
     from block_sparse_attention_blocks_b200 import workloads as W
 
     if world == 1:
         return W.make_qkv(w)
+    if split_heads:
+        return W.make_qkv(w, heads=shard_heads(w.B * w.H, rank, world))
     import torch.distributed as dist
 
     names = None
@@ -346,7 +369,14 @@ def run_gpu(args, w):
     torch.cuda.set_device(dev)
     import block_sparse_attention_blocks_b200 as bsa
 
-    q_np, k_np, v_np = make_inputs(w, rank, world)
+    split = args.split == "heads" and world > 1
+    q_np, k_np, v_np = make_inputs(w, rank, world, split_heads=split)
+    if split:
+        # this rank's heads, as one batch of len(heads) heads (the units never exchange data)
+        from dataclasses import replace
+
+        w_full = w
+        w = replace(w, B=1, H=q_np.shape[1])
     as_bf16 = lambda a: torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16)
     q, k, v = (as_bf16(a).to(dev) for a in (q_np, k_np, v_np))
     B, H, N, d, bs, nb = w.B, w.H, w.N, w.d, w.bs, w.nb
@@ -378,6 +408,9 @@ def run_gpu(args, w):
         raise RuntimeError(f"device error {err} during warm-up")
     flops, pairs = executed_flops(kv_cnt, mask, N, d, bs)
     density = pairs / float(B * H * nb * nb)
+    # FLOPs of the whole job per step: every rank's own call (replicas), or the sum of the
+    # ranks' slices of one call (head split)
+    job_flops = sum_over_ranks(flops, dev) if split else world * flops
 
     # ---------------------------------------------------------------- timed region
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
@@ -428,7 +461,7 @@ def run_gpu(args, w):
         torch.cuda.synchronize(dev)
         ms_e2e = max_over_ranks(s2.elapsed_time(e2) / e2e_steps, dev)
         nbytes = q.numel() * 2
-        e2e = {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOPS",
+        e2e = {"value": job_flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOPS",
                "ms_per_step": ms_e2e, "steps": e2e_steps,
                "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
                "path": "bsa.sparse_attention on pinned host Q,K,V: 8 head chunks, each copied "
@@ -592,16 +625,19 @@ def run_gpu(args, w):
     ps_gbs = ps_bytes / (t_ps * 1e-3) / 1e9
     line = {
         "metric": METRIC,
-        "value": world * flops / (ms_step * 1e-3) / 1e12,
+        "value": job_flops / (ms_step * 1e-3) / 1e12,
         "unit": "TFLOPS",
         "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
         "ms_per_step": ms_step,
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if split else "weak",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": config_dict(w, {"realized_density": density, "executed_pairs": pairs,
+        "config": config_dict(w_full if split else w, {
+            **({"parallelism": f"heads split over {world} ranks ({H} heads on rank 0)"} if split
+               else {"parallelism": f"{world} independent replicas" if world > 1 else "1 GPU"}),
+            "realized_density": density, "executed_pairs": pairs,
                                   "effective_flops_per_call": flops}),
         "roofline": {"kernel": "attn_fwd_kernel<128,128>", "bound": "tensor",
                      "achieved": att_tflops, "peak": peak_tc, "unit": "TFLOP/s",
@@ -680,6 +716,9 @@ def main():
     ap.add_argument("--svg2-clusters", type=lambda s: tuple(int(x) for x in s.split(",")),
                     default=(128, 256), help="query,key cluster counts for --svg2")
     ap.add_argument("--svg2-iters", type=int, default=2, help="k-means update steps for --svg2")
+    ap.add_argument("--split", choices=("replicas", "heads"), default="replicas",
+                    help="with several GPUs: every rank runs the whole call (replicas, weak "
+                         "scaling) or the heads of one call are split across ranks (strong)")
     ap.add_argument("--heads", type=int, default=None,
                     help="run only the first H heads (small cases for profiling; not a bench line)")
     args = ap.parse_args()

@@ -9,6 +9,25 @@
 
 namespace bsa {
 
+// Launch `kern` on `st` with programmatic stream serialization, so that it may begin while the
+// previous kernel on the stream drains; the kernel calls grid_dependency_wait() before it reads
+// what that kernel wrote.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                    cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 cudaError_t pool_blocks(const void *q, const void *k, float *qp, float *kp, long long BH, int N,
                         int d, int bs, cudaStream_t st);
 

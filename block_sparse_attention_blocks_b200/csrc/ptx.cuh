@@ -136,6 +136,13 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_
     }
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream serialization may start
+// while the previous kernel on the stream is finishing; this waits until that kernel has
+// completed and its memory operations are visible (a no-op for an ordinary launch).
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ------------------------------------------------------------------------------------------
 // TMA (tiled, no multicast)
 // ------------------------------------------------------------------------------------------

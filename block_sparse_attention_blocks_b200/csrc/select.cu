@@ -76,6 +76,7 @@ __global__ void __launch_bounds__(256, 2) block_scores_tc_kernel(const float *__
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_BAR + 8);
     const int bh = blockIdx.z, i0 = blockIdx.y * TC_ROWS, j0 = blockIdx.x * TC_ROWS;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    grid_dependency_wait();  // the pooled tiles of a programmatically dependent launch are complete
 
     if (tid == 0) {
         mbar_init(smem_u32(bar), 1);
@@ -273,15 +274,22 @@ __device__ __forceinline__ void search_thresholds(const uint32_t (&key)[EE], con
 //          tied blocks at T_p are taken in id order until the mass reaches p;  m = their count
 //          plus the blocks above T_p.
 //   top-k: T_k = the largest key value with  #{e : key_e >= T_k} >= k.
-// Both thresholds are found together by one bitwise search that stops early.  Masses are summed in fixed
+// The top-p threshold is found by a bitwise search: its first 11 bits over every block held in
+// registers, then the blocks whose keys share those bits (a bucket of at most 64 in practice) are
+// compacted in id order into shared memory and the remaining 21 bits are decided over the bucket
+// alone, with the mass above the bucket added once (a crowded bucket falls back to the search
+// over every block).  The top-k threshold, needed only when the top-p prefix is shorter than k,
+// is found by the register search, which stops as soon as exactly k keys clear the candidate.  Masses are summed in fixed
 // point (round(P * 2^26) in 32 bits), so every warp sum is exact, independent of the order of
 // addition, and one redux.sync instruction; the fixed-point rounding (<= 2^-27 per block, under
 // 8e-6 over a row) stays below the 1e-5 resolution of the cut.  The union is the longer prefix,
 // |keep| = max(min(k, nb), m).
 template <int E>
-__global__ void __launch_bounds__(SEL_WARPS * 32) select_rows_kernel(
+__global__ void __launch_bounds__(SEL_WARPS * 32, E <= 20 ? 8 : 4) select_rows_kernel(
     const float *logits, long long rows, int nb, int topk, float topp, uint8_t *__restrict__ mask,
     int32_t *kv_idx, int32_t *__restrict__ kv_cnt) {
+    __shared__ uint32_t s_cand[SEL_WARPS][2 * 64];
+    grid_dependency_wait();  // the scores of a programmatically dependent launch are complete
     const int lane = threadIdx.x & 31;
     const long long row = (long long)blockIdx.x * SEL_WARPS + (threadIdx.x >> 5);
     if (row >= rows) return;
@@ -331,17 +339,91 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) select_rows_kernel(
 
     // ---- the top-p threshold first; the top-k one only if the top-p prefix is shorter than k
     uint32_t tp = 0u, tk = 0u;
-    if (!all_kept && want_p) search_thresholds<E>(key, pf, pfix, kk, true, false, tp, tk);
-
-    // ---- top-p count m (ties at tp taken in id order until the mass reaches p)
-    int m, ntake = 0;
+    int m, ntake = 0, ntie_tp = -1;  // blocks tied at tp, when known
+    bool counted = false;
     if (!(topp > 0.f)) {
         m = 0;
-    } else if (!want_p) {
-        m = nb;  // p >= 1, or the fixed-point total falls short of p
-    } else if (all_kept) {
-        m = nb;  // k >= nb keeps everything; the top-p cut does not matter
+        counted = true;
+    } else if (!want_p || all_kept) {
+        m = nb;  // p >= 1, the fixed-point total falls short of p, or k >= nb keeps everything
+        counted = true;
     } else {
+        // The first PRE bits of the threshold over every block in registers.  The answer then
+        // lies in the bucket [tp, tp | LOW]: the blocks in it are compacted (in id order) into
+        // shared memory, the mass above the bucket is summed once, and the remaining bits are
+        // decided over the bucket alone; mass{key >= c} = mass above + mass{bucket key >= c}.
+        constexpr int PRE = 11, CAP = 64;
+        constexpr uint32_t LOW = (1u << (32 - PRE)) - 1u;
+#pragma unroll 1
+        for (int bit = 31; bit >= 32 - PRE; --bit) {
+            const uint32_t cp = tp | (1u << bit);
+            uint32_t ms = 0u;
+#pragma unroll
+            for (int r = 0; r < E; ++r) ms += key[r] >= cp ? pf[r] : 0u;
+            if (__reduce_add_sync(0xffffffffu, ms) >= pfix) tp = cp;
+        }
+        const uint32_t hi = tp | LOW;
+        uint32_t am = 0u, ac = 0u;
+        int n = 0;
+        uint32_t *ck = s_cand[threadIdx.x >> 5], *cm = s_cand[threadIdx.x >> 5] + CAP;
+#pragma unroll
+        for (int r = 0; r < E; ++r) {
+            const bool inb = key[r] >= tp && key[r] <= hi;
+            const uint32_t bal = __ballot_sync(0xffffffffu, inb);
+            const int pos = n + __popc(bal & lt_mask);
+            if (inb && pos < CAP) {
+                ck[pos] = key[r];
+                cm[pos] = pf[r];
+            }
+            n += __popc(bal);
+            am += key[r] > hi ? pf[r] : 0u;
+            ac += key[r] > hi ? 1u : 0u;
+        }
+        if (n <= CAP) {
+            const uint32_t above_m = __reduce_add_sync(0xffffffffu, am);
+            const int above_c = (int)__reduce_add_sync(0xffffffffu, ac);
+            __syncwarp();
+            // position j of the bucket: slot j / 32 of lane j % 32 (id order = position order)
+            const uint32_t k0 = lane < n ? ck[lane] : 0u, m0 = lane < n ? cm[lane] : 0u;
+            const uint32_t k1 = lane + 32 < n ? ck[lane + 32] : 0u, m1 = lane + 32 < n ? cm[lane + 32] : 0u;
+            __syncwarp();
+#pragma unroll 1
+            for (int bit = 31 - PRE; bit >= 0; --bit) {
+                const uint32_t cp = tp | (1u << bit);
+                const uint32_t ms = (k0 >= cp ? m0 : 0u) + (k1 >= cp ? m1 : 0u);
+                if (above_m + __reduce_add_sync(0xffffffffu, ms) >= pfix) tp = cp;
+            }
+            // m: the blocks above tp, then the blocks tied at tp in id order until the mass
+            // reaches p (ties can only be bucket members)
+            uint32_t run = above_m + __reduce_add_sync(0xffffffffu, (k0 > tp ? m0 : 0u) + (k1 > tp ? m1 : 0u));
+            const int gt = above_c + (int)__reduce_add_sync(0xffffffffu, (k0 > tp ? 1u : 0u) + (k1 > tp ? 1u : 0u));
+            int need = 0, ntie = 0;
+#pragma unroll
+            for (int sidx = 0; sidx < 2; ++sidx) {
+                const bool tied = (sidx == 0 ? k0 : k1) == tp && (sidx == 0 ? lane : lane + 32) < n;
+                const uint32_t bal = __ballot_sync(0xffffffffu, tied);
+                if (bal) {
+                    uint32_t v = tied ? (sidx == 0 ? m0 : m1) : 0u;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const uint32_t y = __shfl_up_sync(0xffffffffu, v, o);
+                        if (lane >= o) v += y;
+                    }
+                    need += __popc(__ballot_sync(0xffffffffu, tied && run + v < pfix));
+                    run += __shfl_sync(0xffffffffu, v, 31);
+                    ntie += __popc(bal);
+                }
+            }
+            ntake = min(need + 1, ntie);
+            ntie_tp = ntie;
+            m = gt + ntake;
+            counted = true;
+        } else {
+            // a crowded bucket: finish the search over the registers
+            search_thresholds<E>(key, pf, pfix, kk, true, false, tp, tk);
+        }
+    }
+    if (!counted) {
         uint32_t as = 0u, ac = 0u;
 #pragma unroll
         for (int r = 0; r < E; ++r) {
@@ -399,29 +481,43 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) select_rows_kernel(
     uint8_t *mrow = mask + (size_t)row * nb;
     int32_t *idx = kv_idx + (size_t)row * nb;
     int tied_before = 0, pos = 0;
+    // the usual case: every block tied at the threshold is taken (typically the one cut block)
+    const bool all_tied = T == tp && ntie_tp >= 0 && take >= ntie_tp && take > 0;
+    if (all_tied) {
 #pragma unroll
-    for (int r = 0; r < E; ++r) {
-        const int e = r * 32 + lane;
-        const bool tied = key[r] == T;
-        const uint32_t tb = __ballot_sync(0xffffffffu, tied);
-        const bool kept = e < nb && (key[r] > T || (tied && tied_before + __popc(tb & lt_mask) < take));
-        tied_before += __popc(tb);
-        const uint32_t kb = __ballot_sync(0xffffffffu, kept);
-        if (e < nb) mrow[e] = kept ? 1 : 0;
-        if (kept) idx[pos + __popc(kb & lt_mask)] = e;
-        pos += __popc(kb);
+        for (int r = 0; r < E; ++r) {
+            const int e = r * 32 + lane;
+            const bool kept = e < nb && key[r] >= T;
+            const uint32_t kb = __ballot_sync(0xffffffffu, kept);
+            if (e < nb) mrow[e] = kept ? 1 : 0;
+            if (kept) idx[pos + __popc(kb & lt_mask)] = e;
+            pos += __popc(kb);
+        }
+    } else {
+#pragma unroll
+        for (int r = 0; r < E; ++r) {
+            const int e = r * 32 + lane;
+            const bool tied = key[r] == T;
+            const uint32_t tb = __ballot_sync(0xffffffffu, tied);
+            const bool kept = e < nb && (key[r] > T || (tied && tied_before + __popc(tb & lt_mask) < take));
+            tied_before += __popc(tb);
+            const uint32_t kb = __ballot_sync(0xffffffffu, kept);
+            if (e < nb) mrow[e] = kept ? 1 : 0;
+            if (kept) idx[pos + __popc(kb & lt_mask)] = e;
+            pos += __popc(kb);
+        }
     }
     if (lane == 0) kv_cnt[row] = pos;
 }
+
 
 template <int E>
 static cudaError_t launch_select_rows(const float *logits, long long rows, int nb, int topk,
                                       float topp, uint8_t *mask, int32_t *kv_idx, int32_t *kv_cnt,
                                       cudaStream_t st) {
     const long long grid = (rows + SEL_WARPS - 1) / SEL_WARPS;
-    select_rows_kernel<E><<<(unsigned)grid, SEL_WARPS * 32, 0, st>>>(logits, rows, nb, topk, topp,
-                                                                     mask, kv_idx, kv_cnt);
-    return cudaGetLastError();
+    return launch_dependent(select_rows_kernel<E>, dim3((unsigned)grid), dim3(SEL_WARPS * 32), 0,
+                            st, logits, rows, nb, topk, topp, mask, kv_idx, kv_cnt);
 }
 
 cudaError_t select_rows(const float *logits, long long rows, int nb, int topk, float topp,
@@ -448,8 +544,8 @@ static cudaError_t launch_scores_tc(const float *qp, const float *kp, float *log
     if (e != cudaSuccess) return e;
     const int t = (nb + TC_ROWS - 1) / TC_ROWS;
     dim3 grid((unsigned)t, (unsigned)t, (unsigned)BH);
-    block_scores_tc_kernel<D><<<grid, 256, C::SMEM, st>>>(qp, kp, logits, nb, scale, wait_ns);
-    return cudaGetLastError();
+    return launch_dependent(block_scores_tc_kernel<D>, grid, dim3(256), C::SMEM, st, qp, kp, logits,
+                            nb, scale, wait_ns);
 }
 
 cudaError_t block_scores_tc(const float *qp, const float *kp, float *logits, long long BH, int nb,

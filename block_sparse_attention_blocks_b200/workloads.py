@@ -255,24 +255,31 @@ _RECIPES = {"pr1": _head_pr1, "cluster": _head_cluster, "hunyuan": _head_hunyuan
             "mixed": _head_mixed}
 
 
-def make_qkv(w: Workload, seed: int = 0, threads: int | None = None):
-    """Q, K, V for workload `w` as bf16 bit patterns [B, H, N, d] (uint16)."""
+def make_qkv(w: Workload, seed: int = 0, threads: int | None = None, heads=None):
+    """Q, K, V for workload `w` as bf16 bit patterns [B, H, N, d] (uint16).
+
+    heads: optional list of flat (batch, head) indices bh = b * H + h; then only those heads are
+    generated, as [1, len(heads), N, d] in the given order, each bit-identical to its slice of
+    the full tensors (every head has its own seeded stream)."""
     T, Y, X = w.grid
     assert T * Y * X == w.N, (w.name, w.grid, w.N)
-    out = [np.empty((w.B, w.H, w.N, w.d), np.uint16) for _ in range(3)]
+    sel = list(range(w.B * w.H)) if heads is None else [int(x) for x in heads]
+    shape = (w.B, w.H, w.N, w.d) if heads is None else (1, len(sel), w.N, w.d)
+    out = [np.empty(shape, np.uint16) for _ in range(3)]
+    flat = [x.reshape(-1, w.N, w.d) for x in out]
     fn = _RECIPES[w.recipe]
 
-    def one(bh):
-        b, h = divmod(bh, w.H)
+    def one(slot):
+        b, h = divmod(sel[slot], w.H)
         rng = _rng(seed, w, b, h)
-        for dst, x in zip(out, fn(w, rng, h)):
-            dst[b, h] = f32_to_bf16_bits(x)
+        for dst, x in zip(flat, fn(w, rng, h)):
+            dst[slot] = f32_to_bf16_bits(x)
 
-    n = w.B * w.H
-    threads = threads or min(n, os.cpu_count() or 1, 16)
+    n = len(sel)
+    threads = threads or min(max(n, 1), os.cpu_count() or 1, 16)
     if threads <= 1:
-        for bh in range(n):
-            one(bh)
+        for slot in range(n):
+            one(slot)
     else:
         with ThreadPoolExecutor(threads) as ex:
             list(ex.map(one, range(n)))
