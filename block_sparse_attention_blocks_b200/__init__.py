@@ -7,7 +7,7 @@ the library.
 """
 _API = ("pool_blocks", "select_mask_topk_topp", "pool_select_topk_topp", "block_scores", "static_mask",
         "select_from_logits",
-        "block_sparse_attn_fwd",
+        "block_sparse_attn_fwd", "sparsepr_attn_fwd",
         "dense_attn_fwd", "squad_attn_fwd", "kmeans", "cluster_sort", "centroid_topp",
         "cluster_attn_fwd", "svg2_attn_fwd", "sparse_attention", "num_blocks", "device_error", "set_wait_limit_ns",
         "probe_bounded_wait", "SAError", "lib")

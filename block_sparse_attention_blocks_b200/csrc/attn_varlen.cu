@@ -10,6 +10,8 @@
 // clusters.  Keys of a tile past its valid count (they belong to the next cluster) are masked;
 // query rows past the tile's count are computed but not stored.  The output row of permuted
 // query row s is written at its original position perm_q[s], which undoes the permutation.
+// The query tensor may have another length than the keys (Nq rows against N keys), e.g. a set
+// of gathered query rows attending to every key.
 //
 // The pipeline and the roles are those of the block-sparse kernel (one TMA producer lane, one
 // MMA issuer lane, a tensor-memory allocator warp and four softmax warps; S = Q K^T and O += P V
@@ -25,9 +27,9 @@ struct VarlenParams {
     const int2 *units;      // [BH * units_per_head] {q_row0, q_rows << 16 | cluster}; q_rows = 0: no work
     const int32_t *tiles;   // [BH * Cq, tstride] key tiles (k_row0 << 7) | (valid - 1)
     const int32_t *tcnt;    // [BH * Cq] key tiles in each query cluster's list
-    const int32_t *perm_q;  // [BH, N] original token of each permuted query row
-    __nv_bfloat16 *o;       // [BH, N, D] in the original token order
-    int N, Cq, tstride, units_per_head;
+    const int32_t *perm_q;  // [BH, Nq] original position of each permuted query row
+    __nv_bfloat16 *o;       // [BH, Nq, D] in the original order
+    int N, Nq, Cq, tstride, units_per_head;  // N keys, Nq query (and output) rows
     long long nunits;       // BH * units_per_head
     float scale_log2;       // softmax scale * log2(e)
     unsigned long long wait_ns;
@@ -70,7 +72,7 @@ __device__ __forceinline__ VarUnit decode_unit(const VarlenParams &p, long long 
     r.cluster = e.y & 0xFFFF;
     r.row0 = e.x;
     if (r.rows > 0 &&
-        (r.rows > 128 || r.row0 < 0 || r.row0 > p.N - r.rows || r.cluster >= p.Cq)) {
+        (r.rows > 128 || r.row0 < 0 || r.row0 > p.Nq - r.rows || r.cluster >= p.Cq)) {
         atomicOr(&g_bsa_device_error, BSA_DEVERR_BOUNDS);
         r.rows = 0;  // a malformed unit is skipped by every role alike
     }
@@ -304,13 +306,13 @@ __global__ void __launch_bounds__(256, 2)
             const bool row_ok = r < w.rows;
             int orig = 0;
             if (row_ok) {
-                orig = prm.perm_q[(size_t)w.bh * prm.N + w.row0 + r];
-                if (orig < 0 || orig >= prm.N) {
+                orig = prm.perm_q[(size_t)w.bh * prm.Nq + w.row0 + r];
+                if (orig < 0 || orig >= prm.Nq) {
                     atomicOr(&g_bsa_device_error, BSA_DEVERR_BOUNDS);
                     orig = 0;
                 }
             }
-            __nv_bfloat16 *orow = prm.o + ((size_t)w.bh * prm.N + orig) * D;
+            __nv_bfloat16 *orow = prm.o + ((size_t)w.bh * prm.Nq + orig) * D;
             if (cnt == 0) {  // the cluster selected nothing: zeros
                 if (row_ok) {
                     const uint4 z = make_uint4(0u, 0u, 0u, 0u);
@@ -432,7 +434,7 @@ static cudaError_t launch_varlen_t(const CUtensorMap &tq, const CUtensorMap &tk,
 cudaError_t attn_varlen_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                             const int2 *units, int units_per_head, const int32_t *tiles,
                             const int32_t *tcnt, int tstride, const int32_t *perm_q, void *o,
-                            long long BH, int N, int Cq, int d, float scale,
+                            long long BH, int N, int Nq, int Cq, int d, float scale,
                             unsigned long long wait_ns, int num_sms, unsigned int *workspace,
                             cudaStream_t st) {
     VarlenParams p;
@@ -442,6 +444,7 @@ cudaError_t attn_varlen_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const 
     p.perm_q = perm_q;
     p.o = reinterpret_cast<__nv_bfloat16 *>(o);
     p.N = N;
+    p.Nq = Nq;
     p.Cq = Cq;
     p.tstride = tstride;
     p.scale_log2 = scale * 1.4426950408889634f;

@@ -51,7 +51,7 @@ cudaError_t attn_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtenso
 cudaError_t attn_varlen_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                             const int2 *units, int units_per_head, const int32_t *tiles,
                             const int32_t *tcnt, int tstride, const int32_t *perm_q, void *o,
-                            long long BH, int N, int Cq, int d, float scale,
+                            long long BH, int N, int Nq, int Cq, int d, float scale,
                             unsigned long long wait_ns, int num_sms, unsigned int *workspace,
                             cudaStream_t st);
 

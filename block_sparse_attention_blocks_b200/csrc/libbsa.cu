@@ -11,3 +11,4 @@
 #include "squad.cu"
 #include "svg2.cu"
 #include "noalloc.cu"
+#include "sparsepr.cu"

@@ -569,7 +569,7 @@ sa_status cluster_attention_tail(const void *q, const void *k, const void *v, vo
         !make_tmap(&tv, w.vp, BH, N, d, 128))
         return SA_ERR_CUDA;
     return from_cuda(bsa::attn_varlen_fwd(tq, tk, tv, w.units, w.U, w.tiles, w.tcnt, w.tstride,
-                                          w.perm_q, o, BH, N, Cq, d, resolve_scale(scale, d),
+                                          w.perm_q, o, BH, N, N, Cq, d, resolve_scale(scale, d),
                                           g_wait_ns, sms, w.counter, st));
 }
 

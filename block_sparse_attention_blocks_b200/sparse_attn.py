@@ -53,6 +53,10 @@ lib.sa_svg2_workspace_bytes.restype = _Z
 lib.sa_svg2_attn_fwd.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _P, _P,
                                  _Z, _P]
 lib.sa_block_sparse_attn_fwd.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _Z, _P]
+lib.sa_sparsepr_attn_fwd.argtypes = [_P, _P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _F, _P, _Z,
+                                     _P]
+lib.sa_sparsepr_workspace_bytes.argtypes = [_I, _I, _I, _I, _I]
+lib.sa_sparsepr_workspace_bytes.restype = _Z
 lib.sa_dense_attn_fwd.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _Z, _P]
 lib.sa_attn_workspace_bytes.argtypes = []
 lib.sa_attn_workspace_bytes.restype = _Z
@@ -66,7 +70,8 @@ for _f in (lib.sa_pool_blocks, lib.sa_select_mask_topk_topp, lib.sa_select_from_
            lib.sa_pool_select_topk_topp, lib.sa_block_scores, lib.sa_static_mask,
            lib.sa_squad_attn_fwd, lib.sa_kmeans, lib.sa_cluster_sort, lib.sa_centroid_topp,
            lib.sa_cluster_attn_fwd, lib.sa_svg2_attn_fwd,
-           lib.sa_block_sparse_attn_fwd, lib.sa_dense_attn_fwd, lib.sa_get_device_error,
+           lib.sa_block_sparse_attn_fwd, lib.sa_sparsepr_attn_fwd, lib.sa_dense_attn_fwd,
+           lib.sa_get_device_error,
            lib.sa_set_wait_limit_ns, lib.sa_probe_bounded_wait, lib.sa_num_blocks):
     _f.restype = _I
 lib.sa_get_error_string.restype = ctypes.c_char_p
@@ -291,6 +296,42 @@ def block_sparse_attn_fwd(q, k, v, kv_idx, kv_cnt, bs: int, scale: float | None 
     _check(lib.sa_block_sparse_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_idx), _ptr(kv_cnt),
                                         _ptr(o), B, H, N, d, bs, float(scale or 0.0), _ptr(ws),
                                         ws.numel(), _stream(q.device)), "sa_block_sparse_attn_fwd")
+    return o
+
+
+def sparsepr_attn_fwd(q, k, v, kv_idx, kv_cnt, probes, bs: int, scale: float | None = None,
+                      o=None, workspace=None):
+    """Block-sparse attention over (kv_idx, kv_cnt) corrected by the probe fit of SparsePR with the
+    exact outputs of the probe rows probes [B, H, m] int32 -> O [B, H, N, d] bf16."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, torch.bfloat16, 4)
+    _need(kv_idx, "kv_idx", torch.int32, 4)
+    _need(kv_cnt, "kv_cnt", torch.int32, 3)
+    _need(probes, "probes", torch.int32, 3)
+    B, H, N, d = q.shape
+    nb = num_blocks(N, bs)
+    m = probes.shape[2]
+    o = o if o is not None else torch.empty_like(q)
+    _need(o, "o", torch.bfloat16, 4)
+    for n, t in (("k", k), ("v", v), ("o", o)):
+        _shape(t, n, q.shape)
+    _shape(kv_idx, "kv_idx", (B, H, nb, nb))
+    _shape(kv_cnt, "kv_cnt", (B, H, nb))
+    _shape(probes, "probes", (B, H, m))
+    nbytes = int(lib.sa_sparsepr_workspace_bytes(B, H, N, d, m))
+    if nbytes == 0:
+        raise SAError(SA_ERR_INVALID_ARG, "sa_sparsepr_workspace_bytes")
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    _need(workspace, "workspace", torch.uint8, 1)
+    if workspace.numel() < nbytes:
+        raise ValueError(f"workspace must hold {nbytes} bytes, got {workspace.numel()}")
+    _same_device(q, k=k, v=v, o=o, kv_idx=kv_idx, kv_cnt=kv_cnt, probes=probes,
+                 workspace=workspace)
+    _check(lib.sa_sparsepr_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_idx), _ptr(kv_cnt),
+                                    _ptr(probes), m, _ptr(o), B, H, N, d, bs,
+                                    float(scale or 0.0), _ptr(workspace), workspace.numel(),
+                                    _stream(q.device)), "sa_sparsepr_attn_fwd")
     return o
 
 

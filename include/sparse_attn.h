@@ -278,6 +278,32 @@ sa_status sa_block_sparse_attn_fwd_noalloc(const void *q, const void *k, const v
                                            int B, int H, int N, int d, int bs, float scale,
                                            void *stream);
 
+/*
+ * SparsePR: block-sparse attention followed by the probe-fitted residual correction (page
+ * "Partition the Support, Reconstruct the Residual: Training-Free Sparse Attention for Video
+ * Generation and World Models", abstract and summary section 3: a few probe queries are computed
+ * exactly, and their residuals against the sparse output are fitted by an affine map of the
+ * sparse output in the observed output subspace, which then corrects every row).
+ *   O_s = sa_block_sparse_attn_fwd(q, k, v, kv_idx, kv_cnt);  per head, with P = probes[b, h, :]
+ *   X = [O_s[P], 1], R = exact(P) - O_s[P], W = X^+ R (minimum norm), O = O_s + [O_s, 1] W.
+ * probes  : [B, H, m] int32 token ids in [0, N) chosen by the caller (ids outside are clamped);
+ *           1 <= m <= min(N, 8192).  Repeated ids are allowed.
+ * q, k, v, kv_idx, kv_cnt, o, bs, scale: as sa_block_sparse_attn_fwd.
+ * workspace: device memory of sa_sparsepr_workspace_bytes(B, H, N, d, m) bytes, 16-byte
+ *           aligned, owned by the caller (probe rows, their exact outputs, the fp64 fit).
+ * Arithmetic: the sparse and exact outputs in bf16 (fp32 accumulation on the tensor cores), the
+ * fit in fp64 (normal equations of the smaller side, Cholesky with a ridge of 1e-12 times the
+ * mean diagonal), the correction in fp32 rounded to bf16 in place in o.
+ */
+sa_status sa_sparsepr_attn_fwd(const void *q, const void *k, const void *v,
+                               const int32_t *kv_idx, const int32_t *kv_cnt,
+                               const int32_t *probes, int m, void *o, int B, int H, int N, int d,
+                               int bs, float scale, void *workspace, size_t workspace_bytes,
+                               void *stream);
+
+/* Bytes of device workspace sa_sparsepr_attn_fwd needs (0 for unsupported arguments). */
+size_t sa_sparsepr_workspace_bytes(int B, int H, int N, int d, int m);
+
 /* Human-readable name of a status code (static storage). */
 const char *sa_get_error_string(sa_status status);
 

@@ -171,6 +171,34 @@ def test_noalloc_attention_argument_checks(lib):
     assert f(A, A, A, A, A, o_host, 1, 1, 256, 128, 128, 0.0, S) == 1  # o not device memory
 
 
+def test_sparsepr_argument_checks(lib):
+    lib.sa_sparsepr_workspace_bytes.restype = ctypes.c_size_t
+    lib.sa_sparsepr_workspace_bytes.argtypes = [ctypes.c_int] * 5
+    W = lib.sa_sparsepr_workspace_bytes(1, 2, 1000, 128, 40)
+    assert W > 2 * 40 * 128 * 2  # at least the gathered probe rows
+    assert lib.sa_sparsepr_workspace_bytes(1, 2, 1000, 96, 40) == 0      # unsupported d
+    assert lib.sa_sparsepr_workspace_bytes(1, 2, 1000, 128, 0) == 0      # no probes
+    assert lib.sa_sparsepr_workspace_bytes(1, 2, 1000, 128, 9000) == 0   # too many probes
+    f = lib.sa_sparsepr_attn_fwd
+    f.argtypes = ([ctypes.c_void_p] * 6 + [ctypes.c_int, ctypes.c_void_p] + [ctypes.c_int] * 5
+                  + [ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p])
+    ok = lambda **kw: f(kw.get("q", A), A, A, A, A, kw.get("pr", A), kw.get("m", 40),
+                        kw.get("o", A), 1, 2, kw.get("N", 1000), kw.get("d", 128),
+                        kw.get("bs", 128), kw.get("s", 0.0), kw.get("ws", A2), kw.get("wb", W), S)
+    assert ok(q=NUL) == 1
+    assert ok(pr=NUL) == 1
+    assert ok(o=NUL) == 1
+    assert ok(ws=NUL) == 1
+    assert ok(wb=W - 1) == 1
+    assert ok(m=0) == 1
+    assert ok(m=1001) == 1           # more probes than tokens
+    assert ok(d=96) == 2
+    assert ok(bs=32) == 2
+    assert ok(s=float("nan")) == 1
+    assert ok(pr=MIS4) == 1
+    assert ok(o=MIS) == 1
+
+
 def test_python_binding_imports():
     import block_sparse_attention_blocks_b200 as pkg
 
