@@ -284,6 +284,65 @@ def cpu_estimate(w, s, total_flops):
     return ms, total_flops / (ms * 1e-3) / 1e12
 
 
+ORACLE_CONFIGS = (("pr1_1k", None), ("wan1.3b_480p", 64), ("stress_mixed", 64))
+
+
+def oracle_config_timing(name: str, qblocks):
+    """The oracle on workload `name`: pooling and selection of every head in full, then masked
+    attention of every query block (qblocks None) or of `qblocks` seeded query blocks spread over
+    the heads, extrapolated to the whole call by executed-pair FLOPs.  Returns a dict."""
+    import oracle
+    from block_sparse_attention_blocks_b200 import workloads as W
+
+    w = W.get(name)
+    q, k, v = W.make_qkv(w)
+    BH, N, d, bs, nb = w.B * w.H, w.N, w.d, w.bs, w.nb
+    qf, kf, vf = (x.reshape(BH, N, d) for x in (q, k, v))
+    t0 = time.perf_counter()
+    sel = oracle.select(oracle.pool_blocks(qf, bs), oracle.pool_blocks(kf, bs), w.topk, w.topp,
+                        w.scale)
+    t_ps = time.perf_counter() - t0
+    mask = sel.mask.reshape(BH, nb, nb)
+    last = N - (nb - 1) * bs
+    rows_of = np.full(nb, float(bs))
+    rows_of[-1] = last
+    cols = mask.sum(axis=2) * bs - (bs - last) * mask[:, :, nb - 1]
+    flops_block = 4.0 * d * rows_of[None, :] * cols  # [BH, nb]
+    if qblocks is None:
+        picks = [(h, i) for h in range(BH) for i in range(nb)]
+    else:
+        rng = np.random.default_rng(0)
+        picks = sorted({(int(rng.integers(BH)), int(rng.integers(nb))) for _ in range(qblocks)})
+    t0 = time.perf_counter()
+    oracle.masked_attention(qf, kf, vf, mask, bs, w.scale, picks)
+    t_att = time.perf_counter() - t0
+    f_sample = float(sum(flops_block[h, i] for h, i in picks))
+    f_call = float(flops_block.sum())
+    ms_call = (t_ps + t_att * f_call / max(f_sample, 1.0)) * 1e3
+    return {"workload": name, "threads": oracle.num_threads(), "full": qblocks is None,
+            "pool_select_s": t_ps, "attention_s": t_att, "attention_query_blocks": len(picks),
+            "ms_per_call": ms_call, "tflops": f_call / (ms_call * 1e-3) / 1e12}
+
+
+def oracle_config_timings():
+    """oracle_config_timing on every host core and, in a child process, on one core."""
+    out = []
+    for name, qb in ORACLE_CONFIGS:
+        rec = oracle_config_timing(name, qb)
+        env = dict(os.environ, OMP_NUM_THREADS="1")
+        code = ("import json, bench; print(json.dumps(bench.oracle_config_timing(%r, %r)))"
+                % (name, qb))
+        try:
+            res = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env,
+                                 capture_output=True, text=True, timeout=600)
+            one = json.loads(res.stdout.strip().splitlines()[-1])
+            rec["one_core"] = {"ms_per_call": one["ms_per_call"], "threads": one["threads"]}
+        except Exception as e:  # noqa: BLE001 - a missing one-core time is reported, not fatal
+            rec["one_core"] = {"error": str(e)[:200]}
+        out.append(rec)
+    return out
+
+
 def run_reference(args, w):
     """--impl reference: the oracle, as it stands, on the host cores."""
     world, rank, _ = dist_env()
@@ -536,9 +595,9 @@ def run_gpu(args, w):
                             "each position (SQuad, w = tokens of one frame)"}
         del osq
 
-    # ---------------------------------------------------------------- (k, p) sweep (opt-in)
+    # ---------------------------------------------------------------- (k, p) sweep
     sweep = None
-    if args.sweep and rank == 0 and w.sweep:
+    if not args.no_sweep and rank == 0 and w.sweep:
         peaks_s, _ = load_peaks()
         peak_s = peaks_s.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
         sweep = []
@@ -570,9 +629,9 @@ def run_gpu(args, w):
         if err:
             raise RuntimeError(f"device error {err} in the sweep")
 
-    # ---------------------------------------------------------------- SVG2 (context, opt-in)
+    # ---------------------------------------------------------------- SVG2 (context)
     svg2 = None
-    if args.svg2 and rank == 0:
+    if not args.no_svg2 and rank == 0:
         Cq, Ck = args.svg2_clusters
         # first centroid cache: the tokens at evenly spaced positions of each head; every later
         # call starts from the previous call's centroids (the cache of SVG2 section C)
@@ -583,35 +642,101 @@ def run_gpu(args, w):
                          dtype=torch.uint8, device=dev)
         _, sel = bsa.svg2_attn_fwd(q, k, v, cq, ck, args.svg2_iters, w.topp, o=osv, workspace=ws)
         torch.cuda.synchronize(dev)
-        s0, s1, s2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
         reps = 5
-        s0.record(stream)
+        ev[0].record(stream)
         for _ in range(reps):
             bsa.svg2_attn_fwd(q, k, v, cq, ck, args.svg2_iters, w.topp, o=osv, sel=sel,
                               workspace=ws)
-        s1.record(stream)
-        for _ in range(reps):  # the two k-means alone, from copies of the cache
-            bsa.kmeans(q, cq.clone(), args.svg2_iters)
-            bsa.kmeans(k, ck.clone(), args.svg2_iters)
-        s2.record(stream)
+        ev[1].record(stream)
+        # the stages of one call, through their own entry points: the two k-means (from copies
+        # of the cache), the centroid top-p, the attention over the selected clusters (cluster
+        # tables, permuted copies and the variable-length attention kernel)
+        cq2, ck2 = cq.clone(), ck.clone()
+        for _ in range(reps):
+            cq2.copy_(cq)
+            ck2.copy_(ck)
+            aq, _, _, qsz = bsa.kmeans(q, cq2, args.svg2_iters)
+            ak, _, _, ksz = bsa.kmeans(k, ck2, args.svg2_iters)
+        ev[2].record(stream)
+        for _ in range(reps):
+            sel2 = bsa.centroid_topp(cq2, ck2, ksz, w.topp)
+        ev[3].record(stream)
+        for _ in range(reps):
+            bsa.cluster_attn_fwd(q, k, v, aq, ak, sel2, o=osv)
+        ev[4].record(stream)
         torch.cuda.synchronize(dev)
         err = bsa.device_error()
         if err:
             raise RuntimeError(f"device error {err} in the SVG2 timing")
-        # the last call's clusters: its final assignment is the nearest centroid of the cache
-        _, _, _, qsz = bsa.kmeans(q, cq.clone(), 0)
-        _, _, _, ksz = bsa.kmeans(k, ck.clone(), 0)
         qsz, ksz = qsz.double(), ksz.double()
-        pairs_sv = float(torch.einsum("bha,bhaj,bhj->", qsz, sel.double(), ksz))
-        ms_sv = s0.elapsed_time(s1) / reps
+        pairs_sv = float(torch.einsum("bha,bhaj,bhj->", qsz, sel2.double(), ksz))
+        ms_sv = ev[0].elapsed_time(ev[1]) / reps
+        ms_att_sv = ev[3].elapsed_time(ev[4]) / reps
         f_sv = 4.0 * d * pairs_sv
+        # the nearest-centroid contraction of one k-means pass: 2 N C d per head
+        km_flops = 2.0 * B * H * N * d * (Cq + Ck) * (args.svg2_iters + 1)
+        ms_km = ev[1].elapsed_time(ev[2]) / reps
         svg2 = {"query_clusters": Cq, "key_clusters": Ck, "kmeans_iters": args.svg2_iters,
-                "topp": w.topp, "ms": ms_sv, "kmeans_ms": s1.elapsed_time(s2) / reps,
-                "density": pairs_sv / float(B * H * N * N),
+                "topp": w.topp, "ms": ms_sv, "density": pairs_sv / float(B * H * N * N),
                 "tflops": f_sv / (ms_sv * 1e-3) / 1e12,
+                "stages_ms": {"kmeans_q_and_k": ms_km,
+                              "centroid_topp": ev[2].elapsed_time(ev[3]) / reps,
+                              "cluster_attention": ms_att_sv},
+                "kmeans_assign_tflops": km_flops / (ms_km * 1e-3) / 1e12,
+                "cluster_attention_tflops": f_sv / (ms_att_sv * 1e-3) / 1e12,
                 "pattern": "k-means of Q and K warm-started from the previous call's centroids, "
                            "centroid top-p, attention over the selected clusters (SVG2)"}
-        del osv, ws, sel
+        del osv, ws, sel, sel2, cq2, ck2
+
+    # ---------------------------------------------------------------- SparsePR (context)
+    sparsepr = None
+    if not args.no_sparsepr and rank == 0:
+        m = min(args.sparsepr_probes, N)
+        gen = torch.Generator(device="cpu").manual_seed(7)
+        probes = torch.stack([torch.randperm(N, generator=gen)[:m].sort().values
+                              for _ in range(B * H)]).to(torch.int32).reshape(B, H, m).to(dev)
+        opr = torch.empty_like(q)
+        wsp = torch.empty(int(bsa.lib.sa_sparsepr_workspace_bytes(B, H, N, d, m)),
+                          dtype=torch.uint8, device=dev)
+        bsa.sparsepr_attn_fwd(q, k, v, kv_idx, kv_cnt, probes, bs, o=opr, workspace=wsp)
+        torch.cuda.synchronize(dev)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 5
+        s0.record(stream)
+        for _ in range(reps):
+            bsa.sparsepr_attn_fwd(q, k, v, kv_idx, kv_cnt, probes, bs, o=opr, workspace=wsp)
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        err = bsa.device_error()
+        if err:
+            raise RuntimeError(f"device error {err} in the SparsePR timing")
+        ms_pr = s0.elapsed_time(s1) / reps
+        sparsepr = {"probes_per_head": m, "ms": ms_pr,
+                    "correction_ms": ms_pr - t_att,
+                    "pattern": "block-sparse attention at the workload's selection, the exact "
+                               "outputs of m seeded probe rows per head, the per-head fp64 "
+                               "least-squares fit of their residuals and the correction of every "
+                               "row (SparsePR); correction_ms = ms - the sparse attention alone"}
+        del opr, wsp, probes
+
+    # ---------------------------------------------------------------- pool + select, L2 flushed
+    ps_flushed = None
+    if rank == 0:
+        flush = torch.empty(512 * 2**20, dtype=torch.uint8, device=dev)
+        tot = 0.0
+        reps = 10
+        for _ in range(reps):
+            flush.zero_()
+            f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            f0.record(stream)
+            bsa.pool_select_topk_topp(q, k, bs, w.topk, w.topp, qp=qp, kp=kp, mask=mask,
+                                      kv_idx=kv_idx, kv_cnt=kv_cnt)
+            f1.record(stream)
+            torch.cuda.synchronize(dev)
+            tot += f0.elapsed_time(f1)
+        ps_flushed = tot / reps
+        del flush
 
     peaks, peak_src = load_peaks()
     # the attention kernel is timed alone in a short region: the burst GEMM figure is its peak
@@ -655,8 +780,11 @@ def run_gpu(args, w):
                                  "bytes_per_call": ps_bytes,
                                  "timed": "sa_pool_select_topk_topp: pooling, block scores "
                                           "and row selection kernels",
-                                 "peak_source": f"hbm_gbs of {peak_src}"},
-        "kernels_ms": {"pool_select": t_ps, "attention": t_att},
+                                 "peak_source": f"hbm_gbs of {peak_src}",
+                                 "frac_l2_flushed": (ps_bytes / (ps_flushed * 1e-3) / 1e9 / peak_hbm
+                                                     if ps_flushed else None)},
+        "kernels_ms": {"pool_select": t_ps, "attention": t_att,
+                       "pool_select_l2_flushed": ps_flushed},
         "gpu_launches": launches_per_step(B * H) * args.steps,
         "clocks": clk,
     }
@@ -670,6 +798,8 @@ def run_gpu(args, w):
         line["squad"] = squad
     if svg2:
         line["svg2"] = svg2
+    if sparsepr:
+        line["sparsepr"] = sparsepr
     if sweep:
         line["sweep"] = sweep
 
@@ -684,6 +814,8 @@ def run_gpu(args, w):
                       f"({s['t_pool_select']:.2f} s) and masked attention of {s['qblocks']} seeded "
                       f"query blocks ({s['t_attn']:.2f} s); extrapolated to the call by heads and "
                       f"by executed-pair FLOPs"}
+        if not args.no_oracle_configs:
+            line["cpu_baseline"]["other_workloads"] = oracle_config_timings()
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -708,11 +840,17 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-static", action="store_true", help="skip the static-pattern timing")
     ap.add_argument("--no-squad", action="store_true", help="skip the SQuad timing")
-    ap.add_argument("--sweep", action="store_true",
-                    help="also time pool+select and attention at every (k, p) point of the "
-                         "workload's sweep")
-    ap.add_argument("--svg2", action="store_true",
-                    help="also time the SVG2 path (k-means, centroid top-p, cluster attention)")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the pool+select and attention timings at every (k, p) point of "
+                         "the workload's sweep")
+    ap.add_argument("--no-svg2", action="store_true",
+                    help="skip the SVG2 path timing (k-means, centroid top-p, cluster attention)")
+    ap.add_argument("--no-sparsepr", action="store_true",
+                    help="skip the SparsePR timing (sparse attention + probe-fitted correction)")
+    ap.add_argument("--sparsepr-probes", type=int, default=256,
+                    help="probe query rows per head for the SparsePR timing")
+    ap.add_argument("--no-oracle-configs", action="store_true",
+                    help="skip the oracle timings on the other workloads")
     ap.add_argument("--svg2-clusters", type=lambda s: tuple(int(x) for x in s.split(",")),
                     default=(128, 256), help="query,key cluster counts for --svg2")
     ap.add_argument("--svg2-iters", type=int, default=2, help="k-means update steps for --svg2")

@@ -55,9 +55,13 @@ cudaError_t attn_varlen_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const 
                             unsigned long long wait_ns, int num_sms, unsigned int *workspace,
                             cudaStream_t st);
 
+// parts [BH, 3, C, d] bf16 and norms [BH, C] fp32 are scratch for the tensor-core assignment;
+// tx / tp are tensor maps of x ({d, N, BH}) and parts ({d, C, 3 BH}), 128-row boxes.  With
+// parts == nullptr the SIMT assignment runs.
 cudaError_t kmeans_lloyd(const void *x, float *cent, int32_t *assign, int32_t *perm,
                          int32_t *cstart, int32_t *csize, long long BH, int N, int d, int C,
-                         int iters, cudaStream_t st);
+                         int iters, void *parts, float *norms, const CUtensorMap *tx,
+                         const CUtensorMap *tp, unsigned long long wait_ns, cudaStream_t st);
 
 cudaError_t cluster_sort(const int32_t *assign, long long BH, int N, int C, int32_t *perm,
                          int32_t *cstart, int32_t *csize, cudaStream_t st);

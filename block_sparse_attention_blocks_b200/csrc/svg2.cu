@@ -399,6 +399,242 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4 *__restric
     }
 }
 
+}  // namespace bsa
+
+namespace bsa {
+
+template <int D>
+struct KmTcCfg {
+    static constexpr int CHUNKS = D / 64;
+    static constexpr int TILE = CHUNKS * 16384;  // 128 rows x D bf16, 128-byte swizzled chunks
+    static constexpr int OFF_X = 0;
+    static constexpr int OFF_P = TILE;                 // stage s, part p: OFF_P + (s*3 + p)*TILE
+    static constexpr int OFF_BAR = OFF_P + 6 * TILE;
+    static constexpr int SMEM = OFF_BAR + 128 + 1024;  // + alignment slack
+};
+
+enum { KB_XF, KB_PF0, KB_PF1, KB_PE0, KB_PE1, KB_SF0, KB_SF1, KB_SE0, KB_SE1, KB_FIN, KB_COUNT };
+
+template <int D>
+__global__ void __launch_bounds__(256, 1)
+    kmeans_assign_tc_kernel(const __grid_constant__ CUtensorMap tmX,
+                            const __grid_constant__ CUtensorMap tmP, const float *__restrict__ norms,
+                            int32_t *__restrict__ assign, int N, int C,
+                            unsigned long long wait_ns) {
+    using Cf = KmTcCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cf::OFF_BAR);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + Cf::OFF_BAR + 8 * KB_COUNT);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Cf::OFF_BAR + 8 * KB_COUNT + 4);
+    static_assert(8 * KB_COUNT + 8 <= 128, "barrier area");
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.y, n0 = blockIdx.x * 128;
+    const int T = (C + 127) / 128;  // centroid tiles
+    auto bar = [&](int b) { return smem_u32(&bars[b]); };
+    const uint32_t sX = smem_u32(smem + Cf::OFF_X);
+    auto sP = [&](int s, int p) { return smem_u32(smem + Cf::OFF_P + (s * 3 + p) * Cf::TILE); };
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(KB_XF), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(KB_PF0 + s), 1);
+            mbar_init(bar(KB_PE0 + s), 1);
+            mbar_init(bar(KB_SF0 + s), 1);
+            mbar_init(bar(KB_SE0 + s), 128);
+        }
+        mbar_init(bar(KB_FIN), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tmX);
+        prefetch_tmap(&tmP);
+    }
+    if (warp == 2) {
+        tmem_alloc(smem_u32(tmem_holder), 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_holder;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------------ producer
+        bool ok = true;
+        uint32_t issued = 0;
+        if (lane == 0) {
+            mbar_arrive_expect_tx(bar(KB_XF), Cf::TILE);
+            for (int c = 0; c < Cf::CHUNKS; ++c)
+                tma_load_3d(sX + c * 16384, &tmX, bar(KB_XF), c * 64, n0, bh);
+        }
+        for (int t = 0; t < T && ok; ++t) {
+            const int s = t & 1;
+            if (t >= 2 && !(ok = warp_wait(bar(KB_PE0 + s), ((t >> 1) - 1) & 1, wait_ns, abort_flag, 0x91, t)))
+                break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bar(KB_PF0 + s), 3 * Cf::TILE);
+                for (int p = 0; p < 3; ++p)
+                    for (int c = 0; c < Cf::CHUNKS; ++c)
+                        tma_load_3d(sP(s, p) + c * 16384, &tmP, bar(KB_PF0 + s), c * 64, t * 128,
+                                    bh * 3 + p);
+            }
+            ++issued;
+        }
+        if (lane == 0) {  // every started copy lands before the CTA leaves
+            int never = 0;
+            mbar_wait(bar(KB_XF), 0, wait_ns, (volatile int *)&never, 0x98, 0);
+            for (uint32_t t = (issued > 2 ? issued - 2 : 0); t < issued; ++t)
+                mbar_wait(bar(KB_PF0 + (t & 1)), (t >> 1) & 1, wait_ns, (volatile int *)&never, 0x99, t);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------------ MMA issuer
+        constexpr uint32_t IDESC = idesc_bf16_f32(128, 128, 0, 0);
+        bool ok = warp_wait(bar(KB_XF), 0, wait_ns, abort_flag, 0xA1, 0);
+        const uint64_t dX = smem_desc_sw128(sX, 16, 1024);
+        for (int t = 0; t < T && ok; ++t) {
+            const int s = t & 1;  // operand stage and accumulator buffer
+            if (!(ok = warp_wait(bar(KB_PF0 + s), (t >> 1) & 1, wait_ns, abort_flag, 0xA2, t))) break;
+            if (t >= 2 && !(ok = warp_wait(bar(KB_SE0 + s), ((t >> 1) - 1) & 1, wait_ns, abort_flag, 0xA3, t)))
+                break;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t acc = tbase + (uint32_t)(s * 128);
+#pragma unroll
+                for (int p = 0; p < 3; ++p) {
+                    const uint64_t dP = smem_desc_sw128(sP(s, p), 16, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint64_t off = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+                        mma_ss(acc, dX + off, dP + off, IDESC, (p > 0 || kk > 0) ? 1u : 0u);
+                    }
+                }
+                mma_commit(bar(KB_SF0 + s));
+                mma_commit(bar(KB_PE0 + s));
+            }
+            __syncwarp();
+        }
+        if (lane == 0) {
+            int never = 0;
+            mma_commit(bar(KB_FIN));
+            mbar_wait(bar(KB_FIN), 0, wait_ns, (volatile int *)&never, 0xA4, 0);
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------------ epilogue
+        const int q4 = warp & 3;
+        const int r = q4 * 32 + lane;  // token row of the tile == TMEM lane
+        const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+        float best = INFINITY;
+        int arg = 0;
+        bool ok = true;
+        for (int t = 0; t < T && ok; ++t) {
+            const int s = t & 1;
+            // lane e holds the norm of column q * 32 + e (padding centroids are never nearest);
+            // no barrier among the epilogue warps, so a warp that gives up cannot stall the rest
+            float nv[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int c = t * 128 + q * 32 + lane;
+                nv[q] = c < C ? norms[(size_t)bh * C + c] : INFINITY;
+            }
+            if (!(ok = warp_wait(bar(KB_SF0 + s), (t >> 1) & 1, wait_ns, abort_flag, 0xB1, t))) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int q = 0; q < 4; ++q) {
+                uint32_t v[32];
+                tmem_ld32(tbase + lane_off + (uint32_t)(s * 128 + q * 32), v);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const float cn = __shfl_sync(0xffffffffu, nv[q], e);
+                    const float dist = fmaf(-2.f, __uint_as_float(v[e]), cn);
+                    if (dist < best) {
+                        best = dist;
+                        arg = t * 128 + q * 32 + e;
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(bar(KB_SE0 + s));
+        }
+        if (ok && n0 + r < N) assign[(size_t)bh * N + n0 + r] = arg;
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 2) tmem_dealloc(tbase, 256);
+}
+
+// parts[bh, p, c, :] (p = 0, 1, 2: h, m, l of cent[bh, c, :]) and norms[bh, c] = |cent[bh, c]|^2
+template <int D>
+__global__ void __launch_bounds__(256) centroid_split_kernel(const float *__restrict__ cent,
+                                                             __nv_bfloat16 *__restrict__ parts,
+                                                             float *__restrict__ norms, int C) {
+    const int bh = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c = blockIdx.x * 8 + warp;
+    if (c >= C) return;
+    const float *src = cent + ((size_t)bh * C + c) * D;
+    uint16_t *dst = reinterpret_cast<uint16_t *>(parts);
+    float s = 0.f;
+    for (int e = lane; e < D; e += 32) {
+        const float x = src[e];
+        s = fmaf(x, x, s);
+        const uint32_t h = __float_as_uint(x) & 0xFFFF0000u;
+        const float rm = x - __uint_as_float(h);
+        const uint32_t m = __float_as_uint(rm) & 0xFFFF0000u;
+        const uint32_t l = __float_as_uint(rm - __uint_as_float(m));
+        const size_t base = (((size_t)bh * 3) * C + c) * D + e;
+        dst[base] = (uint16_t)(h >> 16);
+        dst[base + (size_t)C * D] = (uint16_t)(m >> 16);
+        dst[base + 2 * (size_t)C * D] = (uint16_t)(l >> 16);
+    }
+    s = warp_sum(s);
+    if (lane == 0) norms[(size_t)bh * C + c] = s;
+}
+
+}  // namespace bsa
+
+namespace bsa {
+
+template <int D>
+static cudaError_t launch_assign_tc(const CUtensorMap &tx, const CUtensorMap &tp,
+                                    const float *norms, int32_t *assign, long long BH, int N,
+                                    int C, unsigned long long wait_ns, cudaStream_t st) {
+    using Cf = KmTcCfg<D>;
+    cudaError_t e = cudaFuncSetAttribute(kmeans_assign_tc_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((unsigned)((N + 127) / 128), (unsigned)BH);
+    kmeans_assign_tc_kernel<D><<<grid, 256, Cf::SMEM, st>>>(tx, tp, norms, assign, N, C, wait_ns);
+    return cudaGetLastError();
+}
+
+cudaError_t kmeans_assign_tc(const CUtensorMap &tx, const CUtensorMap &tp, const float *norms,
+                             int32_t *assign, long long BH, int N, int d, int C,
+                             unsigned long long wait_ns, cudaStream_t st) {
+    if (d == 128) return launch_assign_tc<128>(tx, tp, norms, assign, BH, N, C, wait_ns, st);
+    if (d == 64) return launch_assign_tc<64>(tx, tp, norms, assign, BH, N, C, wait_ns, st);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t centroid_split(const float *cent, void *parts, float *norms, long long BH, int C,
+                           int d, cudaStream_t st) {
+    const dim3 g((unsigned)((C + 7) / 8), (unsigned)BH);
+    auto *p = reinterpret_cast<__nv_bfloat16 *>(parts);
+    if (d == 128)
+        centroid_split_kernel<128><<<g, 256, 0, st>>>(cent, p, norms, C);
+    else
+        centroid_split_kernel<64><<<g, 256, 0, st>>>(cent, p, norms, C);
+    return cudaGetLastError();
+}
+
+}  // namespace bsa
+
+namespace bsa {
+
 // ------------------------------------------------------------------------------------------
 // host side
 // ------------------------------------------------------------------------------------------
@@ -409,18 +645,27 @@ static unsigned grid_for(long long work, int per_block, int num_sms) {
     return (unsigned)(g > 0 ? g : 1);
 }
 
+// parts: [BH, 3, C, d] bf16 scratch and norms [BH, C] fp32 scratch for the tensor-core
+// assignment; tx / tp: tensor maps of x ({d, N, BH}, 128-row boxes) and of parts
+// ({d, C, 3 BH}, 128-row boxes).  With parts == nullptr the SIMT assignment runs.
 cudaError_t kmeans_lloyd(const void *x, float *cent, int32_t *assign, int32_t *perm,
                          int32_t *cstart, int32_t *csize, long long BH, int N, int d, int C,
-                         int iters, cudaStream_t st) {
+                         int iters, void *parts, float *norms, const CUtensorMap *tx,
+                         const CUtensorMap *tp, unsigned long long wait_ns, cudaStream_t st) {
     const dim3 ga((unsigned)((N + 255) / 256), (unsigned)BH);
     const dim3 gu((unsigned)C, (unsigned)BH);
     const size_t sort_smem = (size_t)9 * C * sizeof(int32_t);
     const auto *xb = reinterpret_cast<const __nv_bfloat16 *>(x);
     for (int it = 0;; ++it) {
-        if (d == 128)
+        if (parts) {
+            cudaError_t e = centroid_split(cent, parts, norms, BH, C, d, st);
+            if (e == cudaSuccess) e = kmeans_assign_tc(*tx, *tp, norms, assign, BH, N, d, C, wait_ns, st);
+            if (e != cudaSuccess) return e;
+        } else if (d == 128) {
             kmeans_assign_kernel<128><<<ga, 256, 0, st>>>(xb, cent, assign, N, C);
-        else
+        } else {
             kmeans_assign_kernel<64><<<ga, 256, 0, st>>>(xb, cent, assign, N, C);
+        }
         cluster_sort_kernel<<<(unsigned)BH, 256, sort_smem, st>>>(assign, N, C, perm, cstart, csize);
         if (it == iters) break;
         if (d == 128)
@@ -496,6 +741,8 @@ struct ClusterWorkspace {
     // the full path only: assignments, centroid scores (then the selection's id lists) and counts
     int32_t *assign_q, *assign_k, *sel_cnt;
     float *logits;
+    void *parts;   // centroid parts for the tensor-core assignment, sized for max(Cq, Ck)
+    float *norms;
     int U, tstride;
 };
 
@@ -527,11 +774,16 @@ size_t cluster_workspace(int B, int H, int N, int d, int Cq, int Ck, bool full, 
     t.vp = take(BH * N * (size_t)d * 2);
     t.assign_q = t.assign_k = t.sel_cnt = nullptr;
     t.logits = nullptr;
+    t.parts = nullptr;
+    t.norms = nullptr;
     if (full) {
         t.assign_q = (int32_t *)take(BH * N * 4);
         t.assign_k = (int32_t *)take(BH * N * 4);
         t.logits = (float *)take(BH * Cq * (size_t)Ck * 4);
         t.sel_cnt = (int32_t *)take(BH * Cq * 4);
+        const size_t Cm = (size_t)(Cq > Ck ? Cq : Ck);
+        t.parts = take(BH * 3 * Cm * d * 2);
+        t.norms = (float *)take(BH * Cm * 4);
     }
     t.U = U;
     t.tstride = tstride;
@@ -587,19 +839,34 @@ cudaError_t centroid_select(const float *cq, const float *ck, const int32_t *siz
 
 }  // namespace
 
+extern "C" size_t sa_kmeans_workspace_bytes(int B, int H, int C, int d) {
+    if (B <= 0 || H <= 0 || C <= 0 || d <= 0) return 0;
+    const size_t BH = (size_t)B * H;
+    return round256(BH * 3 * (size_t)C * d * 2) + round256(BH * (size_t)C * 4);
+}
+
 extern "C" sa_status sa_kmeans(const void *x, float *cent, int32_t *assign, int32_t *perm,
                                int32_t *cstart, int32_t *csize, int B, int H, int N, int d, int C,
-                               int iters, void *stream) {
-    if (!x || !cent || !assign || !perm || !cstart || !csize) return SA_ERR_INVALID_ARG;
+                               int iters, void *workspace, size_t workspace_bytes, void *stream) {
+    if (!x || !cent || !assign || !perm || !cstart || !csize || !workspace) return SA_ERR_INVALID_ARG;
     if (!shape_ok(B, H, N) || !clusters_ok(C) || iters < 0) return SA_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return SA_ERR_UNSUPPORTED;
+    if (workspace_bytes < sa_kmeans_workspace_bytes(B, H, C, d) || !aligned16(workspace))
+        return SA_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(cent) || !aligned4(assign) || !aligned4(perm) ||
         !aligned4(cstart) || !aligned4(csize))
         return SA_ERR_INVALID_ARG;
     int dev;
     if (!select_device(assign, &dev)) return SA_ERR_INVALID_ARG;
-    return from_cuda(bsa::kmeans_lloyd(x, cent, assign, perm, cstart, csize, (long long)B * H, N, d,
-                                       C, iters, (cudaStream_t)stream));
+    const long long BH = (long long)B * H;
+    void *parts = workspace;
+    float *norms = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) +
+                                             round256((size_t)BH * 3 * C * d * 2));
+    CUtensorMap tx, tp;
+    if (!make_tmap(&tx, x, BH, N, d, 128) || !make_tmap(&tp, parts, BH * 3, C, d, 128))
+        return SA_ERR_CUDA;
+    return from_cuda(bsa::kmeans_lloyd(x, cent, assign, perm, cstart, csize, BH, N, d, C, iters,
+                                       parts, norms, &tx, &tp, g_wait_ns, (cudaStream_t)stream));
 }
 
 extern "C" sa_status sa_cluster_sort(const int32_t *assign, int B, int H, int N, int C,
@@ -700,11 +967,15 @@ extern "C" sa_status sa_svg2_attn_fwd(const void *q, const void *k, const void *
     ClusterWorkspace w;
     cluster_workspace(B, H, N, d, Cq, Ck, true, workspace, &w);
     const long long BH = (long long)B * H;
+    CUtensorMap txq, txk, tpq, tpk;
+    if (!make_tmap(&txq, q, BH, N, d, 128) || !make_tmap(&txk, k, BH, N, d, 128) ||
+        !make_tmap(&tpq, w.parts, BH * 3, Cq, d, 128) || !make_tmap(&tpk, w.parts, BH * 3, Ck, d, 128))
+        return SA_ERR_CUDA;
     cudaError_t e = bsa::kmeans_lloyd(q, cent_q, w.assign_q, w.perm_q, w.qstart, w.qsize, BH, N, d,
-                                      Cq, iters, st);
+                                      Cq, iters, w.parts, w.norms, &txq, &tpq, g_wait_ns, st);
     if (e == cudaSuccess)
         e = bsa::kmeans_lloyd(k, cent_k, w.assign_k, w.perm_k, w.kstart, w.ksize, BH, N, d, Ck,
-                              iters, st);
+                              iters, w.parts, w.norms, &txk, &tpk, g_wait_ns, st);
     if (e == cudaSuccess)
         e = centroid_select(cent_q, cent_k, w.ksize, BH, Cq, Ck, d, topp, resolve_scale(scale, d),
                             sel, w.logits, w.sel_cnt, num_sms(dev), st);

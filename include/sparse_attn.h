@@ -155,10 +155,15 @@ sa_status sa_squad_attn_fwd(const void *q, const void *k, const void *v, void *o
  *   centroid by squared Euclidean distance in fp32, the lower index on a tie.  Outputs (int32):
  *   assign [B, H, N] the final cluster of each token; perm [B, H, N] the tokens in order of
  *   cluster, ascending within a cluster; cstart, csize [B, H, C] where each cluster's tokens sit
- *   in perm.  Cluster sums run in token order, so results repeat bit for bit.
+ *   in perm.  Cluster sums run in token order, so results repeat bit for bit.  The nearest
+ *   centroid runs on the tensor cores (rows exact in bf16, each fp32 centroid split exactly
+ *   into three bf16 parts, fp32 accumulation); workspace: sa_kmeans_workspace_bytes() bytes,
+ *   16-byte aligned, owned by the caller (the centroid parts and norms).
  */
+size_t sa_kmeans_workspace_bytes(int B, int H, int C, int d);
 sa_status sa_kmeans(const void *x, float *cent, int32_t *assign, int32_t *perm, int32_t *cstart,
-                    int32_t *csize, int B, int H, int N, int d, int C, int iters, void *stream);
+                    int32_t *csize, int B, int H, int N, int d, int C, int iters, void *workspace,
+                    size_t workspace_bytes, void *stream);
 
 /*
  * The stable order of the tokens by cluster id (the permutation of section A) alone:

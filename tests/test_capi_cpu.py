@@ -268,14 +268,21 @@ def test_squad_argument_checks(lib):
 
 def test_cluster_entry_point_argument_checks(lib):
     I, P, F, Z = ctypes.c_int, ctypes.c_void_p, ctypes.c_float, ctypes.c_size_t
+    lib.sa_kmeans_workspace_bytes.restype = Z
+    lib.sa_kmeans_workspace_bytes.argtypes = [I] * 4
+    Wk = lib.sa_kmeans_workspace_bytes(1, 2, 8, 64)
+    assert Wk >= 2 * 3 * 8 * 64 * 2 + 2 * 8 * 4       # centroid parts (bf16) and norms
+    assert lib.sa_kmeans_workspace_bytes(0, 2, 8, 64) == 0
     km = lib.sa_kmeans
-    km.argtypes = [P] * 6 + [I] * 6 + [P]
-    assert km(NUL, A, A, A, A, A, 1, 2, 100, 64, 8, 2, S) == 1
-    assert km(A, A, A, A, A, A, 1, 2, 100, 96, 8, 2, S) == 2          # d
-    assert km(A, A, A, A, A, A, 1, 2, 100, 64, 0, 2, S) == 1          # C < 1
-    assert km(A, A, A, A, A, A, 1, 2, 100, 64, 1025, 2, S) == 1       # C > 1024
-    assert km(A, A, A, A, A, A, 1, 2, 100, 64, 8, -1, S) == 1         # iters
-    assert km(A, MIS, A, A, A, A, 1, 2, 100, 64, 8, 2, S) == 1        # centroids need 16 B
+    km.argtypes = [P] * 6 + [I] * 6 + [P, Z, P]
+    assert km(NUL, A, A, A, A, A, 1, 2, 100, 64, 8, 2, A2, Wk, S) == 1
+    assert km(A, A, A, A, A, A, 1, 2, 100, 96, 8, 2, A2, Wk, S) == 2          # d
+    assert km(A, A, A, A, A, A, 1, 2, 100, 64, 0, 2, A2, Wk, S) == 1          # C < 1
+    assert km(A, A, A, A, A, A, 1, 2, 100, 64, 1025, 2, A2, Wk, S) == 1       # C > 1024
+    assert km(A, A, A, A, A, A, 1, 2, 100, 64, 8, -1, A2, Wk, S) == 1         # iters
+    assert km(A, MIS, A, A, A, A, 1, 2, 100, 64, 8, 2, A2, Wk, S) == 1        # centroids need 16 B
+    assert km(A, A, A, A, A, A, 1, 2, 100, 64, 8, 2, NUL, Wk, S) == 1         # no workspace
+    assert km(A, A, A, A, A, A, 1, 2, 100, 64, 8, 2, A2, Wk - 1, S) == 1      # workspace too small
     cs = lib.sa_cluster_sort
     cs.argtypes = [P] + [I] * 4 + [P] * 4
     assert cs(NUL, 1, 1, 10, 4, A, A, A, S) == 1
