@@ -11,7 +11,9 @@
 // query rows past the tile's count are computed but not stored.  The output row of permuted
 // query row s is written at its original position perm_q[s], which undoes the permutation.
 // The query tensor may have another length than the keys (Nq rows against N keys), e.g. a set
-// of gathered query rows attending to every key.
+// of gathered query rows attending to every key.  In the split form each query "cluster" is one
+// run of the keys and the kernel writes, per cluster, the fp32 output of that run with its
+// log2-sum-exp, for the caller to combine.
 //
 // The pipeline and the roles are those of the block-sparse kernel (one TMA producer lane, one
 // MMA issuer lane, a tensor-memory allocator warp and four softmax warps; S = Q K^T and O += P V
@@ -29,6 +31,9 @@ struct VarlenParams {
     const int32_t *tcnt;    // [BH * Cq] key tiles in each query cluster's list
     const int32_t *perm_q;  // [BH, Nq] original position of each permuted query row
     __nv_bfloat16 *o;       // [BH, Nq, D] in the original order
+    float *part_o;          // or, when set: [Cq, BH, Nq, D] fp32 O / l per query cluster ...
+    float *part_lse;        // ... and [Cq, BH, Nq] its log2-sum-exp (log2 l + the row's max)
+    long long BH;
     int N, Nq, Cq, tstride, units_per_head;  // N keys, Nq query (and output) rows
     long long nunits;       // BH * units_per_head
     float scale_log2;       // softmax scale * log2(e)
@@ -312,9 +317,15 @@ __global__ void __launch_bounds__(256, 2)
                     orig = 0;
                 }
             }
-            __nv_bfloat16 *orow = prm.o + ((size_t)w.bh * prm.Nq + orig) * D;
+            __nv_bfloat16 *orow = prm.o ? prm.o + ((size_t)w.bh * prm.Nq + orig) * D : nullptr;
+            const size_t prow = ((size_t)w.cluster * prm.BH + w.bh) * prm.Nq + orig;
             if (cnt == 0) {  // the cluster selected nothing: zeros
-                if (row_ok) {
+                if (row_ok && prm.part_o) {
+                    float4 *dst = reinterpret_cast<float4 *>(prm.part_o + prow * D);
+#pragma unroll 4
+                    for (int c = 0; c < D / 4; ++c) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    prm.part_lse[prow] = -INFINITY;
+                } else if (row_ok) {
                     const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
                     for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4 *>(orow)[c] = z;
@@ -380,6 +391,24 @@ __global__ void __launch_bounds__(256, 2)
             if (!(ok = warp_wait(bar(V_OD), (npv - 1) & 1, wns, abort_flag, 0x82, (uint32_t)u))) break;
             tc_fence_after();
             const float inv_l = 1.f / l;
+            if (prm.part_o) {  // fp32 partial output of this key list and its log2-sum-exp
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32(tOr + c * 32, v);
+                    if (row_ok) {
+                        float4 *dst = reinterpret_cast<float4 *>(prm.part_o + prow * D + c * 32);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            dst[q] = make_float4(__uint_as_float(v[4 * q]) * inv_l, __uint_as_float(v[4 * q + 1]) * inv_l,
+                                                 __uint_as_float(v[4 * q + 2]) * inv_l, __uint_as_float(v[4 * q + 3]) * inv_l);
+                    }
+                }
+                if (row_ok) prm.part_lse[prow] = m_ref + log2f(l);
+                tc_fence_before();
+                mbar_arrive(bar(V_ED));
+                continue;
+            }
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t v[32];
@@ -436,8 +465,11 @@ cudaError_t attn_varlen_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const 
                             const int32_t *tcnt, int tstride, const int32_t *perm_q, void *o,
                             long long BH, int N, int Nq, int Cq, int d, float scale,
                             unsigned long long wait_ns, int num_sms, unsigned int *workspace,
-                            cudaStream_t st) {
+                            cudaStream_t st, float *part_o, float *part_lse) {
     VarlenParams p;
+    p.part_o = part_o;
+    p.part_lse = part_lse;
+    p.BH = BH;
     p.units_per_head = units_per_head;
     p.tiles = tiles;
     p.tcnt = tcnt;

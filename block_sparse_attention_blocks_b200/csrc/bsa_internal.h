@@ -53,11 +53,10 @@ cudaError_t attn_varlen_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const 
                             const int32_t *tcnt, int tstride, const int32_t *perm_q, void *o,
                             long long BH, int N, int Nq, int Cq, int d, float scale,
                             unsigned long long wait_ns, int num_sms, unsigned int *workspace,
-                            cudaStream_t st);
+                            cudaStream_t st, float *part_o = nullptr, float *part_lse = nullptr);
 
 // parts [BH, 3, C, d] bf16 and norms [BH, C] fp32 are scratch for the tensor-core assignment;
-// tx / tp are tensor maps of x ({d, N, BH}) and parts ({d, C, 3 BH}), 128-row boxes.  With
-// parts == nullptr the SIMT assignment runs.
+// tx / tp are tensor maps of x ({d, N, BH}) and parts ({d, C, 3 BH}), 128-row boxes.
 cudaError_t kmeans_lloyd(const void *x, float *cent, int32_t *assign, int32_t *perm,
                          int32_t *cstart, int32_t *csize, long long BH, int N, int d, int C,
                          int iters, void *parts, float *norms, const CUtensorMap *tx,

@@ -17,122 +17,15 @@
 //   2. the probe rows of Q gathered into [BH, m, d]; their exact outputs by the variable-length
 //      attention kernel with one query cluster covering the m rows and one key list covering
 //      every key (128-key tiles, the last one ragged);
-//   3. X and R in fp64; W by one CTA per head in fp64: the normal equations of the smaller side,
-//      Cholesky with a ridge of 1e-12 times the mean diagonal (which keeps a rank-deficient X
-//      solvable and approximates the pseudo-inverse's minimum-norm choice);
-//   4. O += [O, 1] W in place on the bf16 output (W staged in shared memory per head).
+//   3. [O_s[P] | R] in fp64; the Gram products tiled over CTAs; W by one CTA per head in fp64:
+//      the normal equations of the smaller side, Cholesky in shared memory with a ridge of 1e-12
+//      times the mean diagonal (which keeps a rank-deficient X solvable and approximates the
+//      pseudo-inverse's minimum-norm choice);
+//   4. O += [O, 1] W in place on the bf16 output, on the tensor cores (W in two bf16 parts).
 #include "bsa_internal.h"
 #include "sparse_attn.h"
 
 namespace bsa {
-
-// ------------------------------------------------------------------------------------------
-// minimum-norm least squares for one head, by a team of threads (a CTA), fp64
-// ------------------------------------------------------------------------------------------
-namespace lsq {
-
-// In-place Cholesky of the k x k SPD matrix G (row-major, lower triangle used), G = L L^T.
-template <class Sync>
-__device__ void cholesky(double *G, int k, int tid, int nt, Sync sync) {
-    for (int j = 0; j < k; ++j) {
-        if (tid == 0) G[j * k + j] = sqrt(G[j * k + j] > 0.0 ? G[j * k + j] : 1e-300);
-        sync();
-        const double inv = 1.0 / G[j * k + j];
-        for (int i = j + 1 + tid; i < k; i += nt) G[i * k + j] *= inv;
-        sync();
-        // trailing update of the lower triangle: G[i][c] -= L[i][j] L[c][j], j < c <= i
-        const int w = k - j - 1;
-        const long long pairs = (long long)w * (w + 1) / 2;
-        for (long long p = tid; p < pairs; p += nt) {
-            // p -> (ii, cc) with 0 <= cc <= ii < w
-            int ii = (int)((sqrt(8.0 * (double)p + 1.0) - 1.0) / 2.0);
-            while ((long long)(ii + 1) * (ii + 2) / 2 <= p) ++ii;
-            while ((long long)ii * (ii + 1) / 2 > p) --ii;
-            const int cc = (int)(p - (long long)ii * (ii + 1) / 2);
-            const int i = j + 1 + ii, c = j + 1 + cc;
-            G[i * k + c] -= G[i * k + j] * G[c * k + j];
-        }
-        sync();
-    }
-}
-
-// Solve L L^T Y = B in place for `ncol` right-hand sides (B row-major k x ncol), one column per
-// thread.
-template <class Sync>
-__device__ void chol_solve(const double *L, int k, double *B, int ncol, int tid, int nt, Sync sync) {
-    for (int c = tid; c < ncol; c += nt) {
-        for (int i = 0; i < k; ++i) {  // forward: L y = b
-            double s = B[i * ncol + c];
-            for (int e = 0; e < i; ++e) s -= L[i * k + e] * B[e * ncol + c];
-            B[i * ncol + c] = s / L[i * k + i];
-        }
-        for (int i = k - 1; i >= 0; --i) {  // backward: L^T x = y
-            double s = B[i * ncol + c];
-            for (int e = i + 1; e < k; ++e) s -= L[e * k + i] * B[e * ncol + c];
-            B[i * ncol + c] = s / L[i * k + i];
-        }
-    }
-    sync();
-}
-
-// X [m x n] (n = d + 1, last column ones), R [m x d] -> W [n x d].
-// Scratch: G [min(m, n)^2], Z [min(m, n) * d].
-template <class Sync>
-__device__ void min_norm_lstsq(const double *X, const double *R, int m, int d, double *W, double *G,
-                          double *Z, double eps, int tid, int nt, Sync sync) {
-    const int n = d + 1;
-    if (m >= n) {
-        for (int p = tid; p < n * n; p += nt) {  // G = X^T X
-            const int i = p / n, c = p % n;
-            double s = 0.0;
-            for (int r = 0; r < m; ++r) s += X[r * n + i] * X[r * n + c];
-            G[p] = s;
-        }
-        for (int p = tid; p < n * d; p += nt) {  // Z = X^T R
-            const int i = p / d, c = p % d;
-            double s = 0.0;
-            for (int r = 0; r < m; ++r) s += X[r * n + i] * R[r * d + c];
-            Z[p] = s;
-        }
-        sync();
-        if (tid == 0) {
-            double tr = 0.0;
-            for (int i = 0; i < n; ++i) tr += G[i * n + i];
-            for (int i = 0; i < n; ++i) G[i * n + i] += eps * tr / n;
-        }
-        sync();
-        cholesky(G, n, tid, nt, sync);
-        chol_solve(G, n, Z, d, tid, nt, sync);
-        for (int p = tid; p < n * d; p += nt) W[p] = Z[p];
-        sync();
-    } else {
-        for (int p = tid; p < m * m; p += nt) {  // G = X X^T
-            const int i = p / m, c = p % m;
-            double s = 0.0;
-            for (int e = 0; e < n; ++e) s += X[i * n + e] * X[c * n + e];
-            G[p] = s;
-        }
-        for (int p = tid; p < m * d; p += nt) Z[p] = R[p];
-        sync();
-        if (tid == 0) {
-            double tr = 0.0;
-            for (int i = 0; i < m; ++i) tr += G[i * m + i];
-            for (int i = 0; i < m; ++i) G[i * m + i] += eps * tr / m;
-        }
-        sync();
-        cholesky(G, m, tid, nt, sync);
-        chol_solve(G, m, Z, d, tid, nt, sync);
-        for (int p = tid; p < n * d; p += nt) {  // W = X^T Z
-            const int i = p / d, c = p % d;
-            double s = 0.0;
-            for (int r = 0; r < m; ++r) s += X[r * n + i] * Z[r * d + c];
-            W[p] = s;
-        }
-        sync();
-    }
-}
-
-}  // namespace lsq
 
 // Qpr[bh, i, :] = Q[bh, probes[bh, i], :]   (16-byte vectors)
 __global__ void __launch_bounds__(256) gather_probe_rows_kernel(const uint4 *__restrict__ q,
@@ -151,126 +44,671 @@ __global__ void __launch_bounds__(256) gather_probe_rows_kernel(const uint4 *__r
     }
 }
 
-// X [BH, m, d + 1] and R [BH, m, d] in fp64 from O_s (bf16 [BH, N, d]) and E (bf16 [BH, m, d]).
-__global__ void __launch_bounds__(256) probe_residual_kernel(
-    const __nv_bfloat16 *__restrict__ os, const __nv_bfloat16 *__restrict__ e,
-    const int32_t *__restrict__ probes, double *__restrict__ X, double *__restrict__ R,
-    long long BH, int N, int m, int d) {
-    const long long total = BH * m * (d + 1);
-    for (long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x; x < total;
-         x += (long long)gridDim.x * blockDim.x) {
-        const long long row = x / (d + 1);  // bh * m + i
-        const int c = (int)(x - row * (d + 1));
-        if (c == d) {
-            X[x] = 1.0;
-            continue;
+// E = the exact probe outputs, combined from the S key splits by their log2-sum-exp weights
+// (fp64), and M [BH, m, 2 d] = [O_s[P] | E - O_s[P]] with O_s bf16 [BH, N, d].
+// po [S, BH, m, d] fp32 and plse [S, BH, m] are the split outputs of the variable-length kernel.
+// CTA of 256 threads = 256 / d rows at a time, thread = (row, column); a row's S weights are
+// computed once into shared memory.
+__global__ void __launch_bounds__(256) probe_merge_kernel(
+    const __nv_bfloat16 *__restrict__ os, const float *__restrict__ po, const float *__restrict__ plse,
+    const int32_t *__restrict__ probes, double *__restrict__ M, long long BH, int N, int m, int d, int S) {
+    __shared__ double s_w[4][64];
+    const long long rows = BH * m;
+    const int per = 256 / d, rr = threadIdx.x / d, c = threadIdx.x % d;
+    for (long long r0 = (long long)blockIdx.x * per; r0 < rows; r0 += (long long)gridDim.x * per) {
+        const long long row = r0 + rr;  // bh * m + i
+        const bool live = row < rows;
+        float lmax = -INFINITY;
+        if (live)
+            for (int sp = 0; sp < S; ++sp) lmax = fmaxf(lmax, plse[sp * rows + row]);
+        if (live && c < S) s_w[rr][c] = exp2((double)plse[c * rows + row] - (double)lmax);
+        __syncthreads();
+        if (live) {
+            double num = 0.0, den = 0.0;
+            for (int sp = 0; sp < S; ++sp) {
+                const double w = s_w[rr][sp];
+                num += w * (double)po[(sp * rows + row) * d + c];
+                den += w;
+            }
+            const long long bh = row / m;
+            const int t = min(max(probes[row], 0), N - 1);
+            const double o = (double)__bfloat162float(os[(bh * N + t) * d + c]);
+            M[row * 2 * d + c] = o;
+            M[row * 2 * d + d + c] = num / den - o;
         }
-        const long long bh = row / m;
-        const int t = min(max(probes[row], 0), N - 1);
-        const double o = (double)__bfloat162float(os[(bh * N + t) * d + c]);
-        X[x] = o;
-        R[row * d + c] = (double)__bfloat162float(e[row * d + c]) - o;
+        __syncthreads();
     }
 }
 
-// One CTA per head: W [BH, d + 1, d] (fp32) = X^+ R.  Scratch per head: G [k^2], Z [k d],
-// k = min(m, d + 1) (the normal equations of the smaller side), fp64.
-__global__ void __launch_bounds__(256) probe_solve_kernel(const double *__restrict__ X,
-                                                          const double *__restrict__ R,
-                                                          double *__restrict__ G,
-                                                          double *__restrict__ Z,
-                                                          double *__restrict__ Wd,
-                                                          float *__restrict__ W, int m, int d,
-                                                          double eps) {
-    const long long bh = blockIdx.x;
-    const int n = d + 1, k = m < n ? m : n;
-    auto sync = []() { __syncthreads(); };
-    double *w64 = Wd + bh * n * d;
-    lsq::min_norm_lstsq(X + bh * m * n, R + bh * m * d, m, d, w64, G + bh * k * k,
-                                Z + bh * (long long)k * d, eps, threadIdx.x, blockDim.x, sync);
-    for (int p = threadIdx.x; p < n * d; p += blockDim.x) W[bh * n * d + p] = (float)w64[p];
+// ------------------------------------------------------------------------------------------
+// the per-head fit W = X^+ R, X = [O_s[P], 1], fp64
+// ------------------------------------------------------------------------------------------
+// With m >= d + 1 probes (the usual case) W solves the normal equations
+//   (X^T X + ridge) W = X^T R,  X^T X = [[O^T O, O^T 1], [1^T O, m]],  X^T R = [O^T R; 1^T R]
+// (O = O_s[P]); the products O^T [O | R] and the column sums of [O | R] come from
+// probe_gram_kernel, tiled over many CTAs.  With fewer probes the smaller side is solved:
+// (X X^T + ridge) Y = R, W = X^T Y.  The ridge is 1e-12 times the mean diagonal.
+
+// C [BH, d, 2 d] = O^T [O | R] over the m probe rows (only tiles on or below the diagonal of
+// the O^T O block), sums [BH, 2 d] = column sums of [O | R].  CTA = one 64 x 64 tile of one
+// head (blockIdx.x < tiles) or the sums (blockIdx.x == tiles); thread = 4 x 4 outputs, rows
+// staged through shared memory 32 at a time.
+__global__ void __launch_bounds__(256) probe_gram_kernel(const double *__restrict__ M,
+                                                         double *__restrict__ C,
+                                                         double *__restrict__ sums, int m, int d) {
+    const long long bh = blockIdx.y;
+    const int w2 = 2 * d;
+    const double *Mh = M + bh * m * w2;
+    const int tcols = w2 / 64, tiles = (d / 64) * tcols;
+    if ((int)blockIdx.x == tiles) {
+        for (int j = threadIdx.x; j < w2; j += blockDim.x) {
+            double s = 0.0;
+            for (int r = 0; r < m; ++r) s += Mh[(long long)r * w2 + j];
+            sums[bh * w2 + j] = s;
+        }
+        return;
+    }
+    const int ti = blockIdx.x / tcols, tj = blockIdx.x % tcols;
+    if (tj < d / 64 && tj > ti) return;  // above the diagonal of the symmetric block
+    __shared__ double As[32][64];
+    __shared__ double Bs[32][64];
+    const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+    double acc[4][4] = {};
+    for (int r0 = 0; r0 < m; r0 += 32) {
+        for (int p = threadIdx.x; p < 32 * 64; p += 256) {
+            const int rr = p >> 6, cc = p & 63;
+            const bool in = r0 + rr < m;
+            const double *row = Mh + (long long)(r0 + rr) * w2;
+            As[rr][cc] = in ? row[ti * 64 + cc] : 0.0;
+            Bs[rr][cc] = in ? row[tj * 64 + cc] : 0.0;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int k = 0; k < 32; ++k) {
+            const double2 a01 = *reinterpret_cast<const double2 *>(&As[k][ty * 4]);
+            const double2 a23 = *reinterpret_cast<const double2 *>(&As[k][ty * 4 + 2]);
+            const double2 b01 = *reinterpret_cast<const double2 *>(&Bs[k][tx * 4]);
+            const double2 b23 = *reinterpret_cast<const double2 *>(&Bs[k][tx * 4 + 2]);
+            const double av[4] = {a01.x, a01.y, a23.x, a23.y};
+            const double bv[4] = {b01.x, b01.y, b23.x, b23.y};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fma(av[i], bv[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+    double *Ch = C + bh * d * w2;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) Ch[(long long)(ti * 64 + ty * 4 + i) * w2 + tj * 64 + tx * 4 + j] = acc[i][j];
 }
 
-// O[bh, t, :] += [O[bh, t, :], 1] W[bh]   in place on the bf16 output; CTA = 64 rows of one
-// head, thread = (row, 32-column block); W of the head staged in shared memory.
-template <int D>
-__global__ void __launch_bounds__(256) apply_correction_kernel(__nv_bfloat16 *__restrict__ o,
-                                                               const float *__restrict__ W,
-                                                               int N) {
-    constexpr int ROWS = 64, CB = D / 32;  // rows per CTA, column blocks per row
-    constexpr int TPR = 256 / ROWS;        // threads per row (4)
-    static_assert(CB % TPR == 0 || TPR % CB == 0, "layout");
-    extern __shared__ float sm_apply[];
-    float *ws = sm_apply;                  // [(D + 1) * D]
-    float *os = sm_apply + (D + 1) * D;    // [ROWS][D + 1]
+constexpr int kSolveThreads = 512;
+constexpr int kSolveCols = 32;  // right-hand-side columns per CTA
+
+__device__ __forceinline__ int tri(int i) { return i * (i + 1) / 2; }  // packed lower-row start
+
+__device__ __forceinline__ void tri_decode(int p, int &i, int &j) {  // p -> (i, j), j <= i
+    i = (int)((sqrt(8.0 * (double)p + 1.0) - 1.0) * 0.5);
+    while (tri(i + 1) <= p) ++i;
+    while (tri(i) > p) --i;
+    j = p - tri(i);
+}
+
+// CTA (column block cb, head bh): forms the k x k system (k = d + 1, or m when m <= d), factors
+// it in shared memory (packed lower triangle; every column block factors its own copy) and
+// solves for its 32 right-hand-side columns, then writes those columns of W: the first d rows
+// as two bf16 parts [BH, 2 d, d] (W_hi; W - W_hi) and the offset row [BH, d] fp32.
+__global__ void __launch_bounds__(kSolveThreads, 2)
+    probe_solve_kernel(const double *__restrict__ M, const double *__restrict__ C,
+                       const double *__restrict__ sums, __nv_bfloat16 *__restrict__ wparts,
+                       float *__restrict__ woff, int m, int d, double eps) {
+    extern __shared__ double sm_solve[];
+    constexpr int NC = kSolveCols;
     const long long bh = blockIdx.y;
-    const int r0 = blockIdx.x * ROWS;
-    for (int p = threadIdx.x; p < (D + 1) * D; p += 256) ws[p] = W[bh * (D + 1) * D + p];
-    for (int p = threadIdx.x; p < ROWS * D; p += 256) {
-        const int rr = p / D, c = p % D;
-        const int t = r0 + rr;
-        os[rr * (D + 1) + c] = t < N ? __bfloat162float(o[(bh * N + t) * D + c]) : 0.f;
+    const int c0 = blockIdx.x * NC;
+    const int n = d + 1, w2 = 2 * d;
+    const bool tall = m >= n;
+    const int k = tall ? n : m;
+    double *__restrict__ L = sm_solve;                 // packed lower triangle, tri(k) entries
+    double *__restrict__ invd = sm_solve + tri(k);     // [k] reciprocals of the factor's diagonal
+    double *__restrict__ Z = sm_solve + tri(k) + k;    // [k][NC] right-hand sides, then the solution
+    __shared__ double s_red[kSolveThreads / 32];
+    const int tid = threadIdx.x, nt = blockDim.x;
+    const int warp = tid >> 5, lane = tid & 31, nw = nt >> 5;
+    const double *Mh = M + bh * m * w2;
+
+    // 1. the system
+    if (tall) {
+        const double *Ch = C + bh * d * w2;
+        const double *sh = sums + bh * w2;
+        for (int p = tid; p < tri(k); p += nt) {
+            int i, j;
+            tri_decode(p, i, j);
+            L[p] = i < d ? Ch[(long long)i * w2 + j] : (j < d ? sh[j] : (double)m);
+        }
+        for (int p = tid; p < k * NC; p += nt) {
+            const int i = p / NC, c = c0 + p % NC;
+            Z[p] = i < d ? Ch[(long long)i * w2 + d + c] : sh[d + c];
+        }
+    } else {
+        for (int p = tid; p < tri(k); p += nt) {
+            int i, j;
+            tri_decode(p, i, j);
+            const double *xi = Mh + (long long)i * w2, *xj = Mh + (long long)j * w2;
+            double sum = 1.0;  // the ones column
+            for (int e = 0; e < d; ++e) sum = fma(xi[e], xj[e], sum);
+            L[p] = sum;
+        }
+        for (int p = tid; p < k * NC; p += nt) Z[p] = Mh[(long long)(p / NC) * w2 + d + c0 + p % NC];
     }
     __syncthreads();
-    const int rr = threadIdx.x / TPR, part = threadIdx.x % TPR;
-    const int t = r0 + rr;
-    for (int cb = part; cb < CB; cb += TPR) {
-        float acc[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) acc[j] = ws[D * D + cb * 32 + j];  // the offset row
-        for (int e = 0; e < D; ++e) {
-            const float a = os[rr * (D + 1) + e];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) acc[j] = fmaf(a, ws[e * D + cb * 32 + j], acc[j]);
-        }
-        if (t < N) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int c = cb * 32 + j;
-                o[(bh * N + t) * D + c] = __float2bfloat16(os[rr * (D + 1) + c] + acc[j]);
+    // ridge: eps times the mean diagonal
+    {
+        double sum = 0.0;
+        for (int i = tid; i < k; i += nt) sum += L[tri(i) + i];
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (lane == 0) s_red[warp] = sum;
+        __syncthreads();
+        double tr = 0.0;
+        for (int w = 0; w < nw; ++w) tr += s_red[w];
+        __syncthreads();
+        for (int i = tid; i < k; i += nt) L[tri(i) + i] += eps * tr / k;
+    }
+    __syncthreads();
+
+    // 2. factor G = L L^T in 8-column panels (right-looking): warp 0 factors the panel
+    // (columns i0 .. i1 - 1, every row below) column by column, lane = row; then every warp
+    // (warp = row, lane = column) subtracts the panel's rank-8 term from the trailing matrix.
+    // Non-positive pivots (rounding in a rank-deficient system) count as 1e-300.
+    constexpr int KB = 8;
+    for (int i0 = 0; i0 < k; i0 += KB) {
+        const int nb = min(KB, k - i0), i1 = i0 + nb;
+        if (warp == 0) {
+            for (int j = 0; j < nb; ++j) {
+                const int cj = i0 + j;
+                double piv = L[tri(cj) + cj];
+                piv = piv > 0.0 ? piv : 1e-300;
+                const double sq = sqrt(piv), inv = 1.0 / sq;
+                __syncwarp();
+                if (lane == 0) L[tri(cj) + cj] = sq;
+                for (int r = cj + 1 + lane; r < k; r += 32) L[tri(r) + cj] *= inv;
+                __syncwarp();
+                for (int cc = cj + 1; cc < i1; ++cc) {
+                    const double lcj = L[tri(cc) + cj];
+                    for (int r = cc + lane; r < k; r += 32) L[tri(r) + cc] -= L[tri(r) + cj] * lcj;
+                }
+                __syncwarp();
             }
         }
+        __syncthreads();
+        for (int t = 0; i1 + 32 * t < k; ++t) {
+            const int c = i1 + lane + 32 * t;
+            const bool valid = c < k;
+            double cp[KB];
+#pragma unroll
+            for (int e = 0; e < KB; ++e) cp[e] = valid && e < nb ? L[tri(c) + i0 + e] : 0.0;
+            for (int i = i1 + 32 * t + warp; i < k; i += nw) {
+                if (valid && c <= i) {
+                    const double *li = L + tri(i) + i0;
+                    double s0 = 0.0, s1 = 0.0;
+#pragma unroll
+                    for (int e = 0; e < KB; e += 2) {
+                        if (e < nb) s0 = fma(li[e], cp[e], s0);
+                        if (e + 1 < nb) s1 = fma(li[e + 1], cp[e + 1], s1);
+                    }
+                    L[tri(i) + c] -= s0 + s1;
+                }
+            }
+        }
+        __syncthreads();
+    }
+    for (int i = tid; i < k; i += nt) invd[i] = 1.0 / L[tri(i) + i];
+    __syncthreads();
+
+    // 3. L Y = Z (forward), then L^T W = Y (backward), 8 rows per step: warp 0 (lane = column)
+    // solves the step's 8 x 8 diagonal block in registers; then every warp (a row group, lane =
+    // column) subtracts the block's contribution from the remaining rows.
+    const int c = lane;
+    for (int i0 = 0; i0 < k; i0 += KB) {
+        const int i1 = min(i0 + KB, k);
+        if (warp == 0) {
+            double zb[KB];
+#pragma unroll
+            for (int e = 0; e < KB; ++e) zb[e] = i0 + e < i1 ? Z[(i0 + e) * NC + c] : 0.0;
+#pragma unroll
+            for (int i = 0; i < KB; ++i) {
+                if (i0 + i < i1) {
+                    const double *li = L + tri(i0 + i) + i0;
+                    double sum = zb[i];
+#pragma unroll
+                    for (int e = 0; e < i; ++e) sum -= li[e] * zb[e];
+                    zb[i] = sum * invd[i0 + i];
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < KB; ++e)
+                if (i0 + e < i1) Z[(i0 + e) * NC + c] = zb[e];
+        }
+        __syncthreads();
+        double y[KB];
+#pragma unroll
+        for (int e = 0; e < KB; ++e) y[e] = i0 + e < i1 ? Z[(i0 + e) * NC + c] : 0.0;
+        for (int j = i1 + warp; j < k; j += nw) {
+            const double *lj = L + tri(j) + i0;
+            double lv[KB];
+#pragma unroll
+            for (int e = 0; e < KB; ++e) lv[e] = i0 + e < i1 ? lj[e] : 0.0;
+            double s0 = Z[j * NC + c], s1 = 0.0;
+#pragma unroll
+            for (int e = 0; e < KB; e += 2) {
+                s0 -= lv[e] * y[e];
+                s1 -= lv[e + 1] * y[e + 1];
+            }
+            Z[j * NC + c] = s0 + s1;
+        }
+        __syncthreads();
+    }
+    for (int i1 = k; i1 > 0; i1 -= KB) {
+        const int i0 = max(i1 - KB, 0);
+        if (warp == 0) {
+            double xb[KB];
+#pragma unroll
+            for (int e = 0; e < KB; ++e) xb[e] = i0 + e < i1 ? Z[(i0 + e) * NC + c] : 0.0;
+#pragma unroll
+            for (int i = KB - 1; i >= 0; --i) {
+                if (i0 + i < i1) {
+                    double sum = xb[i];
+#pragma unroll
+                    for (int e = i + 1; e < KB; ++e)
+                        if (i0 + e < i1) sum -= L[tri(i0 + e) + i0 + i] * xb[e];
+                    xb[i] = sum * invd[i0 + i];
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < KB; ++e)
+                if (i0 + e < i1) Z[(i0 + e) * NC + c] = xb[e];
+        }
+        __syncthreads();
+        double x[KB];
+#pragma unroll
+        for (int e = 0; e < KB; ++e) x[e] = i0 + e < i1 ? Z[(i0 + e) * NC + c] : 0.0;
+        for (int j = warp; j < i0; j += nw) {
+            double lv[KB];
+#pragma unroll
+            for (int e = 0; e < KB; ++e) lv[e] = i0 + e < i1 ? L[tri(i0 + e) + j] : 0.0;
+            double s0 = Z[j * NC + c], s1 = 0.0;
+#pragma unroll
+            for (int e = 0; e < KB; e += 2) {
+                s0 -= lv[e] * x[e];
+                s1 -= lv[e + 1] * x[e + 1];
+            }
+            Z[j * NC + c] = s0 + s1;
+        }
+        __syncthreads();
+    }
+
+    // 4. this CTA's columns of W (n x d): the solution itself, or X^T Y on the smaller side
+    __nv_bfloat16 *wp = wparts + bh * 2 * d * d;
+    for (int p = tid; p < n * NC; p += nt) {
+        const int e = p / NC, cl = p % NC, cc = c0 + cl;
+        double w;
+        if (tall) {
+            w = Z[p];
+        } else {
+            w = 0.0;
+            for (int r = 0; r < m; ++r)
+                w = fma(e < d ? Mh[(long long)r * w2 + e] : 1.0, Z[r * NC + cl], w);
+        }
+        if (e < d) {
+            const __nv_bfloat16 h = __double2bfloat16(w);
+            wp[e * d + cc] = h;
+            wp[(d + e) * d + cc] = __double2bfloat16(w - (double)__bfloat162float(h));
+        } else {
+            woff[bh * d + cc] = (float)w;
+        }
     }
 }
 
+size_t probe_solve_smem(int m, int d) {
+    const int n = d + 1, k = m >= n ? n : m;
+    return ((size_t)k * (k + 1) / 2 + k + (size_t)k * kSolveCols) * sizeof(double);
+}
 
-cudaError_t sparsepr_apply(void *o, const float *W, long long BH, int N, int d, cudaStream_t st) {
-    const dim3 g((unsigned)((N + 63) / 64), (unsigned)BH);
-    auto *ob = reinterpret_cast<__nv_bfloat16 *>(o);
-    if (d == 128) {
-        const size_t smem = ((size_t)129 * 128 + 64 * 129) * 4;
-        cudaFuncSetAttribute(apply_correction_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        apply_correction_kernel<128><<<g, 256, smem, st>>>(ob, W, N);
-    } else {
-        const size_t smem = ((size_t)65 * 64 + 64 * 65) * 4;
-        apply_correction_kernel<64><<<g, 256, smem, st>>>(ob, W, N);
+cudaError_t sparsepr_solve(const double *M, double *C, double *sums, __nv_bfloat16 *wparts,
+                           float *woff, long long BH, int m, int d, cudaStream_t st) {
+    if (m >= d + 1) {
+        const int tiles = (d / 64) * (2 * d / 64);
+        probe_gram_kernel<<<dim3((unsigned)tiles + 1, (unsigned)BH), 256, 0, st>>>(M, C, sums, m, d);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
     }
-    return cudaGetLastError();
-}
-cudaError_t sparsepr_solve(const double *X, const double *R, double *G, double *Z, double *Wd,
-                           float *W, long long BH, int m, int d, cudaStream_t st) {
-    probe_solve_kernel<<<(unsigned)BH, 256, 0, st>>>(X, R, G, Z, Wd, W, m, d, 1e-12);
+    const size_t smem = probe_solve_smem(m, d);
+    cudaError_t e = cudaFuncSetAttribute(probe_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    probe_solve_kernel<<<dim3((unsigned)(d / kSolveCols), (unsigned)BH), kSolveThreads, smem, st>>>(
+        M, C, sums, wparts, woff, m, d, 1e-12);
     return cudaGetLastError();
 }
 
-// Probe-row tables for the varlen kernel: per head ceil(m/128) query tiles of cluster 0, one
-// key list covering [0, N) in 128-key tiles, identity output rows.
+// ------------------------------------------------------------------------------------------
+// O += [O, 1] W on the tensor cores, in place on the bf16 output
+// ------------------------------------------------------------------------------------------
+// Per 128-row tile of one head the product O W is a dense 128 x D x D contraction: A is the bf16
+// tile of O itself (exact), B is W's first D rows split into two bf16 parts (W ~ W_hi + W_lo,
+// relative error 2^-17), both accumulated in fp32 in tensor memory; the epilogue adds O and the
+// offset row (fp32) and rounds to bf16 once.  The kernel is bound by reading and writing O.
+//
+// Persistent CTAs (one per SM), each owning a contiguous run of the head-major tile sequence,
+// so W is loaded once per head change:
+//   warp 0 lane 0  TMA producer: W parts per head, O tiles into a 4-slot ring
+//   warp 1 lane 0  MMA issuer:   acc[i % 2] = O_i W_hi + O_i W_lo
+//   warp 2         tensor-memory allocator (2 accumulators of D columns)
+//   warps 4..7     epilogue: thread = tile row; result written over the O slot, then stored by
+//                  TMA (32 rows per warp), the slot released once the store has read it
+template <int D>
+struct ApplyCfg {
+    static constexpr int CHUNKS = D / 64;        // 64-column (128-byte) swizzle chunks
+    static constexpr int O_CHUNK = 128 * 128;    // 128 rows x 128 bytes
+    static constexpr int O_BYTES = CHUNKS * O_CHUNK;
+    static constexpr int W_CHUNK = D * 128;      // D rows x 128 bytes
+    static constexpr int W_PART = CHUNKS * W_CHUNK;
+    static constexpr int W_BYTES = 2 * W_PART;
+    static constexpr int NSLOT = 4, NACC = 2;
+    static constexpr int OFF_W = 0;
+    static constexpr int OFF_O = W_BYTES;
+    static constexpr int OFF_BAR = OFF_O + NSLOT * O_BYTES;
+    static constexpr int SMEM = OFF_BAR + 256 + 1024;  // barriers + slack for 1024-byte alignment
+    static constexpr uint32_t TMEM_COLS = NACC * D;
+};
+
+enum { A_WF, A_WE, A_OF0, A_OE0 = A_OF0 + 4, A_AF0 = A_OE0 + 4, A_AE0 = A_AF0 + 2, A_FIN = A_AE0 + 2,
+       A_COUNT };
+
+struct ApplyParams {
+    const float *woff;   // [BH, D] the offset row of W (fp32)
+    int N, tiles;        // rows per head, 128-row tiles per head
+    long long total;     // BH * tiles
+    unsigned long long wait_ns;
+};
+
+template <int D>
+__global__ void __launch_bounds__(256, 1)
+    apply_correction_tc_kernel(const __grid_constant__ CUtensorMap tmO,
+                               const __grid_constant__ CUtensorMap tmOst,
+                               const __grid_constant__ CUtensorMap tmW, const ApplyParams prm) {
+    using C = ApplyCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_BAR + 8 * A_COUNT);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_BAR + 8 * A_COUNT + 4);
+    static_assert(8 * A_COUNT + 8 <= 256, "barrier area overflow");
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t sW = smem_u32(smem + C::OFF_W), sO = smem_u32(smem + C::OFF_O);
+    auto bar = [&](int b) { return smem_u32(&bars[b]); };
+    // this CTA's run of the head-major tile sequence
+    const long long lo = prm.total * blockIdx.x / gridDim.x;
+    const long long hi = prm.total * (blockIdx.x + 1) / gridDim.x;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(A_WF), 1);
+        mbar_init(bar(A_WE), 1);
+        for (int s = 0; s < C::NSLOT; ++s) {
+            mbar_init(bar(A_OF0 + s), 1);
+            mbar_init(bar(A_OE0 + s), 4);
+        }
+        for (int a = 0; a < C::NACC; ++a) {
+            mbar_init(bar(A_AF0 + a), 1);
+            mbar_init(bar(A_AE0 + a), 4);
+        }
+        mbar_init(bar(A_FIN), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tmO);
+        prefetch_tmap(&tmOst);
+        prefetch_tmap(&tmW);
+    }
+    if (warp == 2) {
+        tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tacc = *tmem_holder;
+    const unsigned long long wns = prm.wait_ns;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- TMA producer
+        uint32_t nw = 0, no = 0;
+        long long cur = -1;
+        bool ok = true;
+        for (long long t = lo; t < hi && ok; ++t) {
+            const long long bh = t / prm.tiles;
+            const int tile = (int)(t - bh * prm.tiles);
+            if (bh != cur) {
+                // W of the previous head must be consumed by its last MMA
+                if (nw > 0 && !(ok = warp_wait(bar(A_WE), (nw - 1) & 1, wns, abort_flag, 0x51, (uint32_t)t)))
+                    break;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(bar(A_WF), C::W_BYTES);
+#pragma unroll
+                    for (int part = 0; part < 2; ++part)
+#pragma unroll
+                        for (int c = 0; c < C::CHUNKS; ++c)
+                            tma_load_3d(sW + part * C::W_PART + c * C::W_CHUNK, &tmW, bar(A_WF), c * 64,
+                                        part * D, (int)bh);
+                }
+                ++nw;
+                cur = bh;
+            }
+            const int slot = no % C::NSLOT;
+            if (no >= C::NSLOT &&
+                !(ok = warp_wait(bar(A_OE0 + slot), ((no / C::NSLOT) - 1) & 1, wns, abort_flag, 0x52, (uint32_t)t)))
+                break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bar(A_OF0 + slot), C::O_BYTES);
+#pragma unroll
+                for (int c = 0; c < C::CHUNKS; ++c)
+                    tma_load_3d(sO + slot * C::O_BYTES + c * C::O_CHUNK, &tmO, bar(A_OF0 + slot), c * 64,
+                                tile * 128, (int)bh);
+            }
+            ++no;
+        }
+        if (!ok && lane == 0) {  // let every copy that was started land before the CTA leaves
+            if (nw) drain_wait(bar(A_WF), (nw - 1) & 1, wns, 0x55);
+            for (uint32_t i = no > C::NSLOT ? no - C::NSLOT : 0; i < no; ++i)
+                drain_wait(bar(A_OF0 + i % C::NSLOT), (i / C::NSLOT) & 1, wns, 0x56);
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        constexpr uint32_t IDESC = idesc_bf16_f32(128, D, 0, 1);
+        const uint64_t dO = smem_desc_sw128(sO, 16, 1024);               // A: K-major tile of O
+        const uint64_t dW = smem_desc_sw128(sW, C::W_CHUNK, 1024);       // B: W rows, N innermost
+        uint32_t nw = 0, no = 0;
+        long long cur = -1;
+        bool ok = true;
+        for (long long t = lo; t < hi && ok; ++t) {
+            const long long bh = t / prm.tiles;
+            if (bh != cur) {
+                if (!(ok = warp_wait(bar(A_WF), nw & 1, wns, abort_flag, 0x61, (uint32_t)t))) break;
+                ++nw;
+                cur = bh;
+            }
+            const int slot = no % C::NSLOT, a = no % C::NACC;
+            if (!(ok = warp_wait(bar(A_OF0 + slot), (no / C::NSLOT) & 1, wns, abort_flag, 0x62, (uint32_t)t)))
+                break;
+            if (no >= C::NACC &&
+                !(ok = warp_wait(bar(A_AE0 + a), ((no / C::NACC) - 1) & 1, wns, abort_flag, 0x63, (uint32_t)t)))
+                break;
+            tc_fence_after();
+            const bool last_of_head = t + 1 >= hi || (t + 1) / prm.tiles != bh;
+            if (lane == 0) {
+                const uint64_t oslot = (uint64_t)((slot * C::O_BYTES) >> 4);
+#pragma unroll
+                for (int part = 0; part < 2; ++part)
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        // A step kk: 32 bytes inside the swizzled row, then the next chunk;
+                        // B step kk: 16 rows of 128 bytes
+                        const uint64_t oa = oslot + (uint64_t)(((kk >> 2) * C::O_CHUNK + (kk & 3) * 32) >> 4);
+                        const uint64_t ob = (uint64_t)((part * C::W_PART + kk * 2048) >> 4);
+                        mma_ss(tacc + a * D, dO + oa, dW + ob, IDESC, (part | kk) ? 1u : 0u);
+                    }
+                mma_commit(bar(A_AF0 + a));
+                if (last_of_head) mma_commit(bar(A_WE));
+            }
+            __syncwarp();
+            ++no;
+        }
+        // every MMA this warp issued must be complete before tensor memory is released
+        if (lane == 0) {
+            mma_commit(bar(A_FIN));
+            drain_wait(bar(A_FIN), 0, wns, 0x64);
+        }
+    } else if (warp >= 4) {
+        // ---------------------------------------------------------------- epilogue
+        const int q4 = warp & 3;
+        const int r = q4 * 32 + lane;  // tile row == TMEM lane
+        const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+        uint32_t no = 0;
+        bool ok = true;
+        int prev_slot = -1;
+        for (long long t = lo; t < hi && ok; ++t) {
+            const long long bh = t / prm.tiles;
+            const int tile = (int)(t - bh * prm.tiles);
+            const int slot = no % C::NSLOT, a = no % C::NACC;
+            if (!(ok = warp_wait(bar(A_AF0 + a), (no / C::NACC) & 1, wns, abort_flag, 0x71, (uint32_t)t)))
+                break;
+            // the O load into this slot has landed (its MMAs have completed); waiting on its
+            // barrier too makes the TMA writes visible to this warp's own reads of the slot
+            if (!(ok = warp_wait(bar(A_OF0 + slot), (no / C::NSLOT) & 1, wns, abort_flag, 0x72, (uint32_t)t)))
+                break;
+            tc_fence_after();
+            uint32_t acc[D];
+            tmem_ld_cols<D>(tacc + a * D + lane_off, acc);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(A_AE0 + a));
+            // the slot holds this tile's O (the load completed before the MMAs that read it)
+            uint8_t *rowp = smem + C::OFF_O + slot * C::O_BYTES + r * 128;
+            const float *off = prm.woff + bh * D;
+#pragma unroll
+            for (int u = 0; u < D / 8; ++u) {  // 16-byte units of 8 columns
+                const int c = u >> 3, pu = (u & 7) ^ (r & 7);
+                uint4 *p = reinterpret_cast<uint4 *>(rowp + c * C::O_CHUNK + pu * 16);
+                const uint4 ov = *p;
+                const float4 f0 = __ldg(reinterpret_cast<const float4 *>(off + u * 8));
+                const float4 f1 = __ldg(reinterpret_cast<const float4 *>(off + u * 8 + 4));
+                const float fo[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+                const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w};
+                uint32_t res[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float x0 = __uint_as_float(ow[e] << 16), x1 = __uint_as_float(ow[e] & 0xFFFF0000u);
+                    res[e] = pack_bf16(x0 + (__uint_as_float(acc[u * 8 + 2 * e]) + fo[2 * e]),
+                                       x1 + (__uint_as_float(acc[u * 8 + 2 * e + 1]) + fo[2 * e + 1]));
+                }
+                *p = make_uint4(res[0], res[1], res[2], res[3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                const int row0 = tile * 128 + q4 * 32;
+                if (row0 < prm.N) {
+#pragma unroll
+                    for (int c = 0; c < C::CHUNKS; ++c)
+                        tma_store_3d(&tmOst, sO + slot * C::O_BYTES + c * C::O_CHUNK + q4 * 4096, c * 64,
+                                     row0, (int)bh);
+                }
+                bulk_commit_group();
+                // the previous tile's store has read its slot: release it to the producer
+                bulk_wait_group_read<1>();
+                if (prev_slot >= 0) mbar_arrive(bar(A_OE0 + prev_slot));
+            }
+            __syncwarp();
+            prev_slot = slot;
+            ++no;
+        }
+        if (lane == 0) bulk_wait_group<0>();  // every store written before the CTA leaves
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 2) tmem_dealloc(tacc, C::TMEM_COLS);
+}
+
+template <int D>
+static cudaError_t launch_apply_t(const CUtensorMap &tmO, const CUtensorMap &tmOst,
+                                  const CUtensorMap &tmW, const ApplyParams &p, int num_sms,
+                                  cudaStream_t st) {
+    using C = ApplyCfg<D>;
+    cudaError_t e = cudaFuncSetAttribute(apply_correction_tc_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    long long grid = num_sms;
+    if (grid > p.total) grid = p.total;
+    if (grid <= 0) return cudaSuccess;
+    apply_correction_tc_kernel<D><<<(unsigned)grid, 256, C::SMEM, st>>>(tmO, tmOst, tmW, p);
+    return cudaGetLastError();
+}
+
+// tmO: O with 128-row boxes (loads), tmOst: O with 32-row boxes (stores), tmW: the W parts
+// [BH, 2 D, D] with D-row boxes.
+cudaError_t sparsepr_apply(const CUtensorMap &tmO, const CUtensorMap &tmOst, const CUtensorMap &tmW,
+                           const float *woff, long long BH, int N, int d, unsigned long long wait_ns,
+                           int num_sms, cudaStream_t st) {
+    ApplyParams p;
+    p.woff = woff;
+    p.N = N;
+    p.tiles = (N + 127) / 128;
+    p.total = BH * p.tiles;
+    p.wait_ns = wait_ns;
+    return d == 128 ? launch_apply_t<128>(tmO, tmOst, tmW, p, num_sms, st)
+                    : launch_apply_t<64>(tmO, tmOst, tmW, p, num_sms, st);
+}
+// Probe-row tables for the variable-length kernel with the keys split S ways: unit (s, u) is
+// query tile u (128 probe rows) of "cluster" s, whose key list is the s-th contiguous run of the
+// ceil(N / 128) key tiles (the last tile ragged); output rows are the identity.
 __global__ void __launch_bounds__(256) probe_tables_kernel(int2 *__restrict__ units,
                                                            int32_t *__restrict__ tiles,
                                                            int32_t *__restrict__ tcnt,
                                                            int32_t *__restrict__ perm,
                                                            long long BH, int N, int m, int U,
-                                                           int tstride) {
+                                                           int S, int tstride) {
     const long long bh = blockIdx.x;
-    for (int u = threadIdx.x; u < U; u += blockDim.x) {
-        const int r0 = u * 128;
-        units[bh * U + u] = r0 < m ? make_int2(r0, min(128, m - r0) << 16) : make_int2(0, 0);
+    for (int x = threadIdx.x; x < U * S; x += blockDim.x) {
+        const int sp = x / U, r0 = (x - sp * U) * 128;
+        units[bh * U * S + x] = r0 < m ? make_int2(r0, (min(128, m - r0) << 16) | sp) : make_int2(0, 0);
     }
     const int nt = (N + 127) / 128;
-    for (int t = threadIdx.x; t < tstride; t += blockDim.x)
-        if (t < nt) tiles[bh * tstride + t] = ((t * 128) << 7) | (min(128, N - t * 128) - 1);
-    if (threadIdx.x == 0) tcnt[bh] = nt;
+    for (int x = threadIdx.x; x < S * tstride; x += blockDim.x) {
+        const int sp = x / tstride, i = x - sp * tstride;
+        const int t = (int)((long long)sp * nt / S) + i;
+        if (t < (int)((long long)(sp + 1) * nt / S))
+            tiles[(bh * S + sp) * tstride + i] = ((t * 128) << 7) | (min(128, N - t * 128) - 1);
+    }
+    for (int sp = threadIdx.x; sp < S; sp += blockDim.x)
+        tcnt[bh * S + sp] = (int)((long long)(sp + 1) * nt / S - (long long)sp * nt / S);
     for (int i = threadIdx.x; i < m; i += blockDim.x) perm[bh * m + i] = i;
+}
+
+// Key splits of the probe attention: enough (query tile, key run) units to keep every SM of a
+// 148-SM device busy with two CTAs about twice over, at most one per key tile and 64 in all.
+int probe_splits(long long BH, int N, int m) {
+    const long long units = BH * ((m + 127) / 128);
+    long long s = (592 + units - 1) / units;
+    const int nt = (N + 127) / 128;
+    if (s > nt) s = nt;
+    if (s > 64) s = 64;
+    return s < 1 ? 1 : (int)s;
 }
 
 }  // namespace bsa
@@ -279,20 +717,22 @@ namespace {
 
 struct ProbeWorkspace {
     unsigned int *counter;
-    void *qpr, *e;
+    void *qpr;
+    float *po, *plse;
     int2 *units;
     int32_t *tiles, *tcnt, *perm;
-    double *X, *R, *G, *Z, *Wd;
-    float *W;
-    int U, tstride, k;
+    double *M, *C, *sums;
+    __nv_bfloat16 *wparts;
+    float *woff;
+    int U, S, tstride;
 };
 
 size_t probe_workspace(int B, int H, int N, int d, int m, void *base, ProbeWorkspace *w) {
     const size_t BH = (size_t)B * H;
     ProbeWorkspace t;
     t.U = (m + 127) / 128;
-    t.tstride = (N + 127) / 128;
-    t.k = m < d + 1 ? m : d + 1;
+    t.S = bsa::probe_splits(BH, N, m);
+    t.tstride = ((N + 127) / 128 + t.S - 1) / t.S;
     size_t off = 0;
     uint8_t *p = reinterpret_cast<uint8_t *>(base);
     auto take = [&](size_t bytes) -> void * {
@@ -302,17 +742,17 @@ size_t probe_workspace(int B, int H, int N, int d, int m, void *base, ProbeWorks
     };
     t.counter = (unsigned int *)take(256);
     t.qpr = take(BH * m * d * 2);
-    t.e = take(BH * m * d * 2);
-    t.units = (int2 *)take(BH * t.U * 8);
-    t.tiles = (int32_t *)take(BH * t.tstride * 4);
-    t.tcnt = (int32_t *)take(BH * 4);
+    t.po = (float *)take((size_t)t.S * BH * m * d * 4);
+    t.plse = (float *)take((size_t)t.S * BH * m * 4);
+    t.units = (int2 *)take(BH * t.U * t.S * 8);
+    t.tiles = (int32_t *)take(BH * t.S * t.tstride * 4);
+    t.tcnt = (int32_t *)take(BH * t.S * 4);
     t.perm = (int32_t *)take(BH * m * 4);
-    t.X = (double *)take(BH * m * (d + 1) * 8);
-    t.R = (double *)take(BH * m * d * 8);
-    t.G = (double *)take(BH * (size_t)t.k * t.k * 8);
-    t.Z = (double *)take(BH * (size_t)t.k * d * 8);
-    t.Wd = (double *)take(BH * (size_t)(d + 1) * d * 8);
-    t.W = (float *)take(BH * (size_t)(d + 1) * d * 4);
+    t.M = (double *)take(BH * m * 2 * d * 8);
+    t.C = (double *)take(m >= d + 1 ? BH * (size_t)d * 2 * d * 8 : 0);
+    t.sums = (double *)take(BH * 2 * d * 8);
+    t.wparts = (__nv_bfloat16 *)take(BH * (size_t)2 * d * d * 2);
+    t.woff = (float *)take(BH * (size_t)d * 4);
     if (w) *w = t;
     return off;
 }
@@ -356,23 +796,26 @@ extern "C" sa_status sa_sparsepr_attn_fwd(const void *q, const void *k, const vo
     bsa::gather_probe_rows_kernel<<<(unsigned)((BH * m * vec + 255) / 256 < sms * 16 ? (BH * m * vec + 255) / 256 : sms * 16), 256, 0, st>>>(
         reinterpret_cast<const uint4 *>(q), probes, reinterpret_cast<uint4 *>(w.qpr), BH, N, m, vec);
     bsa::probe_tables_kernel<<<(unsigned)BH, 256, 0, st>>>(w.units, w.tiles, w.tcnt, w.perm, BH, N, m,
-                                                           w.U, w.tstride);
+                                                           w.U, w.S, w.tstride);
     if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
     CUtensorMap tq, tk, tv;
     if (!make_tmap(&tq, w.qpr, BH, m, d, 128) || !make_tmap(&tk, k, BH, N, d, 128) ||
         !make_tmap(&tv, v, BH, N, d, 128))
         return SA_ERR_CUDA;
-    cudaError_t e = bsa::attn_varlen_fwd(tq, tk, tv, w.units, w.U, w.tiles, w.tcnt, w.tstride, w.perm,
-                                         w.e, BH, N, m, 1, d, resolve_scale(scale, d), g_wait_ns,
-                                         sms, w.counter, st);
+    cudaError_t e = bsa::attn_varlen_fwd(tq, tk, tv, w.units, w.U * w.S, w.tiles, w.tcnt, w.tstride,
+                                         w.perm, nullptr, BH, N, m, w.S, d, resolve_scale(scale, d),
+                                         g_wait_ns, sms, w.counter, st, w.po, w.plse);
     if (e != cudaSuccess) return SA_ERR_CUDA;
     // 3. residuals, the per-head least-squares map, the correction of every row
-    const long long nres = BH * m * (d + 1);
-    bsa::probe_residual_kernel<<<(unsigned)((nres + 255) / 256 < sms * 16 ? (nres + 255) / 256 : sms * 16), 256, 0, st>>>(
-        reinterpret_cast<const __nv_bfloat16 *>(o), reinterpret_cast<const __nv_bfloat16 *>(w.e),
-        probes, w.X, w.R, BH, N, m, d);
+    const long long nres = BH * m * d;
+    bsa::probe_merge_kernel<<<(unsigned)((nres + 255) / 256 < sms * 8 ? (nres + 255) / 256 : sms * 8), 256, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16 *>(o), w.po, w.plse, probes, w.M, BH, N, m, d, w.S);
     if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
-    e = bsa::sparsepr_solve(w.X, w.R, w.G, w.Z, w.Wd, w.W, BH, m, d, st);
-    if (e == cudaSuccess) e = bsa::sparsepr_apply(o, w.W, BH, N, d, st);
-    return from_cuda(e);
+    e = bsa::sparsepr_solve(w.M, w.C, w.sums, w.wparts, w.woff, BH, m, d, st);
+    if (e != cudaSuccess) return SA_ERR_CUDA;
+    CUtensorMap to, tost, tw;
+    if (!make_tmap(&to, o, BH, N, d, 128) || !make_tmap(&tost, o, BH, N, d, 32) ||
+        !make_tmap(&tw, w.wparts, BH, 2 * d, d, d))
+        return SA_ERR_CUDA;
+    return from_cuda(bsa::sparsepr_apply(to, tost, tw, w.woff, BH, N, d, g_wait_ns, sms, st));
 }

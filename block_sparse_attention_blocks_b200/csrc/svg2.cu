@@ -26,82 +26,6 @@ constexpr int kMaxClusters = 1024;   // Cq, Ck: one selection row per warp, sort
 constexpr int kMaxVarlenN = 1 << 24; // key tile entries pack (first row << 7) into 31 bits
 
 // ------------------------------------------------------------------------------------------
-// k-means assignment: thread per token, its row in registers; centroids staged 32 at a time in
-// shared memory with their squared norms; |x - c|^2 - |x|^2 = |c|^2 - 2 x . c in fp32.
-// ------------------------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(256) kmeans_assign_kernel(const __nv_bfloat16 *__restrict__ x,
-                                                            const float *__restrict__ cent,
-                                                            int32_t *__restrict__ assign, int N,
-                                                            int C) {
-    constexpr int CH = 32;
-    __shared__ __align__(16) float cs[CH * D];
-    __shared__ float cn[CH];
-    const int bh = blockIdx.y;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n = blockIdx.x * 256 + threadIdx.x;
-    const bool ok = n < N;
-    float xr[D];
-    {
-        const uint4 *src = reinterpret_cast<const uint4 *>(x + ((size_t)bh * N + (ok ? n : 0)) * D);
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-            const uint4 w = src[c];
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                xr[8 * c + 2 * h] = __uint_as_float(ws[h] << 16);
-                xr[8 * c + 2 * h + 1] = __uint_as_float(ws[h] & 0xFFFF0000u);
-            }
-        }
-    }
-    const float *cb = cent + (size_t)bh * C * D;
-    float best = INFINITY;
-    int arg = 0;
-    for (int c0 = 0; c0 < C; c0 += CH) {
-        __syncthreads();  // every thread is done with the previous chunk
-        for (int i = threadIdx.x; i < CH * D / 4; i += 256) {
-            const int cc = i / (D / 4);
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (c0 + cc < C) v = reinterpret_cast<const float4 *>(cb + (size_t)(c0 + cc) * D)[i % (D / 4)];
-            reinterpret_cast<float4 *>(cs)[i] = v;
-        }
-        __syncthreads();
-        for (int cc = warp; cc < CH; cc += 8) {
-            float s = 0.f;
-            for (int e = lane; e < D; e += 32) s = fmaf(cs[cc * D + e], cs[cc * D + e], s);
-            s = warp_sum(s);
-            if (lane == 0) cn[cc] = c0 + cc < C ? s : INFINITY;  // padding is never nearest
-        }
-        __syncthreads();
-        const int m = min(CH, C - c0);
-        for (int cc = 0; cc < m; cc += 4) {
-            float a[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int e = 0; e < D; e += 4) {
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float4 c4 = *reinterpret_cast<const float4 *>(&cs[(cc + j) * D + e]);
-                    a[j] = fmaf(xr[e], c4.x, a[j]);
-                    a[j] = fmaf(xr[e + 1], c4.y, a[j]);
-                    a[j] = fmaf(xr[e + 2], c4.z, a[j]);
-                    a[j] = fmaf(xr[e + 3], c4.w, a[j]);
-                }
-            }
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float dist = fmaf(-2.f, a[j], cn[cc + j]);
-                if (dist < best) {  // strict: the lower index keeps a tie
-                    best = dist;
-                    arg = c0 + cc + j;
-                }
-            }
-        }
-    }
-    if (ok) assign[(size_t)bh * N + n] = arg;
-}
-
-// ------------------------------------------------------------------------------------------
 // Stable counting sort of one head's assignment (one CTA of 8 warps per head).  Warp w owns a
 // contiguous eighth of the tokens: it counts its tokens per cluster, the counts are scanned in
 // (cluster, warp) order, and each warp then places its tokens in token order (lanes of a 32-token
@@ -403,6 +327,21 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4 *__restric
 
 namespace bsa {
 
+// ------------------------------------------------------------------------------------------
+// nearest centroid on the tensor cores
+// ------------------------------------------------------------------------------------------
+// For a 128-token tile of one head, the nearest centroid is argmin_c |c|^2 - 2 x.c (|x|^2 is
+// common to every c).  The dot products x.c are a 128 x C x d contraction: x is bf16 already
+// (exact), each fp32 centroid is split exactly into three bf16 parts c = h + m + l
+// (centroid_split_kernel), and the three products x.h + x.m + x.l accumulate in one fp32
+// tensor-memory tile, so the result is an fp32 dot product up to accumulation rounding.  CTA =
+// one token tile, centroids in 128-wide tiles:
+//   warp 0 lane 0  TMA producer: the token tile once, then the three parts of each centroid
+//                  tile into a 2-stage ring
+//   warp 1 lane 0  MMA issuer: 3 x d/16 MMAs per centroid tile into one of two accumulators
+//   warp 2         tensor-memory allocator (2 x 128 columns)
+//   warps 4..7     epilogue: thread = token; scans its accumulator row for |c|^2 - 2 x.c,
+//                  keeping the first minimum (the lower index on a tie, as Lloyd's step is read)
 template <int D>
 struct KmTcCfg {
     static constexpr int CHUNKS = D / 64;
@@ -647,32 +586,25 @@ static unsigned grid_for(long long work, int per_block, int num_sms) {
 
 // parts: [BH, 3, C, d] bf16 scratch and norms [BH, C] fp32 scratch for the tensor-core
 // assignment; tx / tp: tensor maps of x ({d, N, BH}, 128-row boxes) and of parts
-// ({d, C, 3 BH}, 128-row boxes).  With parts == nullptr the SIMT assignment runs.
+// ({d, C, 3 BH}, 128-row boxes).
 cudaError_t kmeans_lloyd(const void *x, float *cent, int32_t *assign, int32_t *perm,
                          int32_t *cstart, int32_t *csize, long long BH, int N, int d, int C,
                          int iters, void *parts, float *norms, const CUtensorMap *tx,
                          const CUtensorMap *tp, unsigned long long wait_ns, cudaStream_t st) {
-    const dim3 ga((unsigned)((N + 255) / 256), (unsigned)BH);
     const dim3 gu((unsigned)C, (unsigned)BH);
     const size_t sort_smem = (size_t)9 * C * sizeof(int32_t);
     const auto *xb = reinterpret_cast<const __nv_bfloat16 *>(x);
     for (int it = 0;; ++it) {
-        if (parts) {
-            cudaError_t e = centroid_split(cent, parts, norms, BH, C, d, st);
-            if (e == cudaSuccess) e = kmeans_assign_tc(*tx, *tp, norms, assign, BH, N, d, C, wait_ns, st);
-            if (e != cudaSuccess) return e;
-        } else if (d == 128) {
-            kmeans_assign_kernel<128><<<ga, 256, 0, st>>>(xb, cent, assign, N, C);
-        } else {
-            kmeans_assign_kernel<64><<<ga, 256, 0, st>>>(xb, cent, assign, N, C);
-        }
+        cudaError_t e = centroid_split(cent, parts, norms, BH, C, d, st);
+        if (e == cudaSuccess) e = kmeans_assign_tc(*tx, *tp, norms, assign, BH, N, d, C, wait_ns, st);
+        if (e != cudaSuccess) return e;
         cluster_sort_kernel<<<(unsigned)BH, 256, sort_smem, st>>>(assign, N, C, perm, cstart, csize);
         if (it == iters) break;
         if (d == 128)
             kmeans_update_kernel<128><<<gu, 512, 0, st>>>(xb, perm, cstart, csize, cent, N, C);
         else
             kmeans_update_kernel<64><<<gu, 512, 0, st>>>(xb, perm, cstart, csize, cent, N, C);
-        const cudaError_t e = cudaGetLastError();
+        e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();

@@ -230,7 +230,11 @@ sa_status sa_select_from_logits(const float *logits, int B, int H, int nb, int t
                                 uint8_t *mask, int32_t *kv_idx, int32_t *kv_cnt, void *stream);
 
 /*
- * Block-sparse attention forward (online softmax over the kept key blocks only).
+ * Block-sparse attention forward (online softmax over the kept key blocks only): the attention
+ * that the hybrid mask of the SpargeAttention2 page (section "ハイブリッドマスキングと蒸留微調整")
+ * restricts to the kept blocks, computed as the Sparse VideoGen2 page's kernel description
+ * (section 2.C) puts it: sparse loads of the kept key/value blocks, dense compute on a
+ * contiguous query tile.
  *   O[b,h,t,:] = sum over kept blocks j of query block i = t / bs, keys s in block j with s < N,
  *                of softmax_s(scale * Q[t] . K[s]) V[s]; zero when the block keeps nothing.
  * q, k, v : [B, H, N, d] bf16.       o : [B, H, N, d] bf16, written.
@@ -248,7 +252,9 @@ sa_status sa_block_sparse_attn_fwd(const void *q, const void *k, const void *v,
                                    size_t workspace_bytes, void *stream);
 
 /*
- * Dense attention forward, the 0 %-sparsity control: O = softmax(scale Q K^T) V over all N keys.
+ * Dense attention forward, the 0 %-sparsity control: O = softmax(scale Q K^T) V over all N keys
+ * (the full attention that the SpargeAttention2 page's speed-ups and quality comparisons are
+ * measured against, section "実験結果：速度と品質の両立").
  * Same layouts, workspace and arithmetic as sa_block_sparse_attn_fwd (internally bs = 128).
  */
 sa_status sa_dense_attn_fwd(const void *q, const void *k, const void *v, void *o, int B, int H,
