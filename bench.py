@@ -56,6 +56,7 @@ def load_peaks():
 
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fwd_kernel_wan14b_720p_traffic.txt")
 KERNEL_SOURCES = ("block_sparse_attention_blocks_b200/csrc/attn.cu",
+                  "block_sparse_attention_blocks_b200/csrc/softmax.cuh",
                   "block_sparse_attention_blocks_b200/csrc/ptx.cuh")
 
 

@@ -22,6 +22,7 @@
 // differs is where tiles start: a TMA row coordinate may be any row, so tiles start inside
 // clusters rather than on block boundaries.
 #include "bsa_internal.h"
+#include "softmax.cuh"
 
 namespace bsa {
 

@@ -55,15 +55,19 @@ cudaError_t attn_varlen_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const 
                             unsigned long long wait_ns, int num_sms, unsigned int *workspace,
                             cudaStream_t st, float *part_o = nullptr, float *part_lse = nullptr);
 
-// parts [BH, 3, C, d] bf16 and norms [BH, C] fp32 are scratch for the tensor-core assignment;
-// tx / tp are tensor maps of x ({d, N, BH}) and parts ({d, C, 3 BH}), 128-row boxes.
+// parts [BH, 3, C, d] bf16, norms [BH, C] fp32 and, when C > 128, partial
+// [ceil(C / 128), BH, N] uint64 are scratch for the tensor-core assignment, hist the cluster
+// sort's chunk counts (cluster_sort_scratch_bytes); tx / tp are tensor maps of x ({d, N, BH})
+// and parts ({d, C, 3 BH}), 128-row boxes.
 cudaError_t kmeans_lloyd(const void *x, float *cent, int32_t *assign, int32_t *perm,
                          int32_t *cstart, int32_t *csize, long long BH, int N, int d, int C,
-                         int iters, void *parts, float *norms, const CUtensorMap *tx,
-                         const CUtensorMap *tp, unsigned long long wait_ns, cudaStream_t st);
+                         int iters, void *parts, float *norms, uint64_t *partial, int32_t *hist,
+                         const CUtensorMap *tx, const CUtensorMap *tp, unsigned long long wait_ns,
+                         cudaStream_t st);
 
 cudaError_t cluster_sort(const int32_t *assign, long long BH, int N, int C, int32_t *perm,
-                         int32_t *cstart, int32_t *csize, cudaStream_t st);
+                         int32_t *cstart, int32_t *csize, int32_t *hist, cudaStream_t st);
+size_t cluster_sort_scratch_bytes(long long BH, int N, int C);
 
 cudaError_t centroid_logits(const float *cq, const float *ck, const int32_t *size_k,
                             float *logits, long long BH, int Cq, int Ck, int d, float scale,

@@ -101,6 +101,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
     }
 }
 
+// Waits used while unwinding after an abort: they ignore the abort flag but stay bounded.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, unsigned long long ns,
+                                           uint32_t tag) {
+    int never = 0;
+    mbar_wait(bar, parity, ns, (volatile int *)&never, tag, 0);
+}
+
 // Warp-uniform bounded wait.  Every lane polls the barrier (so every lane is ordered after the
 // phase completion it consumes) and a warp vote decides when to leave, so the warp stays
 // converged for the .sync.aligned tcgen05 instructions and the final CTA barrier that follow.

@@ -26,71 +26,113 @@ constexpr int kMaxClusters = 1024;   // Cq, Ck: one selection row per warp, sort
 constexpr int kMaxVarlenN = 1 << 24; // key tile entries pack (first row << 7) into 31 bits
 
 // ------------------------------------------------------------------------------------------
-// Stable counting sort of one head's assignment (one CTA of 8 warps per head).  Warp w owns a
-// contiguous eighth of the tokens: it counts its tokens per cluster, the counts are scanned in
-// (cluster, warp) order, and each warp then places its tokens in token order (lanes of a 32-token
-// step that share a cluster are ranked with match.any).  Cluster c occupies
-// perm[cstart[c] .. cstart[c] + csize[c]) with its tokens ascending.
+// Stable counting sort of each head's assignment, in three launches over chunks of
+// kSortChunk tokens: per-chunk cluster counts; per head, the cluster ranges and each chunk's
+// first position in every cluster (counts scanned in (cluster, chunk) order); then each chunk
+// places its tokens in token order (one CTA per chunk, 8 warps each owning a contiguous eighth,
+// their counts scanned in warp order; lanes of a 32-token step that share a cluster are ranked
+// with match.any).  Cluster c occupies perm[cstart[c] .. cstart[c] + csize[c]) with its tokens
+// ascending.
 // ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) cluster_sort_kernel(const int32_t *__restrict__ assign,
-                                                           int N, int C, int32_t *__restrict__ perm,
-                                                           int32_t *__restrict__ cstart,
-                                                           int32_t *__restrict__ csize) {
-    extern __shared__ int32_t sm_sort[];
-    int32_t *cnt = sm_sort;           // [8][C]: count, then the warp's next free position
-    int32_t *start = sm_sort + 8 * C; // [C]
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long bh = blockIdx.x;
-    const int32_t *as = assign + bh * N;
-    for (int i = threadIdx.x; i < 8 * C; i += 256) cnt[i] = 0;
+constexpr int kSortChunk = 4096;
+
+// hist[bh, chunk, c] = the chunk's tokens assigned to c (out-of-range clusters are clamped and
+// flagged)
+__global__ void __launch_bounds__(256) cluster_hist_kernel(const int32_t *__restrict__ assign,
+                                                           int N, int C, int nchunk,
+                                                           int32_t *__restrict__ hist) {
+    extern __shared__ int32_t sm_hist[];
+    const long long bh = blockIdx.y;
+    const int ch = blockIdx.x;
+    for (int c = threadIdx.x; c < C; c += 256) sm_hist[c] = 0;
     __syncthreads();
-    const int per = (N + 7) / 8;
-    const int lo = min(N, warp * per), hi = min(N, lo + per);
+    const int lo = ch * kSortChunk, hi = min(N, lo + kSortChunk);
     bool bad = false;
-    for (int s = lo; s < hi; s += 32) {
-        const int n = s + lane;
-        if (n < hi) {
-            int a = as[n];
-            if (a < 0 || a >= C) {
-                bad = true;
-                a = a < 0 ? 0 : C - 1;
-            }
-            atomicAdd(&cnt[warp * C + a], 1);
+    for (int n = lo + threadIdx.x; n < hi; n += 256) {
+        int a = assign[bh * N + n];
+        if (a < 0 || a >= C) {
+            bad = true;
+            a = a < 0 ? 0 : C - 1;
         }
+        atomicAdd(&sm_hist[a], 1);
     }
     if (bad) atomicOr(&g_bsa_device_error, BSA_DEVERR_BOUNDS);
     __syncthreads();
-    for (int c = threadIdx.x; c < C; c += 256) {
-        int t = 0;
-        for (int w = 0; w < 8; ++w) t += cnt[w * C + c];
-        start[c] = t;
-    }
-    __syncthreads();
-    if (warp == 0) {  // exclusive scan of the cluster sizes
-        int run = 0;
-        for (int c0 = 0; c0 < C; c0 += 32) {
-            const int c = c0 + lane;
-            const int v = c < C ? start[c] : 0;
-            int incl = v;
+    for (int c = threadIdx.x; c < C; c += 256) hist[(bh * nchunk + ch) * C + c] = sm_hist[c];
+}
+
+// Per head: cstart / csize, and hist rewritten in place to each chunk's first position in
+// every cluster.  One CTA per head, thread per cluster (C <= 1024).
+__global__ void __launch_bounds__(1024) cluster_scan_kernel(int32_t *__restrict__ hist, int nchunk,
+                                                            int C, int32_t *__restrict__ cstart,
+                                                            int32_t *__restrict__ csize) {
+    __shared__ int32_t s_warp[32];
+    const long long bh = blockIdx.x;
+    const int c = threadIdx.x, warp = c >> 5, lane = c & 31;
+    int32_t *h = hist + bh * nchunk * C;
+    int total = 0;
+    if (c < C)
+        for (int ch = 0; ch < nchunk; ++ch) total += h[ch * C + c];
+    // exclusive scan of the totals over c (warp scans, then the warp sums)
+    int incl = total;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
-            }
-            if (c < C) start[c] = run + incl - v;
-            run += __shfl_sync(0xffffffffu, incl, 31);
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int v = lane < (int)(blockDim.x >> 5) ? s_warp[lane] : 0;
+        int wi = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += y;
         }
+        s_warp[lane] = wi - v;
     }
     __syncthreads();
-    for (int c = threadIdx.x; c < C; c += 256) {
-        int run = start[c];
+    if (c < C) {
+        int run = s_warp[warp] + incl - total;
         cstart[bh * C + c] = run;
-        for (int w = 0; w < 8; ++w) {
-            const int t = cnt[w * C + c];
-            cnt[w * C + c] = run;
+        csize[bh * C + c] = total;
+        for (int ch = 0; ch < nchunk; ++ch) {
+            const int t = h[ch * C + c];
+            h[ch * C + c] = run;
             run += t;
         }
-        csize[bh * C + c] = run - start[c];
+    }
+}
+
+// One CTA per (chunk, head): the chunk's tokens into perm at their stable positions.
+__global__ void __launch_bounds__(256) cluster_place_kernel(const int32_t *__restrict__ assign,
+                                                            const int32_t *__restrict__ base,
+                                                            int N, int C, int nchunk,
+                                                            int32_t *__restrict__ perm) {
+    extern __shared__ int32_t sm_place[];  // [8][C]: count, then the warp's next free position
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long bh = blockIdx.y;
+    const int ch = blockIdx.x;
+    const int32_t *as = assign + bh * N;
+    for (int i = threadIdx.x; i < 8 * C; i += 256) sm_place[i] = 0;
+    __syncthreads();
+    const int c0 = ch * kSortChunk, c1 = min(N, c0 + kSortChunk);
+    const int per = (c1 - c0 + 7) / 8;
+    const int lo = min(c1, c0 + warp * per), hi = min(c1, lo + per);
+    for (int s = lo; s < hi; s += 32) {
+        const int n = s + lane;
+        if (n < hi) atomicAdd(&sm_place[warp * C + min(max(as[n], 0), C - 1)], 1);
+    }
+    __syncthreads();
+    const int32_t *bs = base + (bh * nchunk + ch) * C;
+    for (int c = threadIdx.x; c < C; c += 256) {
+        int run = bs[c];
+        for (int w = 0; w < 8; ++w) {
+            const int t = sm_place[w * C + c];
+            sm_place[w * C + c] = run;
+            run += t;
+        }
     }
     __syncthreads();
     const uint32_t lt = (1u << lane) - 1u;
@@ -101,17 +143,18 @@ __global__ void __launch_bounds__(256) cluster_sort_kernel(const int32_t *__rest
         if (v) a = min(max(as[n], 0), C - 1);
         const uint32_t peers = __match_any_sync(0xffffffffu, a);
         const int rank = __popc(peers & lt);
-        if (v) perm[bh * N + cnt[warp * C + a] + rank] = n;
+        if (v) perm[bh * N + sm_place[warp * C + a] + rank] = n;
         __syncwarp();
-        if (v && rank == 0) cnt[warp * C + a] += __popc(peers);
+        if (v && rank == 0) sm_place[warp * C + a] += __popc(peers);
         __syncwarp();
     }
 }
 
 // ------------------------------------------------------------------------------------------
-// k-means update: one CTA per (cluster, head).  Column pairs x token lanes; each lane sums its
-// tokens in permuted (= token) order, the lanes are added in lane order, so the result does not
-// depend on scheduling.  A cluster without tokens keeps its centroid.
+// k-means update: one CTA per (cluster, head).  Thread = (16-byte column group, token lane);
+// each lane sums its tokens in permuted (= token) order with several rows in flight, the lanes
+// are added in lane order, so the result does not depend on scheduling.  A cluster without
+// tokens keeps its centroid.
 // ------------------------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(512) kmeans_update_kernel(const __nv_bfloat16 *__restrict__ x,
@@ -119,35 +162,46 @@ __global__ void __launch_bounds__(512) kmeans_update_kernel(const __nv_bfloat16 
                                                             const int32_t *__restrict__ cstart,
                                                             const int32_t *__restrict__ csize,
                                                             float *__restrict__ cent, int N, int C) {
-    constexpr int P = D / 2;    // bf16 pairs per row
-    constexpr int G = 512 / P;  // token lanes
-    __shared__ float2 part[G][P];
+    constexpr int V = D / 8;     // 16-byte groups (8 channels) per row
+    constexpr int G = 512 / V;   // token lanes
+    constexpr int U = 4;         // rows in flight per lane
+    __shared__ float part[G][D + 1];
     const int c = blockIdx.x;
     const long long bh = blockIdx.y;
-    const int pr = threadIdx.x % P, g = threadIdx.x / P;
+    const int vg = threadIdx.x % V, g = threadIdx.x / V;
     const int sz = csize[bh * C + c];
     if (sz <= 0) return;  // the whole CTA leaves together
     const int32_t *pm = perm + bh * N + cstart[bh * C + c];
-    const uint32_t *xb = reinterpret_cast<const uint32_t *>(x) + (size_t)bh * N * P;
-    float sx = 0.f, sy = 0.f;
-#pragma unroll 4
-    for (int s = g; s < sz; s += G) {
-        const int n = min(max(pm[s], 0), N - 1);
-        const uint32_t w = xb[(size_t)n * P + pr];
-        sx += __uint_as_float(w << 16);
-        sy += __uint_as_float(w & 0xFFFF0000u);
-    }
-    part[g][pr] = make_float2(sx, sy);
-    __syncthreads();
-    if (g == 0) {
-        float tx = 0.f, ty = 0.f;
-        for (int i = 0; i < G; ++i) {
-            tx += part[i][pr].x;
-            ty += part[i][pr].y;
+    const uint4 *xb = reinterpret_cast<const uint4 *>(x) + (size_t)bh * N * V;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int s0 = g; s0 < sz; s0 += G * U) {
+        int n[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int s = s0 + u * G;
+            n[u] = s < sz ? min(max(pm[s], 0), N - 1) : -1;
         }
-        float *dst = cent + (bh * C + c) * D + 2 * pr;
-        dst[0] = tx / (float)sz;
-        dst[1] = ty / (float)sz;
+        uint4 w[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) w[u] = n[u] >= 0 ? xb[(size_t)n[u] * V + vg] : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int u = 0; u < U; ++u) {  // in token order within the lane
+            if (n[u] < 0) break;
+            const uint32_t ws[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                acc[2 * h] += __uint_as_float(ws[h] << 16);
+                acc[2 * h + 1] += __uint_as_float(ws[h] & 0xFFFF0000u);
+            }
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) part[g][vg * 8 + e] = acc[e];
+    __syncthreads();
+    for (int j = threadIdx.x; j < D; j += 512) {
+        float t = 0.f;
+        for (int i = 0; i < G; ++i) t += part[i][j];
+        cent[(bh * C + c) * D + j] = t / (float)sz;
     }
 }
 
@@ -334,32 +388,55 @@ namespace bsa {
 // common to every c).  The dot products x.c are a 128 x C x d contraction: x is bf16 already
 // (exact), each fp32 centroid is split exactly into three bf16 parts c = h + m + l
 // (centroid_split_kernel), and the three products x.h + x.m + x.l accumulate in one fp32
-// tensor-memory tile, so the result is an fp32 dot product up to accumulation rounding.  CTA =
-// one token tile, centroids in 128-wide tiles:
-//   warp 0 lane 0  TMA producer: the token tile once, then the three parts of each centroid
-//                  tile into a 2-stage ring
-//   warp 1 lane 0  MMA issuer: 3 x d/16 MMAs per centroid tile into one of two accumulators
+// tensor-memory tile, so the result is an fp32 dot product up to accumulation rounding.
+//
+// Work items are (head, 128-centroid tile, 128-token tile), ordered by (head, centroid tile)
+// and then token tile; persistent CTAs (one per SM) own contiguous runs of that order, so a
+// CTA keeps one centroid tile's three parts resident in shared memory while the token tiles
+// stream past it:
+//   warp 0 lane 0  TMA producer: the parts on every change of (head, centroid tile), token
+//                  tiles into a 3-stage ring
+//   warp 1 lane 0  MMA issuer: 3 x d/16 MMAs per item into one of two accumulators
 //   warp 2         tensor-memory allocator (2 x 128 columns)
-//   warps 4..7     epilogue: thread = token; scans its accumulator row for |c|^2 - 2 x.c,
-//                  keeping the first minimum (the lower index on a tie, as Lloyd's step is read)
+//   warps 4..7     epilogue: thread = token; the first minimum of |c|^2 - 2 x.c over the
+//                  tile's centroids (the lower index on a tie, as Lloyd's step is read).  With
+//                  one centroid tile this is the assignment; with several, each tile's
+//                  (distance, index) goes out packed as an order-preserving 64-bit key and
+//                  kmeans_merge_kernel keeps the least, which is again the first minimum.
 template <int D>
 struct KmTcCfg {
     static constexpr int CHUNKS = D / 64;
     static constexpr int TILE = CHUNKS * 16384;  // 128 rows x D bf16, 128-byte swizzled chunks
-    static constexpr int OFF_X = 0;
-    static constexpr int OFF_P = TILE;                 // stage s, part p: OFF_P + (s*3 + p)*TILE
-    static constexpr int OFF_BAR = OFF_P + 6 * TILE;
+    static constexpr int NX = 3;                 // token-tile stages
+    static constexpr int OFF_P = 0;              // part p of the resident centroid tile
+    static constexpr int OFF_X = 3 * TILE;       // stage s of the token-tile ring
+    static constexpr int OFF_BAR = OFF_X + NX * TILE;
     static constexpr int SMEM = OFF_BAR + 128 + 1024;  // + alignment slack
 };
 
-enum { KB_XF, KB_PF0, KB_PF1, KB_PE0, KB_PE1, KB_SF0, KB_SF1, KB_SE0, KB_SE1, KB_FIN, KB_COUNT };
+enum { KB_PF, KB_PE, KB_XF0, KB_XE0 = KB_XF0 + 3, KB_AF0 = KB_XE0 + 3, KB_AE0 = KB_AF0 + 2,
+       KB_FIN = KB_AE0 + 2, KB_COUNT };
+
+struct KmParams {
+    const float *norms;     // [BH, C] |c|^2
+    int32_t *assign;        // [BH, N], written when T == 1
+    uint64_t *partial;      // [T, BH, N] packed (distance key, index), written when T > 1
+    long long BH, total;    // heads; items = BH * T * NT
+    int N, C, T, NT;        // tokens, centroids, centroid tiles, token tiles
+    unsigned long long wait_ns;
+};
+
+// order-preserving key of a float (-0 taken as +0), in the high half; the index in the low half
+__device__ __forceinline__ uint64_t pack_dist(float dist, int idx) {
+    const uint32_t u = __float_as_uint(dist + 0.0f);
+    const uint32_t key = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return ((uint64_t)key << 32) | (uint32_t)idx;
+}
 
 template <int D>
 __global__ void __launch_bounds__(256, 1)
     kmeans_assign_tc_kernel(const __grid_constant__ CUtensorMap tmX,
-                            const __grid_constant__ CUtensorMap tmP, const float *__restrict__ norms,
-                            int32_t *__restrict__ assign, int N, int C,
-                            unsigned long long wait_ns) {
+                            const __grid_constant__ CUtensorMap tmP, const KmParams prm) {
     using Cf = KmTcCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -370,19 +447,22 @@ __global__ void __launch_bounds__(256, 1)
     static_assert(8 * KB_COUNT + 8 <= 128, "barrier area");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int bh = blockIdx.y, n0 = blockIdx.x * 128;
-    const int T = (C + 127) / 128;  // centroid tiles
+    const long long lo = prm.total * blockIdx.x / gridDim.x;
+    const long long hi = prm.total * (blockIdx.x + 1) / gridDim.x;
+    const unsigned long long wns = prm.wait_ns;
     auto bar = [&](int b) { return smem_u32(&bars[b]); };
-    const uint32_t sX = smem_u32(smem + Cf::OFF_X);
-    auto sP = [&](int s, int p) { return smem_u32(smem + Cf::OFF_P + (s * 3 + p) * Cf::TILE); };
+    const uint32_t sP = smem_u32(smem + Cf::OFF_P), sX = smem_u32(smem + Cf::OFF_X);
 
     if (threadIdx.x == 0) {
-        mbar_init(bar(KB_XF), 1);
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(bar(KB_PF0 + s), 1);
-            mbar_init(bar(KB_PE0 + s), 1);
-            mbar_init(bar(KB_SF0 + s), 1);
-            mbar_init(bar(KB_SE0 + s), 128);
+        mbar_init(bar(KB_PF), 1);
+        mbar_init(bar(KB_PE), 1);
+        for (int s = 0; s < Cf::NX; ++s) {
+            mbar_init(bar(KB_XF0 + s), 1);
+            mbar_init(bar(KB_XE0 + s), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(bar(KB_AF0 + a), 1);
+            mbar_init(bar(KB_AE0 + a), 4);
         }
         mbar_init(bar(KB_FIN), 1);
         *abort_flag = 0;
@@ -402,101 +482,150 @@ __global__ void __launch_bounds__(256, 1)
     if (warp == 0) {
         // ------------------------------------------------------------------ producer
         bool ok = true;
-        uint32_t issued = 0;
-        if (lane == 0) {
-            mbar_arrive_expect_tx(bar(KB_XF), Cf::TILE);
-            for (int c = 0; c < Cf::CHUNKS; ++c)
-                tma_load_3d(sX + c * 16384, &tmX, bar(KB_XF), c * 64, n0, bh);
-        }
-        for (int t = 0; t < T && ok; ++t) {
-            const int s = t & 1;
-            if (t >= 2 && !(ok = warp_wait(bar(KB_PE0 + s), ((t >> 1) - 1) & 1, wait_ns, abort_flag, 0x91, t)))
+        uint32_t np = 0, nx = 0;
+        long long cur = -1;
+        for (long long t = lo; t < hi && ok; ++t) {
+            const long long g = t / prm.NT;  // (head, centroid tile)
+            const int tt = (int)(t - g * prm.NT);
+            const int bh = (int)(g / prm.T), ct = (int)(g - (long long)bh * prm.T);
+            if (g != cur) {
+                if (np > 0 && !(ok = warp_wait(bar(KB_PE), (np - 1) & 1, wns, abort_flag, 0x91, (uint32_t)t)))
+                    break;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(bar(KB_PF), 3 * Cf::TILE);
+                    for (int p = 0; p < 3; ++p)
+                        for (int c = 0; c < Cf::CHUNKS; ++c)
+                            tma_load_3d(sP + p * Cf::TILE + c * 16384, &tmP, bar(KB_PF), c * 64, ct * 128,
+                                        bh * 3 + p);
+                }
+                ++np;
+                cur = g;
+            }
+            const int s = nx % Cf::NX;
+            if (nx >= Cf::NX &&
+                !(ok = warp_wait(bar(KB_XE0 + s), ((nx / Cf::NX) - 1) & 1, wns, abort_flag, 0x92, (uint32_t)t)))
                 break;
             if (lane == 0) {
-                mbar_arrive_expect_tx(bar(KB_PF0 + s), 3 * Cf::TILE);
-                for (int p = 0; p < 3; ++p)
-                    for (int c = 0; c < Cf::CHUNKS; ++c)
-                        tma_load_3d(sP(s, p) + c * 16384, &tmP, bar(KB_PF0 + s), c * 64, t * 128,
-                                    bh * 3 + p);
+                mbar_arrive_expect_tx(bar(KB_XF0 + s), Cf::TILE);
+                for (int c = 0; c < Cf::CHUNKS; ++c)
+                    tma_load_3d(sX + s * Cf::TILE + c * 16384, &tmX, bar(KB_XF0 + s), c * 64, tt * 128, bh);
             }
-            ++issued;
+            ++nx;
         }
-        if (lane == 0) {  // every started copy lands before the CTA leaves
-            int never = 0;
-            mbar_wait(bar(KB_XF), 0, wait_ns, (volatile int *)&never, 0x98, 0);
-            for (uint32_t t = (issued > 2 ? issued - 2 : 0); t < issued; ++t)
-                mbar_wait(bar(KB_PF0 + (t & 1)), (t >> 1) & 1, wait_ns, (volatile int *)&never, 0x99, t);
+        if (!ok && lane == 0) {  // every started copy lands before the CTA leaves
+            if (np) drain_wait(bar(KB_PF), (np - 1) & 1, wns, 0x98);
+            for (uint32_t i = nx > Cf::NX ? nx - Cf::NX : 0; i < nx; ++i)
+                drain_wait(bar(KB_XF0 + i % Cf::NX), (i / Cf::NX) & 1, wns, 0x99);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------------ MMA issuer
         constexpr uint32_t IDESC = idesc_bf16_f32(128, 128, 0, 0);
-        bool ok = warp_wait(bar(KB_XF), 0, wait_ns, abort_flag, 0xA1, 0);
+        const uint64_t dP = smem_desc_sw128(sP, 16, 1024);
         const uint64_t dX = smem_desc_sw128(sX, 16, 1024);
-        for (int t = 0; t < T && ok; ++t) {
-            const int s = t & 1;  // operand stage and accumulator buffer
-            if (!(ok = warp_wait(bar(KB_PF0 + s), (t >> 1) & 1, wait_ns, abort_flag, 0xA2, t))) break;
-            if (t >= 2 && !(ok = warp_wait(bar(KB_SE0 + s), ((t >> 1) - 1) & 1, wait_ns, abort_flag, 0xA3, t)))
+        bool ok = true;
+        uint32_t np = 0, nx = 0;
+        long long cur = -1;
+        for (long long t = lo; t < hi && ok; ++t) {
+            const long long g = t / prm.NT;
+            if (g != cur) {
+                if (!(ok = warp_wait(bar(KB_PF), np & 1, wns, abort_flag, 0xA1, (uint32_t)t))) break;
+                ++np;
+                cur = g;
+            }
+            const int s = nx % Cf::NX, a = nx & 1;  // token stage, accumulator
+            if (!(ok = warp_wait(bar(KB_XF0 + s), (nx / Cf::NX) & 1, wns, abort_flag, 0xA2, (uint32_t)t))) break;
+            if (nx >= 2 && !(ok = warp_wait(bar(KB_AE0 + a), ((nx >> 1) - 1) & 1, wns, abort_flag, 0xA3, (uint32_t)t)))
                 break;
             tc_fence_after();
+            const bool last_of_group = t + 1 >= hi || (t + 1) / prm.NT != g;
             if (lane == 0) {
-                const uint32_t acc = tbase + (uint32_t)(s * 128);
+                const uint32_t acc = tbase + (uint32_t)(a * 128);
+                const uint64_t xs = (uint64_t)((s * Cf::TILE) >> 4);
 #pragma unroll
                 for (int p = 0; p < 3; ++p) {
-                    const uint64_t dP = smem_desc_sw128(sP(s, p), 16, 1024);
+                    const uint64_t ps = (uint64_t)((p * Cf::TILE) >> 4);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint64_t off = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
-                        mma_ss(acc, dX + off, dP + off, IDESC, (p > 0 || kk > 0) ? 1u : 0u);
+                        mma_ss(acc, dX + xs + off, dP + ps + off, IDESC, (p > 0 || kk > 0) ? 1u : 0u);
                     }
                 }
-                mma_commit(bar(KB_SF0 + s));
-                mma_commit(bar(KB_PE0 + s));
+                mma_commit(bar(KB_AF0 + a));
+                mma_commit(bar(KB_XE0 + s));
+                if (last_of_group) mma_commit(bar(KB_PE));
             }
             __syncwarp();
+            ++nx;
         }
-        if (lane == 0) {
-            int never = 0;
+        if (lane == 0) {  // every MMA complete before tensor memory is released
             mma_commit(bar(KB_FIN));
-            mbar_wait(bar(KB_FIN), 0, wait_ns, (volatile int *)&never, 0xA4, 0);
+            drain_wait(bar(KB_FIN), 0, wns, 0xA4);
         }
     } else if (warp >= 4) {
         // ------------------------------------------------------------------ epilogue
         const int q4 = warp & 3;
         const int r = q4 * 32 + lane;  // token row of the tile == TMEM lane
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-        float best = INFINITY;
-        int arg = 0;
         bool ok = true;
-        for (int t = 0; t < T && ok; ++t) {
-            const int s = t & 1;
-            // lane e holds the norm of column q * 32 + e (padding centroids are never nearest);
-            // no barrier among the epilogue warps, so a warp that gives up cannot stall the rest
-            float nv[4];
+        uint32_t nx = 0;
+        long long cur = -1;
+        float nv[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+        for (long long t = lo; t < hi && ok; ++t) {
+            const long long g = t / prm.NT;
+            const int tt = (int)(t - g * prm.NT);
+            const int bh = (int)(g / prm.T), ct = (int)(g - (long long)bh * prm.T);
+            if (g != cur) {
+                // lane e holds the norm of column q * 32 + e (padding centroids are never nearest)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int c = ct * 128 + q * 32 + lane;
+                    nv[q] = c < prm.C ? prm.norms[(size_t)bh * prm.C + c] : INFINITY;
+                }
+                cur = g;
+            }
+            const int a = nx & 1;  // accumulator
+            if (!(ok = warp_wait(bar(KB_AF0 + a), (nx >> 1) & 1, wns, abort_flag, 0xB1, (uint32_t)t))) break;
+            tc_fence_after();
+            // four independent first-minimum chains (one per 32 columns), merged in column order
+            float bq[4];
+            int aq[4];
+            uint32_t v[128];
+            tmem_ld_cols<128>(tbase + lane_off + (uint32_t)(a * 128), v);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const int c = t * 128 + q * 32 + lane;
-                nv[q] = c < C ? norms[(size_t)bh * C + c] : INFINITY;
-            }
-            if (!(ok = warp_wait(bar(KB_SF0 + s), (t >> 1) & 1, wait_ns, abort_flag, 0xB1, t))) break;
-            tc_fence_after();
-#pragma unroll 1
-            for (int q = 0; q < 4; ++q) {
-                uint32_t v[32];
-                tmem_ld32(tbase + lane_off + (uint32_t)(s * 128 + q * 32), v);
+                bq[q] = INFINITY;
+                aq[q] = ct * 128 + q * 32;
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                     const float cn = __shfl_sync(0xffffffffu, nv[q], e);
-                    const float dist = fmaf(-2.f, __uint_as_float(v[e]), cn);
-                    if (dist < best) {
-                        best = dist;
-                        arg = t * 128 + q * 32 + e;
+                    const float dist = fmaf(-2.f, __uint_as_float(v[q * 32 + e]), cn);
+                    if (dist < bq[q]) {
+                        bq[q] = dist;
+                        aq[q] = ct * 128 + q * 32 + e;
                     }
                 }
             }
+            float best = bq[0];
+            int arg = aq[0];
+#pragma unroll
+            for (int q = 1; q < 4; ++q) {
+                if (bq[q] < best) {
+                    best = bq[q];
+                    arg = aq[q];
+                }
+            }
             tc_fence_before();
-            mbar_arrive(bar(KB_SE0 + s));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(KB_AE0 + a));
+            const int n = tt * 128 + r;
+            if (n < prm.N) {
+                if (prm.T == 1)
+                    prm.assign[(size_t)bh * prm.N + n] = arg;
+                else
+                    prm.partial[((size_t)ct * prm.BH + bh) * prm.N + n] = pack_dist(best, arg);
+            }
+            ++nx;
         }
-        if (ok && n0 + r < N) assign[(size_t)bh * N + n0 + r] = arg;
     }
 
     __syncwarp();
@@ -504,6 +633,21 @@ __global__ void __launch_bounds__(256, 1)
     __syncthreads();
     tc_fence_after();
     if (warp == 2) tmem_dealloc(tbase, 256);
+}
+
+// assign[x] = the index of the least packed (distance, index) over the T centroid tiles
+__global__ void __launch_bounds__(256) kmeans_merge_kernel(const uint64_t *__restrict__ partial,
+                                                           int32_t *__restrict__ assign,
+                                                           long long total, int T) {
+    for (long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x; x < total;
+         x += (long long)gridDim.x * blockDim.x) {
+        uint64_t b = partial[x];
+        for (int t = 1; t < T; ++t) {
+            const uint64_t v = partial[(size_t)t * total + x];
+            b = v < b ? v : b;
+        }
+        assign[x] = (int32_t)(uint32_t)(b & 0xFFFFFFFFull);
+    }
 }
 
 // parts[bh, p, c, :] (p = 0, 1, 2: h, m, l of cent[bh, c, :]) and norms[bh, c] = |cent[bh, c]|^2
@@ -539,23 +683,44 @@ __global__ void __launch_bounds__(256) centroid_split_kernel(const float *__rest
 namespace bsa {
 
 template <int D>
-static cudaError_t launch_assign_tc(const CUtensorMap &tx, const CUtensorMap &tp,
-                                    const float *norms, int32_t *assign, long long BH, int N,
-                                    int C, unsigned long long wait_ns, cudaStream_t st) {
+static cudaError_t launch_assign_tc(const CUtensorMap &tx, const CUtensorMap &tp, const KmParams &p,
+                                    cudaStream_t st) {
     using Cf = KmTcCfg<D>;
     cudaError_t e = cudaFuncSetAttribute(kmeans_assign_tc_kernel<D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
     if (e != cudaSuccess) return e;
-    const dim3 grid((unsigned)((N + 127) / 128), (unsigned)BH);
-    kmeans_assign_tc_kernel<D><<<grid, 256, Cf::SMEM, st>>>(tx, tp, norms, assign, N, C, wait_ns);
+    int dev = 0, sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const long long grid = p.total < sms ? p.total : sms;
+    if (grid <= 0) return cudaSuccess;
+    kmeans_assign_tc_kernel<D><<<(unsigned)grid, 256, Cf::SMEM, st>>>(tx, tp, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || p.T == 1) return e;
+    const long long n = p.BH * p.N;
+    const long long blocks = (n + 255) / 256 < 16LL * sms ? (n + 255) / 256 : 16LL * sms;
+    kmeans_merge_kernel<<<(unsigned)blocks, 256, 0, st>>>(p.partial, p.assign, n, p.T);
     return cudaGetLastError();
 }
 
+// partial: [ceil(C / 128), BH, N] uint64 scratch, used when C > 128
 cudaError_t kmeans_assign_tc(const CUtensorMap &tx, const CUtensorMap &tp, const float *norms,
-                             int32_t *assign, long long BH, int N, int d, int C,
+                             int32_t *assign, uint64_t *partial, long long BH, int N, int d, int C,
                              unsigned long long wait_ns, cudaStream_t st) {
-    if (d == 128) return launch_assign_tc<128>(tx, tp, norms, assign, BH, N, C, wait_ns, st);
-    if (d == 64) return launch_assign_tc<64>(tx, tp, norms, assign, BH, N, C, wait_ns, st);
+    KmParams p;
+    p.norms = norms;
+    p.assign = assign;
+    p.partial = partial;
+    p.BH = BH;
+    p.N = N;
+    p.C = C;
+    p.T = (C + 127) / 128;
+    p.NT = (N + 127) / 128;
+    p.total = BH * p.T * p.NT;
+    p.wait_ns = wait_ns;
+    if (d == 128) return launch_assign_tc<128>(tx, tp, p, st);
+    if (d == 64) return launch_assign_tc<64>(tx, tp, p, st);
     return cudaErrorInvalidValue;
 }
 
@@ -584,21 +749,23 @@ static unsigned grid_for(long long work, int per_block, int num_sms) {
     return (unsigned)(g > 0 ? g : 1);
 }
 
-// parts: [BH, 3, C, d] bf16 scratch and norms [BH, C] fp32 scratch for the tensor-core
-// assignment; tx / tp: tensor maps of x ({d, N, BH}, 128-row boxes) and of parts
-// ({d, C, 3 BH}, 128-row boxes).
+// parts: [BH, 3, C, d] bf16, norms [BH, C] fp32 and (C > 128) partial [ceil(C / 128), BH, N]
+// uint64 scratch for the tensor-core assignment; tx / tp: tensor maps of x ({d, N, BH},
+// 128-row boxes) and of parts ({d, C, 3 BH}, 128-row boxes).
 cudaError_t kmeans_lloyd(const void *x, float *cent, int32_t *assign, int32_t *perm,
                          int32_t *cstart, int32_t *csize, long long BH, int N, int d, int C,
-                         int iters, void *parts, float *norms, const CUtensorMap *tx,
-                         const CUtensorMap *tp, unsigned long long wait_ns, cudaStream_t st) {
+                         int iters, void *parts, float *norms, uint64_t *partial, int32_t *hist,
+                         const CUtensorMap *tx, const CUtensorMap *tp, unsigned long long wait_ns,
+                         cudaStream_t st) {
     const dim3 gu((unsigned)C, (unsigned)BH);
-    const size_t sort_smem = (size_t)9 * C * sizeof(int32_t);
     const auto *xb = reinterpret_cast<const __nv_bfloat16 *>(x);
     for (int it = 0;; ++it) {
         cudaError_t e = centroid_split(cent, parts, norms, BH, C, d, st);
-        if (e == cudaSuccess) e = kmeans_assign_tc(*tx, *tp, norms, assign, BH, N, d, C, wait_ns, st);
+        if (e == cudaSuccess)
+            e = kmeans_assign_tc(*tx, *tp, norms, assign, partial, BH, N, d, C, wait_ns, st);
         if (e != cudaSuccess) return e;
-        cluster_sort_kernel<<<(unsigned)BH, 256, sort_smem, st>>>(assign, N, C, perm, cstart, csize);
+        e = cluster_sort(assign, BH, N, C, perm, cstart, csize, hist, st);
+        if (e != cudaSuccess) return e;
         if (it == iters) break;
         if (d == 128)
             kmeans_update_kernel<128><<<gu, 512, 0, st>>>(xb, perm, cstart, csize, cent, N, C);
@@ -610,11 +777,20 @@ cudaError_t kmeans_lloyd(const void *x, float *cent, int32_t *assign, int32_t *p
     return cudaGetLastError();
 }
 
+// hist: [BH, ceil(N / kSortChunk), C] int32 scratch
 cudaError_t cluster_sort(const int32_t *assign, long long BH, int N, int C, int32_t *perm,
-                         int32_t *cstart, int32_t *csize, cudaStream_t st) {
-    cluster_sort_kernel<<<(unsigned)BH, 256, (size_t)9 * C * sizeof(int32_t), st>>>(
-        assign, N, C, perm, cstart, csize);
+                         int32_t *cstart, int32_t *csize, int32_t *hist, cudaStream_t st) {
+    const int nchunk = (N + kSortChunk - 1) / kSortChunk;
+    const dim3 g((unsigned)nchunk, (unsigned)BH);
+    cluster_hist_kernel<<<g, 256, (size_t)C * sizeof(int32_t), st>>>(assign, N, C, nchunk, hist);
+    cluster_scan_kernel<<<(unsigned)BH, 1024, 0, st>>>(hist, nchunk, C, cstart, csize);
+    cluster_place_kernel<<<g, 256, (size_t)8 * C * sizeof(int32_t), st>>>(assign, hist, N, C, nchunk,
+                                                                          perm);
     return cudaGetLastError();
+}
+
+size_t cluster_sort_scratch_bytes(long long BH, int N, int C) {
+    return (size_t)BH * ((N + kSortChunk - 1) / kSortChunk) * C * sizeof(int32_t);
 }
 
 cudaError_t centroid_logits(const float *cq, const float *ck, const int32_t *size_k,
@@ -675,6 +851,8 @@ struct ClusterWorkspace {
     float *logits;
     void *parts;   // centroid parts for the tensor-core assignment, sized for max(Cq, Ck)
     float *norms;
+    uint64_t *partial;  // per-centroid-tile nearest candidates, when max(Cq, Ck) > 128
+    int32_t *hist;      // cluster-sort chunk counts
     int U, tstride;
 };
 
@@ -708,6 +886,8 @@ size_t cluster_workspace(int B, int H, int N, int d, int Cq, int Ck, bool full, 
     t.logits = nullptr;
     t.parts = nullptr;
     t.norms = nullptr;
+    t.partial = nullptr;
+    t.hist = (int32_t *)take(bsa::cluster_sort_scratch_bytes((long long)BH, N, Cq > Ck ? Cq : Ck));
     if (full) {
         t.assign_q = (int32_t *)take(BH * N * 4);
         t.assign_k = (int32_t *)take(BH * N * 4);
@@ -716,6 +896,7 @@ size_t cluster_workspace(int B, int H, int N, int d, int Cq, int Ck, bool full, 
         const size_t Cm = (size_t)(Cq > Ck ? Cq : Ck);
         t.parts = take(BH * 3 * Cm * d * 2);
         t.norms = (float *)take(BH * Cm * 4);
+        t.partial = Cm > 128 ? (uint64_t *)take(((Cm + 127) / 128) * BH * N * 8) : nullptr;
     }
     t.U = U;
     t.tstride = tstride;
@@ -771,10 +952,13 @@ cudaError_t centroid_select(const float *cq, const float *ck, const int32_t *siz
 
 }  // namespace
 
-extern "C" size_t sa_kmeans_workspace_bytes(int B, int H, int C, int d) {
-    if (B <= 0 || H <= 0 || C <= 0 || d <= 0) return 0;
+extern "C" size_t sa_kmeans_workspace_bytes(int B, int H, int N, int C, int d) {
+    if (B <= 0 || H <= 0 || N <= 0 || C <= 0 || d <= 0) return 0;
     const size_t BH = (size_t)B * H;
-    return round256(BH * 3 * (size_t)C * d * 2) + round256(BH * (size_t)C * 4);
+    const size_t T = ((size_t)C + 127) / 128;
+    return round256(BH * 3 * (size_t)C * d * 2) + round256(BH * (size_t)C * 4) +
+           (T > 1 ? round256(T * BH * (size_t)N * 8) : 0) +
+           round256(bsa::cluster_sort_scratch_bytes((long long)BH, N, C));
 }
 
 extern "C" sa_status sa_kmeans(const void *x, float *cent, int32_t *assign, int32_t *perm,
@@ -783,7 +967,7 @@ extern "C" sa_status sa_kmeans(const void *x, float *cent, int32_t *assign, int3
     if (!x || !cent || !assign || !perm || !cstart || !csize || !workspace) return SA_ERR_INVALID_ARG;
     if (!shape_ok(B, H, N) || !clusters_ok(C) || iters < 0) return SA_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return SA_ERR_UNSUPPORTED;
-    if (workspace_bytes < sa_kmeans_workspace_bytes(B, H, C, d) || !aligned16(workspace))
+    if (workspace_bytes < sa_kmeans_workspace_bytes(B, H, N, C, d) || !aligned16(workspace))
         return SA_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(cent) || !aligned4(assign) || !aligned4(perm) ||
         !aligned4(cstart) || !aligned4(csize))
@@ -794,23 +978,37 @@ extern "C" sa_status sa_kmeans(const void *x, float *cent, int32_t *assign, int3
     void *parts = workspace;
     float *norms = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) +
                                              round256((size_t)BH * 3 * C * d * 2));
+    uint8_t *after_norms = reinterpret_cast<uint8_t *>(norms) + round256((size_t)BH * C * 4);
+    uint64_t *partial = C > 128 ? reinterpret_cast<uint64_t *>(after_norms) : nullptr;
+    const size_t T = ((size_t)C + 127) / 128;
+    int32_t *hist = reinterpret_cast<int32_t *>(after_norms +
+                                                (T > 1 ? round256(T * BH * (size_t)N * 8) : 0));
     CUtensorMap tx, tp;
     if (!make_tmap(&tx, x, BH, N, d, 128) || !make_tmap(&tp, parts, BH * 3, C, d, 128))
         return SA_ERR_CUDA;
     return from_cuda(bsa::kmeans_lloyd(x, cent, assign, perm, cstart, csize, BH, N, d, C, iters,
-                                       parts, norms, &tx, &tp, g_wait_ns, (cudaStream_t)stream));
+                                       parts, norms, partial, hist, &tx, &tp, g_wait_ns,
+                                       (cudaStream_t)stream));
+}
+
+extern "C" size_t sa_cluster_sort_workspace_bytes(int B, int H, int N, int C) {
+    if (B <= 0 || H <= 0 || N <= 0 || C <= 0) return 0;
+    return round256(bsa::cluster_sort_scratch_bytes((long long)B * H, N, C));
 }
 
 extern "C" sa_status sa_cluster_sort(const int32_t *assign, int B, int H, int N, int C,
                                      int32_t *perm, int32_t *cstart, int32_t *csize,
-                                     void *stream) {
-    if (!assign || !perm || !cstart || !csize) return SA_ERR_INVALID_ARG;
+                                     void *workspace, size_t workspace_bytes, void *stream) {
+    if (!assign || !perm || !cstart || !csize || !workspace) return SA_ERR_INVALID_ARG;
     if (!shape_ok(B, H, N) || !clusters_ok(C)) return SA_ERR_INVALID_ARG;
     if (!aligned4(assign) || !aligned4(perm) || !aligned4(cstart) || !aligned4(csize))
+        return SA_ERR_INVALID_ARG;
+    if (workspace_bytes < sa_cluster_sort_workspace_bytes(B, H, N, C) || !aligned16(workspace))
         return SA_ERR_INVALID_ARG;
     int dev;
     if (!select_device(perm, &dev)) return SA_ERR_INVALID_ARG;
     return from_cuda(bsa::cluster_sort(assign, (long long)B * H, N, C, perm, cstart, csize,
+                                       reinterpret_cast<int32_t *>(workspace),
                                        (cudaStream_t)stream));
 }
 
@@ -868,8 +1066,9 @@ extern "C" sa_status sa_cluster_attn_fwd(const void *q, const void *k, const voi
     ClusterWorkspace w;
     cluster_workspace(B, H, N, d, Cq, Ck, false, workspace, &w);
     const long long BH = (long long)B * H;
-    cudaError_t e = bsa::cluster_sort(assign_q, BH, N, Cq, w.perm_q, w.qstart, w.qsize, st);
-    if (e == cudaSuccess) e = bsa::cluster_sort(assign_k, BH, N, Ck, w.perm_k, w.kstart, w.ksize, st);
+    cudaError_t e = bsa::cluster_sort(assign_q, BH, N, Cq, w.perm_q, w.qstart, w.qsize, w.hist, st);
+    if (e == cudaSuccess)
+        e = bsa::cluster_sort(assign_k, BH, N, Ck, w.perm_k, w.kstart, w.ksize, w.hist, st);
     if (e != cudaSuccess) return SA_ERR_CUDA;
     return cluster_attention_tail(q, k, v, o, sel, w, B, H, N, d, Cq, Ck, scale, dev, st);
 }
@@ -904,10 +1103,12 @@ extern "C" sa_status sa_svg2_attn_fwd(const void *q, const void *k, const void *
         !make_tmap(&tpq, w.parts, BH * 3, Cq, d, 128) || !make_tmap(&tpk, w.parts, BH * 3, Ck, d, 128))
         return SA_ERR_CUDA;
     cudaError_t e = bsa::kmeans_lloyd(q, cent_q, w.assign_q, w.perm_q, w.qstart, w.qsize, BH, N, d,
-                                      Cq, iters, w.parts, w.norms, &txq, &tpq, g_wait_ns, st);
+                                      Cq, iters, w.parts, w.norms, w.partial, w.hist, &txq, &tpq,
+                                      g_wait_ns, st);
     if (e == cudaSuccess)
         e = bsa::kmeans_lloyd(k, cent_k, w.assign_k, w.perm_k, w.kstart, w.ksize, BH, N, d, Ck,
-                              iters, w.parts, w.norms, &txk, &tpk, g_wait_ns, st);
+                              iters, w.parts, w.norms, w.partial, w.hist, &txk, &tpk, g_wait_ns,
+                              st);
     if (e == cudaSuccess)
         e = centroid_select(cent_q, cent_k, w.ksize, BH, Cq, Ck, d, topp, resolve_scale(scale, d),
                             sel, w.logits, w.sel_cnt, num_sms(dev), st);

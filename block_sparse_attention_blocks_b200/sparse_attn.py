@@ -40,9 +40,11 @@ lib.sa_squad_workspace_bytes.argtypes = [_I, _I, _I, _I]
 lib.sa_squad_workspace_bytes.restype = _Z
 lib.sa_squad_attn_fwd.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _Z, _P]
 lib.sa_kmeans.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _Z, _P]
-lib.sa_kmeans_workspace_bytes.argtypes = [_I, _I, _I, _I]
+lib.sa_kmeans_workspace_bytes.argtypes = [_I, _I, _I, _I, _I]
 lib.sa_kmeans_workspace_bytes.restype = _Z
-lib.sa_cluster_sort.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P, _P]
+lib.sa_cluster_sort.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P, _P, _Z, _P]
+lib.sa_cluster_sort_workspace_bytes.argtypes = [_I, _I, _I, _I]
+lib.sa_cluster_sort_workspace_bytes.restype = _Z
 lib.sa_centroid_topp_workspace_bytes.argtypes = [_I, _I, _I, _I]
 lib.sa_centroid_topp_workspace_bytes.restype = _Z
 lib.sa_centroid_topp.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _F, _F, _P, _P, _Z, _P]
@@ -389,7 +391,7 @@ def kmeans(x, cent, iters: int):
     perm = torch.empty_like(assign)
     cstart = torch.empty(B, H, C, device=x.device, dtype=torch.int32)
     csize = torch.empty_like(cstart)
-    nbytes = int(lib.sa_kmeans_workspace_bytes(B, H, C, d))
+    nbytes = int(lib.sa_kmeans_workspace_bytes(B, H, N, C, d))
     ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=x.device)
     _check(lib.sa_kmeans(_ptr(x), _ptr(cent), _ptr(assign), _ptr(perm), _ptr(cstart), _ptr(csize),
                          B, H, N, d, C, int(iters), _ptr(ws), ws.numel(), _stream(x.device)),
@@ -405,8 +407,11 @@ def cluster_sort(assign, C: int):
     perm = torch.empty_like(assign)
     cstart = torch.empty(B, H, C, device=assign.device, dtype=torch.int32)
     csize = torch.empty_like(cstart)
+    nbytes = int(lib.sa_cluster_sort_workspace_bytes(B, H, N, int(C)))
+    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=assign.device)
     _check(lib.sa_cluster_sort(_ptr(assign), B, H, N, int(C), _ptr(perm), _ptr(cstart),
-                               _ptr(csize), _stream(assign.device)), "sa_cluster_sort")
+                               _ptr(csize), _ptr(ws), ws.numel(), _stream(assign.device)),
+           "sa_cluster_sort")
     return perm, cstart, csize
 
 

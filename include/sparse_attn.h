@@ -158,9 +158,10 @@ sa_status sa_squad_attn_fwd(const void *q, const void *k, const void *v, void *o
  *   in perm.  Cluster sums run in token order, so results repeat bit for bit.  The nearest
  *   centroid runs on the tensor cores (rows exact in bf16, each fp32 centroid split exactly
  *   into three bf16 parts, fp32 accumulation); workspace: sa_kmeans_workspace_bytes() bytes,
- *   16-byte aligned, owned by the caller (the centroid parts and norms).
+ *   16-byte aligned, owned by the caller (the centroid parts and norms, and for C > 128 each
+ *   128-centroid tile's nearest candidate per token).
  */
-size_t sa_kmeans_workspace_bytes(int B, int H, int C, int d);
+size_t sa_kmeans_workspace_bytes(int B, int H, int N, int C, int d);
 sa_status sa_kmeans(const void *x, float *cent, int32_t *assign, int32_t *perm, int32_t *cstart,
                     int32_t *csize, int B, int H, int N, int d, int C, int iters, void *workspace,
                     size_t workspace_bytes, void *stream);
@@ -168,10 +169,13 @@ sa_status sa_kmeans(const void *x, float *cent, int32_t *assign, int32_t *perm, 
 /*
  * The stable order of the tokens by cluster id (the permutation of section A) alone:
  * assign [B, H, N] int32 ids in [0, C) (others are clamped and flagged in the device error word)
- * -> perm, cstart, csize as for sa_kmeans.
+ * -> perm, cstart, csize as for sa_kmeans.  workspace: sa_cluster_sort_workspace_bytes() bytes,
+ * 16-byte aligned, owned by the caller (per-chunk cluster counts).
  */
+size_t sa_cluster_sort_workspace_bytes(int B, int H, int N, int C);
 sa_status sa_cluster_sort(const int32_t *assign, int B, int H, int N, int C, int32_t *perm,
-                          int32_t *cstart, int32_t *csize, void *stream);
+                          int32_t *cstart, int32_t *csize, void *workspace,
+                          size_t workspace_bytes, void *stream);
 
 /*
  * Centroid top-p (section B).  For query cluster a of head (b, h), key cluster j is estimated to

@@ -269,10 +269,14 @@ def test_squad_argument_checks(lib):
 def test_cluster_entry_point_argument_checks(lib):
     I, P, F, Z = ctypes.c_int, ctypes.c_void_p, ctypes.c_float, ctypes.c_size_t
     lib.sa_kmeans_workspace_bytes.restype = Z
-    lib.sa_kmeans_workspace_bytes.argtypes = [I] * 4
-    Wk = lib.sa_kmeans_workspace_bytes(1, 2, 8, 64)
+    lib.sa_kmeans_workspace_bytes.argtypes = [I] * 5
+    Wk = lib.sa_kmeans_workspace_bytes(1, 2, 100, 8, 64)
     assert Wk >= 2 * 3 * 8 * 64 * 2 + 2 * 8 * 4       # centroid parts (bf16) and norms
-    assert lib.sa_kmeans_workspace_bytes(0, 2, 8, 64) == 0
+    assert lib.sa_kmeans_workspace_bytes(0, 2, 100, 8, 64) == 0
+    assert lib.sa_kmeans_workspace_bytes(1, 2, 0, 8, 64) == 0
+    # above 128 centroids, each 128-centroid tile's candidate per token (8 bytes) is kept too
+    assert (lib.sa_kmeans_workspace_bytes(1, 2, 100, 300, 64)
+            >= 2 * 3 * 300 * 64 * 2 + 2 * 300 * 4 + 3 * 2 * 100 * 8)
     km = lib.sa_kmeans
     km.argtypes = [P] * 6 + [I] * 6 + [P, Z, P]
     assert km(NUL, A, A, A, A, A, 1, 2, 100, 64, 8, 2, A2, Wk, S) == 1
@@ -283,10 +287,17 @@ def test_cluster_entry_point_argument_checks(lib):
     assert km(A, MIS, A, A, A, A, 1, 2, 100, 64, 8, 2, A2, Wk, S) == 1        # centroids need 16 B
     assert km(A, A, A, A, A, A, 1, 2, 100, 64, 8, 2, NUL, Wk, S) == 1         # no workspace
     assert km(A, A, A, A, A, A, 1, 2, 100, 64, 8, 2, A2, Wk - 1, S) == 1      # workspace too small
+    lib.sa_cluster_sort_workspace_bytes.restype = Z
+    lib.sa_cluster_sort_workspace_bytes.argtypes = [I] * 4
+    Ws = lib.sa_cluster_sort_workspace_bytes(1, 2, 10000, 40)
+    assert Ws >= 2 * 3 * 40 * 4                         # counts of every 4096-token chunk
+    assert lib.sa_cluster_sort_workspace_bytes(1, 2, 0, 40) == 0
     cs = lib.sa_cluster_sort
-    cs.argtypes = [P] + [I] * 4 + [P] * 4
-    assert cs(NUL, 1, 1, 10, 4, A, A, A, S) == 1
-    assert cs(A, 1, 1, 10, 4, MIS4, A, A, S) == 1
+    cs.argtypes = [P] + [I] * 4 + [P] * 4 + [Z, P]
+    assert cs(NUL, 1, 1, 10, 4, A, A, A, A2, Ws, S) == 1
+    assert cs(A, 1, 1, 10, 4, MIS4, A, A, A2, Ws, S) == 1
+    assert cs(A, 1, 2, 10000, 40, A, A, A, NUL, Ws, S) == 1       # no workspace
+    assert cs(A, 1, 2, 10000, 40, A, A, A, A2, Ws - 1, S) == 1    # workspace too small
 
     lib.sa_centroid_topp_workspace_bytes.restype = Z
     lib.sa_centroid_topp_workspace_bytes.argtypes = [I] * 4
