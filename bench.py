@@ -765,7 +765,7 @@ def run_gpu(args, w):
                else {"parallelism": f"{world} independent replicas" if world > 1 else "1 GPU"}),
             "realized_density": density, "executed_pairs": pairs,
                                   "effective_flops_per_call": flops}),
-        "roofline": {"kernel": "attn_fwd_kernel<128,128>", "bound": "tensor",
+        "roofline": {"kernel": "attn_fwd_kernel<128,128,BlockWalk>", "bound": "tensor",
                      "achieved": att_tflops, "peak": peak_tc, "unit": "TFLOP/s",
                      "frac": att_tflops / peak_tc,
                      "traffic": attention_traffic(w.name, B * H, pairs),

@@ -1,7 +1,10 @@
-// Block-sparse attention forward over a compacted per-query-block key-block list, and the dense
-// control (every key block).
+// Attention forward on the tensor cores over per-unit lists of key tiles: the block-sparse
+// attention over a compacted per-query-block key-block list and its dense control (every key
+// block), and attention over clusters of variable size (the kernel behind the semantic-aware
+// permutation of Sparse VideoGen2, section 2.A and 2.C), in one kernel template whose tile
+// addressing is a policy (BlockWalk, TileWalk).
 //
-// For each query block i and each kept key block j, S = Q_i K_j^T is a dense 128 x BS x d
+// Block lists: for each query block i and each kept key block j, S = Q_i K_j^T is a dense 128 x BS x d
 // contraction and O_i += P V_j a dense 128 x d x BS one, so both run on the tcgen05 tensor cores
 // with fp32 accumulators in tensor memory; softmax is online as in FlashAttention (a reference
 // max per row from the first kept block, P allowed to reach 2^30 before the reference moves and
@@ -11,9 +14,20 @@
 // for BS = 64, rows of the next query block inside the 128-row tile) are computed but not
 // stored.  A query block with an empty list writes zeros.
 //
+// Variable-length tiles: Q, K and V arrive already permuted (each cluster a contiguous range of
+// rows of its head).  A work unit is a query tile, up to 128 consecutive rows of one query
+// cluster; its key list is its cluster's list of key tiles of up to 128 consecutive permuted rows,
+// each given by its first row and its number of valid keys (keys past that count belong to the
+// next cluster and are masked).  A TMA row coordinate may be any row, so tiles start inside
+// clusters rather than on block boundaries.  The output row of permuted query row s is written at
+// its original position perm_q[s], which undoes the permutation.  The query tensor may have
+// another length than the keys (Nq rows against N keys).  In the split form each query
+// "cluster" is one run of the keys and the kernel writes, per cluster, the fp32 output of that run
+// with its log2-sum-exp, for the caller to combine.
+//
 // CTA roles (256 threads, two CTAs per SM, persistent; query blocks are claimed dynamically
 // from a counter in the caller's workspace, in head-major order):
-//   warp 0 lane 0  TMA producer: Q tile once per query block, then K_j and V_j per kept block
+//   warp 0 lane 0  TMA producer: Q tile once per unit, then K and V per key tile
 //   warp 1 lane 0  MMA issuer:   S = Q K_j^T (SS form), O += P V_j (P read from tensor memory)
 //   warp 2         tensor-memory allocator (256 columns: S/P at 0, O at 128)
 //   warps 4..7     softmax: one thread per query row; reads S, writes P (bf16) over S, rescales
@@ -25,16 +39,123 @@
 
 namespace bsa {
 
-struct AttnParams {
+// Parameters common to both tile-addressing policies.
+struct AttnCommon {
+    float scale_log2;        // softmax scale * log2(e)
+    unsigned long long wait_ns;
+    unsigned int *progress;  // optional host-mapped [grid, 8] stage words for diagnosis
+    unsigned int *next_unit; // work counter in the caller's workspace, zero at launch
+};
+
+// One work unit as the roles see it: its head, its query tile (first row, rows to store; 0
+// rows: no work), its key-tile count and list, and its query cluster.
+struct AttnUnit {
+    int bh, q0, rows, cnt, cluster;
+    const int32_t *list;
+};
+struct KeyTile {
+    int k0, valid;  // first key row, keys in the tile
+};
+struct AttnOut {
+    __nv_bfloat16 *row;  // bf16 output row
+    float *part, *lse;   // or, in the split form, the fp32 row and its log2-sum-exp
+};
+
+// Block lists: unit u = query block i of head bh (head-major), key tile j = key block j.
+template <int D, int BS>
+struct BlockWalk {
+    static constexpr int kD = D, kBS = BS;
+    static constexpr bool kSplit = false;
     const int32_t *kv_idx;  // [units, nbk] ascending key-block ids, or null for dense
     const int32_t *kv_cnt;  // [units], or null for dense
     __nv_bfloat16 *o;       // [BH, N, D]
     int N, nbq, nbk;
-    long long units;        // BH * nbq
-    float scale_log2;       // softmax scale * log2(e)
-    unsigned long long wait_ns;
-    unsigned int *progress;  // optional host-mapped [grid, 8] stage words for diagnosis
-    unsigned int *next_unit; // work counter in the caller's workspace, zero at launch
+    long long nunits;       // BH * nbq
+
+    __device__ __forceinline__ AttnUnit unit(long long u) const {
+        AttnUnit w;
+        w.bh = (int)(u / nbq);
+        w.q0 = (int)(u - (long long)w.bh * nbq) * BS;
+        w.rows = min(BS, N - w.q0);
+        w.cnt = kv_idx ? min(max(kv_cnt[u], 0), nbk) : nbk;
+        w.cluster = 0;
+        w.list = kv_idx ? kv_idx + (size_t)u * nbk : nullptr;
+        return w;
+    }
+    __device__ __forceinline__ int32_t entry(const AttnUnit &w, int t) const {
+        return w.list ? w.list[t] : t;
+    }
+    // an id outside [0, nbk) is clamped (and flagged once, by the producer)
+    __device__ __forceinline__ KeyTile key(int32_t j, bool flag) const {
+        if (j < 0 || j >= nbk) {
+            if (flag) atomicOr(&g_bsa_device_error, BSA_DEVERR_BOUNDS);
+            j = j < 0 ? 0 : nbk - 1;
+        }
+        return KeyTile{j * BS, min(BS, N - j * BS)};
+    }
+    __device__ __forceinline__ AttnOut out(const AttnUnit &w, int r, bool row_ok) const {
+        return AttnOut{o + ((size_t)w.bh * N + (row_ok ? w.q0 + r : 0)) * D, nullptr, nullptr};
+    }
+};
+
+// Variable-length tiles: unit u = entry u of the query-tile table (units_per_head per head),
+// key tile = entry (k_row0 << 7) | (valid - 1) of its cluster's list.
+template <int D>
+struct TileWalk {
+    static constexpr int kD = D;
+    static constexpr bool kSplit = true;
+    const int2 *units;      // [BH * units_per_head] {q_row0, q_rows << 16 | cluster}; q_rows = 0: none
+    const int32_t *tiles;   // [BH * Cq, tstride] key tiles (k_row0 << 7) | (valid - 1)
+    const int32_t *tcnt;    // [BH * Cq] key tiles in each query cluster's list
+    const int32_t *perm_q;  // [BH, Nq] original position of each permuted query row
+    __nv_bfloat16 *o;       // [BH, Nq, D] in the original order
+    float *part_o;          // or, when set: [Cq, BH, Nq, D] fp32 O / l per query cluster ...
+    float *part_lse;        // ... and [Cq, BH, Nq] its log2-sum-exp (log2 l + the row's max)
+    long long BH, nunits;   // nunits = BH * units_per_head
+    int N, Nq, Cq, tstride, units_per_head;  // N keys, Nq query (and output) rows
+
+    __device__ __forceinline__ AttnUnit unit(long long u) const {
+        const int2 e = units[u];
+        AttnUnit w;
+        w.bh = (int)(u / units_per_head);
+        w.rows = (int)((uint32_t)e.y >> 16);
+        w.cluster = e.y & 0xFFFF;
+        w.q0 = e.x;
+        if (w.rows > 0 && (w.rows > 128 || w.q0 < 0 || w.q0 > Nq - w.rows || w.cluster >= Cq)) {
+            atomicOr(&g_bsa_device_error, BSA_DEVERR_BOUNDS);
+            w.rows = 0;  // a malformed unit is skipped by every role alike
+        }
+        const size_t row = (size_t)w.bh * Cq + (w.rows ? w.cluster : 0);
+        w.cnt = w.rows ? min(max(tcnt[row], 0), tstride) : 0;
+        w.list = tiles + row * tstride;
+        return w;
+    }
+    __device__ __forceinline__ int32_t entry(const AttnUnit &w, int t) const { return w.list[t]; }
+    // first row and valid count of a key tile entry, clamped into the head
+    __device__ __forceinline__ KeyTile key(int32_t e, bool flag) const {
+        KeyTile k;
+        k.k0 = (int)((uint32_t)e >> 7);
+        k.valid = (e & 127) + 1;
+        if (k.k0 >= N) {
+            if (flag) atomicOr(&g_bsa_device_error, BSA_DEVERR_BOUNDS);
+            k.k0 = N - 1;
+        }
+        k.valid = min(k.valid, N - k.k0);
+        return k;
+    }
+    __device__ __forceinline__ AttnOut out(const AttnUnit &w, int r, bool row_ok) const {
+        int orig = 0;
+        if (row_ok) {
+            orig = perm_q[(size_t)w.bh * Nq + w.q0 + r];
+            if (orig < 0 || orig >= Nq) {
+                atomicOr(&g_bsa_device_error, BSA_DEVERR_BOUNDS);
+                orig = 0;
+            }
+        }
+        const size_t prow = ((size_t)w.cluster * BH + w.bh) * Nq + orig;
+        return AttnOut{o ? o + ((size_t)w.bh * Nq + orig) * D : nullptr,
+                       part_o ? part_o + prow * D : nullptr, part_lse ? part_lse + prow : nullptr};
+    }
 };
 
 // Stage report for diagnosis: word (cta, role) = stage << 24 | step << 12 | unit (low bits).
@@ -77,18 +198,10 @@ enum { B_QF, B_QE, B_KF, B_KE, B_VF, B_VE, B_SF, B_PF, B_OD, B_ED, B_FIN,
        B_COUNT };
 constexpr int UNIT_RING = 4;
 
-__device__ __forceinline__ int clamp_block(int j, int nbk) {
-    if (j < 0 || j >= nbk) {
-        atomicOr(&g_bsa_device_error, BSA_DEVERR_BOUNDS);
-        j = j < 0 ? 0 : nbk - 1;
-    }
-    return j;
-}
-
-template <int D, int BS>
+template <int D, int BS, class Walk>
 __global__ void __launch_bounds__(256, 2)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const AttnParams prm) {
+                    const __grid_constant__ CUtensorMap tmV, const Walk walk, const AttnCommon prm) {
     using C = AttnCfg<D, BS>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -141,7 +254,6 @@ __global__ void __launch_bounds__(256, 2)
     const uint32_t tS = tbase + C::COL_S;
     const uint32_t tO = tbase + C::COL_O;
     const unsigned long long wns = prm.wait_ns;
-    const bool dense = prm.kv_idx == nullptr;
 
     if (warp == 0) {
         regs_dec<C::REGS_LO>();
@@ -161,16 +273,14 @@ __global__ void __launch_bounds__(256, 2)
             long long u = 0;
             if (lane == 0) {
                 u = (long long)atomicAdd(prm.next_unit, 1u);
-                s_unit[slot] = u < prm.units ? (int)u : -1;
+                s_unit[slot] = u < walk.nunits ? (int)u : -1;
                 mbar_arrive(bar(B_UF0 + slot));
             }
             u = __shfl_sync(0xffffffffu, u, 0);
-            if (u >= prm.units) break;
-            const int cnt = dense ? prm.nbk : min(max(prm.kv_cnt[u], 0), prm.nbk);
-            if (cnt == 0) continue;
-            const int bh = (int)(u / prm.nbq);
-            const int i = (int)(u - (long long)bh * prm.nbq);
-            const int32_t *list = dense ? nullptr : prm.kv_idx + (size_t)u * prm.nbk;
+            if (u >= walk.nunits) break;
+            const AttnUnit w = walk.unit(u);
+            const int cnt = w.cnt;
+            if (w.rows == 0 || cnt == 0) continue;
             report(prm.progress, 0, 1, 0, u);
             if (nq > 0 && !(ok = warp_wait(bar(B_QE), (nq - 1) & 1, wns, abort_flag, 0x11, (uint32_t)u)))
                 break;
@@ -178,14 +288,14 @@ __global__ void __launch_bounds__(256, 2)
                 mbar_arrive_expect_tx(bar(B_QF), C::Q_BYTES);
 #pragma unroll
                 for (int c = 0; c < C::CHUNKS; ++c)
-                    tma_load_3d(sQ + c * C::Q_CHUNK, &tmQ, bar(B_QF), c * 64, i * BS, bh);
+                    tma_load_3d(sQ + c * C::Q_CHUNK, &tmQ, bar(B_QF), c * 64, w.q0, w.bh);
             }
             ++nq;
-            int jn = dense ? 0 : list[0];
+            int32_t en = walk.entry(w, 0);
             for (int t = 0; t < cnt; ++t) {
                 const uint32_t where = ((uint32_t)t << 16) | ((uint32_t)u & 0xFFFFu);
-                const int j = dense ? t : clamp_block(jn, prm.nbk);
-                if (!dense && t + 1 < cnt) jn = list[t + 1];  // next id, fetched early
+                const KeyTile kt = walk.key(en, true);
+                if (t + 1 < cnt) en = walk.entry(w, t + 1);  // next entry, fetched early
                 report(prm.progress, 0, 2, t, u);
                 if (nk > 0 && !(ok = warp_wait(bar(B_KE), (nk - 1) & 1, wns, abort_flag, 0x12, where)))
                     break;
@@ -193,7 +303,7 @@ __global__ void __launch_bounds__(256, 2)
                     mbar_arrive_expect_tx(bar(B_KF), C::KV_BYTES);
 #pragma unroll
                     for (int c = 0; c < C::CHUNKS; ++c)
-                        tma_load_3d(sK + c * C::KV_CHUNK, &tmK, bar(B_KF), c * 64, j * BS, bh);
+                        tma_load_3d(sK + c * C::KV_CHUNK, &tmK, bar(B_KF), c * 64, kt.k0, w.bh);
                 }
                 ++nk;
                 report(prm.progress, 0, 3, t, u);
@@ -203,7 +313,7 @@ __global__ void __launch_bounds__(256, 2)
                     mbar_arrive_expect_tx(bar(B_VF), C::KV_BYTES);
 #pragma unroll
                     for (int c = 0; c < C::CHUNKS; ++c)
-                        tma_load_3d(sV + c * C::KV_CHUNK, &tmV, bar(B_VF), c * 64, j * BS, bh);
+                        tma_load_3d(sV + c * C::KV_CHUNK, &tmV, bar(B_VF), c * 64, kt.k0, w.bh);
                 }
                 ++nv;
             }
@@ -238,8 +348,9 @@ __global__ void __launch_bounds__(256, 2)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_UE0 + slot));
             if (u < 0) break;
-            const int cnt = dense ? prm.nbk : min(max(prm.kv_cnt[u], 0), prm.nbk);
-            if (cnt == 0) continue;
+            const AttnUnit w = walk.unit(u);
+            const int cnt = w.cnt;
+            if (w.rows == 0 || cnt == 0) continue;
             report(prm.progress, 1, 1, 0, u);
             if (!(ok = warp_wait(bar(B_QF), nq & 1, wns, abort_flag, 0x21, (uint32_t)u))) break;
             ++nq;
@@ -322,28 +433,33 @@ __global__ void __launch_bounds__(256, 2)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_UE0 + slot));
             if (u < 0) break;
-            const int cnt = dense ? prm.nbk : min(max(prm.kv_cnt[u], 0), prm.nbk);
-            const int bh = (int)(u / prm.nbq);
-            const int i = (int)(u - (long long)bh * prm.nbq);
-            const int grow = i * BS + r;
-            const bool row_ok = r < BS && grow < prm.N;
-            __nv_bfloat16 *orow = prm.o + ((size_t)bh * prm.N + (row_ok ? grow : 0)) * D;
-            if (cnt == 0) {
+            const AttnUnit w = walk.unit(u);
+            if (w.rows == 0) continue;  // no query rows in this unit
+            const int cnt = w.cnt;
+            const bool row_ok = r < w.rows;
+            const AttnOut out = walk.out(w, r, row_ok);
+            if (cnt == 0) {  // nothing kept: zeros
                 if (row_ok) {
-                    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                    if (Walk::kSplit && out.part) {
+                        float4 *dst = reinterpret_cast<float4 *>(out.part);
+#pragma unroll 4
+                        for (int c = 0; c < D / 4; ++c) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        *out.lse = -INFINITY;
+                    } else {
+                        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-                    for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4 *>(orow)[c] = z;
+                        for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4 *>(out.row)[c] = z;
+                    }
                 }
                 continue;
             }
-            const int32_t *list = dense ? nullptr : prm.kv_idx + (size_t)u * prm.nbk;
             float m_ref = 0.f;        // reference max, log2 domain (set by the first block)
             float l = 0.f;            // running sum
-            int jn = dense ? 0 : list[0];
+            int32_t en = walk.entry(w, 0);
             for (int t = 0; t < cnt; ++t) {
-                const int j = dense ? t : min(max(jn, 0), prm.nbk - 1);
-                if (!dense && t + 1 < cnt) jn = list[t + 1];  // next id, fetched early
-                const int valid = min(BS, prm.N - j * BS);
+                const KeyTile kt = walk.key(en, false);
+                if (t + 1 < cnt) en = walk.entry(w, t + 1);  // next entry, fetched early
+                const int valid = kt.valid;
                 report(prm.progress, 4 + q4, 1, t, u);
                 if (!(ok = warp_wait(bar(B_SF), ns & 1, wns, abort_flag, 0x31, ((uint32_t)t << 16) | ((uint32_t)u & 0xFFFFu)))) break;
                 ++ns;
@@ -351,7 +467,7 @@ __global__ void __launch_bounds__(256, 2)
                 // the whole S row of this thread: BS fp32 scores, one TMEM round trip
                 uint32_t s[BS];
                 tmem_ld_cols<BS>(tSr, s);
-                if (valid < BS) {  // ragged last key block (warp-uniform branch)
+                if (valid < BS) {  // keys past the tile's valid count (warp-uniform branch)
 #pragma unroll
                     for (int e = 0; e < BS; ++e)
                         if (e >= valid) s[e] = __float_as_uint(-INFINITY);
@@ -408,6 +524,24 @@ __global__ void __launch_bounds__(256, 2)
             if (!(ok = warp_wait(bar(B_OD), (npv - 1) & 1, wns, abort_flag, 0x32, (uint32_t)u))) break;
             tc_fence_after();
             const float inv_l = 1.f / l;
+            if (Walk::kSplit && out.part) {  // fp32 output of this key run and its log2-sum-exp
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32(tOr + c * 32, v);
+                    if (row_ok) {
+                        float4 *dst = reinterpret_cast<float4 *>(out.part + c * 32);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            dst[q] = make_float4(__uint_as_float(v[4 * q]) * inv_l, __uint_as_float(v[4 * q + 1]) * inv_l,
+                                                 __uint_as_float(v[4 * q + 2]) * inv_l, __uint_as_float(v[4 * q + 3]) * inv_l);
+                    }
+                }
+                if (row_ok) *out.lse = m_ref + log2f(l);
+                tc_fence_before();
+                mbar_arrive(bar(B_ED));
+                continue;
+            }
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t v[32];
@@ -418,7 +552,7 @@ __global__ void __launch_bounds__(256, 2)
                     for (int e = 0; e < 32; e += 2)
                         pk[e >> 1] = pack_bf16(__uint_as_float(v[e]) * inv_l,
                                                __uint_as_float(v[e + 1]) * inv_l);
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+                    uint4 *dst = reinterpret_cast<uint4 *>(out.row + c * 32);
 #pragma unroll
                     for (int w = 0; w < 4; ++w)
                         dst[w] = make_uint4(pk[4 * w], pk[4 * w + 1], pk[4 * w + 2], pk[4 * w + 3]);
@@ -445,27 +579,27 @@ __global__ void __launch_bounds__(256, 2)
 // ------------------------------------------------------------------------------------------
 // host side
 // ------------------------------------------------------------------------------------------
-template <int D, int BS>
+template <int D, int BS, class Walk>
 static cudaError_t launch_attn_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                 const AttnParams &p, int num_sms, cudaStream_t st) {
+                                 const Walk &w, const AttnCommon &cm, int num_sms, cudaStream_t st) {
     using C = AttnCfg<D, BS>;
+    auto *kern = attn_fwd_kernel<D, BS, Walk>;
     // at least 80 KB per CTA so that no more than two CTAs (2 x 256 TMEM columns) share an SM
     const int smem = C::SMEM > 80 * 1024 ? C::SMEM : 80 * 1024;
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, BS>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     // setmaxnreg.inc only succeeds within the registers the CTA was launched with: refuse to
     // launch a build whose per-thread count differs from the split's assumption.
     cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, BS>);
+    e = cudaFuncGetAttributes(&fa, kern);
     if (e != cudaSuccess) return e;
     if (fa.numRegs != C::LAUNCH_REGS) return cudaErrorInvalidConfiguration;
     long long grid = 2LL * num_sms;
-    if (grid > p.units) grid = p.units;
+    if (grid > w.nunits) grid = w.nunits;
     if (grid <= 0) return cudaSuccess;
-    e = cudaMemsetAsync(p.next_unit, 0, sizeof(unsigned int), st);
+    e = cudaMemsetAsync(cm.next_unit, 0, sizeof(unsigned int), st);
     if (e != cudaSuccess) return e;
-    attn_fwd_kernel<D, BS><<<(unsigned)grid, 256, smem, st>>>(tq, tk, tv, p);
+    kern<<<(unsigned)grid, 256, smem, st>>>(tq, tk, tv, w, cm);
     return cudaGetLastError();
 }
 
@@ -473,22 +607,60 @@ cudaError_t attn_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtenso
                      const int32_t *kv_idx, const int32_t *kv_cnt, void *o, long long BH, int N,
                      int d, int bs, float scale, unsigned long long wait_ns, int num_sms,
                      unsigned int *progress, unsigned int *workspace, cudaStream_t st) {
-    AttnParams p;
-    p.progress = progress;
-    p.next_unit = workspace;
-    p.kv_idx = kv_idx;
-    p.kv_cnt = kv_cnt;
-    p.o = reinterpret_cast<__nv_bfloat16 *>(o);
-    p.N = N;
-    p.nbq = (N + bs - 1) / bs;
-    p.nbk = p.nbq;
-    p.units = BH * p.nbq;
-    p.scale_log2 = scale * 1.4426950408889634f;
-    p.wait_ns = wait_ns;
-    if (d == 128 && bs == 128) return launch_attn_t<128, 128>(tq, tk, tv, p, num_sms, st);
-    if (d == 128 && bs == 64) return launch_attn_t<128, 64>(tq, tk, tv, p, num_sms, st);
-    if (d == 64 && bs == 128) return launch_attn_t<64, 128>(tq, tk, tv, p, num_sms, st);
-    if (d == 64 && bs == 64) return launch_attn_t<64, 64>(tq, tk, tv, p, num_sms, st);
+    AttnCommon cm;
+    cm.scale_log2 = scale * 1.4426950408889634f;
+    cm.wait_ns = wait_ns;
+    cm.progress = progress;
+    cm.next_unit = workspace;
+    auto run = [&](auto walk) {
+        using W = decltype(walk);
+        walk.kv_idx = kv_idx;
+        walk.kv_cnt = kv_cnt;
+        walk.o = reinterpret_cast<__nv_bfloat16 *>(o);
+        walk.N = N;
+        walk.nbq = (N + bs - 1) / bs;
+        walk.nbk = walk.nbq;
+        walk.nunits = BH * walk.nbq;
+        return launch_attn_t<W::kD, W::kBS, W>(tq, tk, tv, walk, cm, num_sms, st);
+    };
+    if (d == 128 && bs == 128) return run(BlockWalk<128, 128>{});
+    if (d == 128 && bs == 64) return run(BlockWalk<128, 64>{});
+    if (d == 64 && bs == 128) return run(BlockWalk<64, 128>{});
+    if (d == 64 && bs == 64) return run(BlockWalk<64, 64>{});
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t attn_varlen_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                            const int2 *units, int units_per_head, const int32_t *tiles,
+                            const int32_t *tcnt, int tstride, const int32_t *perm_q, void *o,
+                            long long BH, int N, int Nq, int Cq, int d, float scale,
+                            unsigned long long wait_ns, int num_sms, unsigned int *workspace,
+                            cudaStream_t st, float *part_o, float *part_lse) {
+    AttnCommon cm;
+    cm.scale_log2 = scale * 1.4426950408889634f;
+    cm.wait_ns = wait_ns;
+    cm.progress = nullptr;
+    cm.next_unit = workspace;
+    auto run = [&](auto walk) {
+        using W = decltype(walk);
+        walk.units = units;
+        walk.tiles = tiles;
+        walk.tcnt = tcnt;
+        walk.perm_q = perm_q;
+        walk.o = reinterpret_cast<__nv_bfloat16 *>(o);
+        walk.part_o = part_o;
+        walk.part_lse = part_lse;
+        walk.BH = BH;
+        walk.nunits = BH * units_per_head;
+        walk.N = N;
+        walk.Nq = Nq;
+        walk.Cq = Cq;
+        walk.tstride = tstride;
+        walk.units_per_head = units_per_head;
+        return launch_attn_t<W::kD, 128, W>(tq, tk, tv, walk, cm, num_sms, st);
+    };
+    if (d == 128) return run(TileWalk<128>{});
+    if (d == 64) return run(TileWalk<64>{});
     return cudaErrorInvalidValue;
 }
 

@@ -48,6 +48,7 @@ cudaError_t attn_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtenso
                      int d, int bs, float scale, unsigned long long wait_ns, int num_sms,
                      unsigned int *progress, unsigned int *workspace, cudaStream_t st);
 
+// attention over variable-length tiles (attn.cu, TileWalk); part_o / part_lse select the split form
 cudaError_t attn_varlen_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                             const int2 *units, int units_per_head, const int32_t *tiles,
                             const int32_t *tcnt, int tstride, const int32_t *perm_q, void *o,

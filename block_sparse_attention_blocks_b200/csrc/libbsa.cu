@@ -4,7 +4,6 @@
 #include "select.cu"
 #include "static.cu"
 #include "attn.cu"
-#include "attn_varlen.cu"
 #include "probe.cu"
 #include "capi.cu"
 #include "pipeline.cu"

@@ -16,7 +16,8 @@
 // range), the update step (the mean of each cluster's rows, summed in token order), the
 // centroid scores, the tables of query tiles and key tiles, and the row gather.  Selection runs
 // on the top-p kernel of the block path (top-k = 0) over the scores log|j| + scale mu_q . mu_k,
-// whose softmax is the estimate above; the attention is attn_varlen.cu.
+// whose softmax is the estimate above; the attention is attn.cu's kernel with variable-length
+// tiles (TileWalk).
 #include "bsa_internal.h"
 #include "sparse_attn.h"
 
