@@ -39,7 +39,7 @@
 
 namespace bsa {
 
-// Parameters common to both tile-addressing policies.
+// Parameters common to the tile-addressing policies.
 struct AttnCommon {
     float scale_log2;        // softmax scale * log2(e)
     unsigned long long wait_ns;
@@ -65,7 +65,7 @@ struct AttnOut {
 template <int D, int BS>
 struct BlockWalk {
     static constexpr int kD = D, kBS = BS;
-    static constexpr bool kSplit = false;
+    static constexpr bool kSplit = false, kGroups = false;
     const int32_t *kv_idx;  // [units, nbk] ascending key-block ids, or null for dense
     const int32_t *kv_cnt;  // [units], or null for dense
     __nv_bfloat16 *o;       // [BH, N, D]
@@ -103,7 +103,7 @@ struct BlockWalk {
 template <int D>
 struct TileWalk {
     static constexpr int kD = D;
-    static constexpr bool kSplit = true;
+    static constexpr bool kSplit = true, kGroups = false;
     const int2 *units;      // [BH * units_per_head] {q_row0, q_rows << 16 | cluster}; q_rows = 0: none
     const int32_t *tiles;   // [BH * Cq, tstride] key tiles (k_row0 << 7) | (valid - 1)
     const int32_t *tcnt;    // [BH * Cq] key tiles in each query cluster's list
@@ -155,6 +155,37 @@ struct TileWalk {
         const size_t prow = ((size_t)w.cluster * BH + w.bh) * Nq + orig;
         return AttnOut{o ? o + ((size_t)w.bh * Nq + orig) * D : nullptr,
                        part_o ? part_o + prow * D : nullptr, part_lse ? part_lse + prow : nullptr};
+    }
+};
+
+// Many short independent sequences (W tokens each, stored one after another: Ntot rows in all)
+// packed into 128-row tiles: unit u = rows [u P W, u P W + P W) with P = 128 / W sequences, one
+// key tile over the same rows, and row r of the tile attends only to the keys of its own
+// sequence (a block-diagonal mask in the softmax).
+template <int D>
+struct GroupWalk {
+    static constexpr int kD = D;
+    static constexpr bool kSplit = false, kGroups = true;
+    __nv_bfloat16 *o;  // [Ntot, D]
+    long long nunits;  // ceil(Ntot / per_tile)
+    int Ntot, W, per_tile;  // rows, tokens per sequence, rows per tile (P W)
+
+    __device__ __forceinline__ AttnUnit unit(long long u) const {
+        AttnUnit w;
+        w.bh = 0;
+        w.q0 = (int)(u * per_tile);
+        w.rows = min(per_tile, Ntot - w.q0);
+        w.cnt = 1;
+        w.cluster = 0;
+        w.list = nullptr;
+        return w;
+    }
+    __device__ __forceinline__ int32_t entry(const AttnUnit &w, int) const { return w.q0; }
+    __device__ __forceinline__ KeyTile key(int32_t k0, bool) const {
+        return KeyTile{k0, min(per_tile, Ntot - k0)};
+    }
+    __device__ __forceinline__ AttnOut out(const AttnUnit &w, int r, bool row_ok) const {
+        return AttnOut{o + (size_t)(row_ok ? w.q0 + r : 0) * D, nullptr, nullptr};
     }
 };
 
@@ -467,11 +498,27 @@ __global__ void __launch_bounds__(256, 2)
                 // the whole S row of this thread: BS fp32 scores, one TMEM round trip
                 uint32_t s[BS];
                 tmem_ld_cols<BS>(tSr, s);
-                if (valid < BS) {  // keys past the tile's valid count (warp-uniform branch)
-#pragma unroll
-                    for (int e = 0; e < BS; ++e)
-                        if (e >= valid) s[e] = __float_as_uint(-INFINITY);
+                // keys this row may see: [klo, khi) of the tile (its own sequence for packed
+                // sequences; otherwise the tile's valid keys)
+                int klo = 0, khi = valid;
+                if constexpr (Walk::kGroups) {
+                    if (row_ok) {
+                        klo = (r / walk.W) * walk.W;
+                        khi = min(klo + walk.W, valid);
+                    }
                 }
+                auto mask_keys = [&](uint32_t (&sv)[BS]) {
+                    if constexpr (Walk::kGroups) {
+#pragma unroll
+                        for (int e = 0; e < BS; ++e)
+                            if (e < klo || e >= khi) sv[e] = __float_as_uint(-INFINITY);
+                    } else if (valid < BS) {  // keys past the tile's valid count (warp-uniform)
+#pragma unroll
+                        for (int e = 0; e < BS; ++e)
+                            if (e >= valid) sv[e] = __float_as_uint(-INFINITY);
+                    }
+                };
+                mask_keys(s);
                 // Reference max: the first block of a query block sets it from its own scores.
                 // Later blocks reuse it while their P stays below 2^30 (bf16 and the fp32 sums
                 // have room for that), which the block's row sum shows, so the row max is not
@@ -485,11 +532,7 @@ __global__ void __launch_bounds__(256, 2)
                 if (__any_sync(0xffffffffu, !(ts < kMaxP) || xpoly > kMaxLog2P)) {
                     // rare: S is read again from tensor memory (still intact: P is written below)
                     tmem_ld_cols<BS>(tSr, s);
-                    if (valid < BS) {
-#pragma unroll
-                        for (int e = 0; e < BS; ++e)
-                            if (e >= valid) s[e] = __float_as_uint(-INFINITY);
-                    }
+                    mask_keys(s);
                     const float m_new = fmaxf(m_ref, row_max<BS>(s) * sl2);
                     const float alpha = ex2(m_ref - m_new);  // 1 for rows that keep theirs
                     if (t > 0) {
@@ -627,6 +670,30 @@ cudaError_t attn_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtenso
     if (d == 128 && bs == 64) return run(BlockWalk<128, 64>{});
     if (d == 64 && bs == 128) return run(BlockWalk<64, 128>{});
     if (d == 64 && bs == 64) return run(BlockWalk<64, 64>{});
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t attn_group_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                           void *o, long long Ntot, int W, int d, float scale,
+                           unsigned long long wait_ns, int num_sms, unsigned int *workspace,
+                           cudaStream_t st) {
+    if (W < 1 || W > 128 || Ntot < 1 || Ntot > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+    AttnCommon cm;
+    cm.scale_log2 = scale * 1.4426950408889634f;
+    cm.wait_ns = wait_ns;
+    cm.progress = nullptr;
+    cm.next_unit = workspace;
+    auto run = [&](auto walk) {
+        using W_ = decltype(walk);
+        walk.o = reinterpret_cast<__nv_bfloat16 *>(o);
+        walk.Ntot = (int)Ntot;
+        walk.W = W;
+        walk.per_tile = (128 / W) * W;
+        walk.nunits = (Ntot + walk.per_tile - 1) / walk.per_tile;
+        return launch_attn_t<W_::kD, 128, W_>(tq, tk, tv, walk, cm, num_sms, st);
+    };
+    if (d == 128) return run(GroupWalk<128>{});
+    if (d == 64) return run(GroupWalk<64>{});
     return cudaErrorInvalidValue;
 }
 

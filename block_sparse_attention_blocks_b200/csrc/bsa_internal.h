@@ -48,6 +48,13 @@ cudaError_t attn_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtenso
                      int d, int bs, float scale, unsigned long long wait_ns, int num_sms,
                      unsigned int *progress, unsigned int *workspace, cudaStream_t st);
 
+// attention within short sequences of W tokens stored back to back (Ntot rows), packed 128 / W
+// to a tile with a block-diagonal mask (attn.cu, GroupWalk); W <= 128
+cudaError_t attn_group_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                           void *o, long long Ntot, int W, int d, float scale,
+                           unsigned long long wait_ns, int num_sms, unsigned int *workspace,
+                           cudaStream_t st);
+
 // attention over variable-length tiles (attn.cu, TileWalk); part_o / part_lse select the split form
 cudaError_t attn_varlen_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                             const int2 *units, int units_per_head, const int32_t *tiles,

@@ -6,8 +6,9 @@
 //                                                                            (values Y)
 // The local pass is one dense attention call over B*H*W "heads" of w tokens (a reshape of the
 // [B, H, n, d] tensors, no copy).  Q, K and Y are then regrouped by position, [W, w] -> [w, W]
-// within each (b, h), the global pass is one dense attention call over B*H*w heads of W tokens,
-// and its output is regrouped back into O.  For video with w = the tokens of one latent frame,
+// within each (b, h); the global pass attends within each of the B*H*w sequences of W tokens
+// (for W <= 64 packed 128 / W sequences to a 128-row tile with a block-diagonal mask, else one
+// dense call over B*H*w heads), and its output is regrouped back into O.  For video with w = the tokens of one latent frame,
 // the local pass is spatial attention within a frame and the global pass temporal attention
 // across frames at each spatial position.
 #include "bsa_internal.h"
@@ -94,10 +95,22 @@ extern "C" sa_status sa_squad_attn_fwd(const void *q, const void *k, const void 
     if (e == cudaSuccess) e = bsa::permute_tokens(k, kg, G, W, w, d, sms, st);
     if (e == cudaSuccess) e = bsa::permute_tokens(o, yg, G, W, w, d, sms, st);
     if (e != cudaSuccess) return SA_ERR_CUDA;
-    // global pass: B*H*w heads of W tokens, values Y
-    s = run_attention(qg, kg, yg, nullptr, nullptr, og, 1, (int)heads_global, W, d, 128, scale,
-                      counter, stream);
-    if (s != SA_OK) return s;
+    // global pass: B*H*w sequences of W tokens, values Y.  Short sequences are packed 128 / W to
+    // a tile with a block-diagonal mask; longer ones run as B*H*w heads of the dense kernel.
+    const long long Ntot = heads_global * W;
+    if (W <= 64 && Ntot <= 0x7FFFFFFFLL) {
+        CUtensorMap tq, tk, tv;
+        if (!make_tmap(&tq, qg, 1, (int)Ntot, d, 128) || !make_tmap(&tk, kg, 1, (int)Ntot, d, 128) ||
+            !make_tmap(&tv, yg, 1, (int)Ntot, d, 128))
+            return SA_ERR_CUDA;
+        e = bsa::attn_group_fwd(tq, tk, tv, og, Ntot, W, d, resolve_scale(scale, d), g_wait_ns, sms,
+                                reinterpret_cast<unsigned int *>(counter), st);
+        if (e != cudaSuccess) return SA_ERR_CUDA;
+    } else {
+        s = run_attention(qg, kg, yg, nullptr, nullptr, og, 1, (int)heads_global, W, d, 128, scale,
+                          counter, stream);
+        if (s != SA_OK) return s;
+    }
     // back to token order
     return from_cuda(bsa::permute_tokens(og, o, G, w, W, d, sms, st));
 }

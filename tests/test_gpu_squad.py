@@ -22,7 +22,12 @@ DEV = torch.device("cuda", 0)
 @pytest.mark.parametrize("B,H,N,d,w", [(1, 2, 512, 64, 64),     # 8 windows of one tile
                                        (1, 2, 900, 128, 300),   # windows with a ragged tile
                                        (2, 1, 384, 128, 128),   # 3 windows
-                                       (1, 1, 256, 64, 256)])   # one window: dense attention
+                                       (1, 1, 256, 64, 256),    # one window: dense attention
+                                       # global pass packed 6 sequences of 21 to a tile, the
+                                       # last tile holding 2
+                                       (1, 2, 2100, 128, 100),
+                                       (1, 1, 1024, 64, 16),    # 64-token sequences, 2 per tile
+                                       (1, 1, 1400, 64, 20)])   # 70-token sequences: unpacked
 def test_squad_parity(orc, B, H, N, d, w):
     rng = np.random.default_rng(N + w)
     q, k, v = (f32_to_bf16_bits(rng.standard_normal((B, H, N, d)).astype(np.float32))
