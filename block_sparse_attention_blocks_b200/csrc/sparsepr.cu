@@ -14,13 +14,14 @@
 //
 // Steps (one stream, no host synchronisation):
 //   1. O_s by the block-sparse attention kernel;
-//   2. the probe rows of Q gathered into [BH, m, d]; their exact outputs by the variable-length
-//      attention kernel with one query cluster covering the m rows and one key list covering
-//      every key (128-key tiles, the last one ragged);
-//   3. [O_s[P] | R] in fp64; the Gram products tiled over CTAs; W by one CTA per head in fp64:
-//      the normal equations of the smaller side, Cholesky in shared memory with a ridge of 1e-12
-//      times the mean diagonal (which keeps a rank-deficient X solvable and approximates the
-//      pseudo-inverse's minimum-norm choice);
+//   2. the probe rows of Q gathered into [BH, m, d]; their exact outputs by the attention kernel
+//      over variable-length tiles in its split form: the keys of each head cut into S runs of
+//      128-key tiles (enough units to fill the GPU), each run's fp32 output and log2-sum-exp
+//      combined in fp64 (probe_merge_kernel);
+//   3. [O_s[P] | R] in fp64; the Gram products tiled over CTAs; W by d / 32 CTAs per head in
+//      fp64 (32 right-hand-side columns each): the normal equations of the smaller side,
+//      Cholesky in shared memory with a ridge of 1e-12 times the mean diagonal (which keeps a
+//      rank-deficient X solvable and approximates the pseudo-inverse's minimum-norm choice);
 //   4. O += [O, 1] W in place on the bf16 output, on the tensor cores (W in two bf16 parts).
 #include "bsa_internal.h"
 #include "sparse_attn.h"

@@ -306,9 +306,11 @@ sa_status sa_block_sparse_attn_fwd_noalloc(const void *q, const void *k, const v
  * q, k, v, kv_idx, kv_cnt, o, bs, scale: as sa_block_sparse_attn_fwd.
  * workspace: device memory of sa_sparsepr_workspace_bytes(B, H, N, d, m) bytes, 16-byte
  *           aligned, owned by the caller (probe rows, their exact outputs, the fp64 fit).
- * Arithmetic: the sparse and exact outputs in bf16 (fp32 accumulation on the tensor cores), the
+ * Arithmetic: the sparse output in bf16 and the probes' exact outputs in fp32 (fp32
+ * accumulation on the tensor cores; the exact outputs combined from runs of keys in fp64), the
  * fit in fp64 (normal equations of the smaller side, Cholesky with a ridge of 1e-12 times the
- * mean diagonal), the correction in fp32 rounded to bf16 in place in o.
+ * mean diagonal), the correction [O_s, 1] W on the tensor cores in fp32 with W's first d rows
+ * split into two bf16 parts (relative error 2^-17), rounded to bf16 once, in place in o.
  */
 sa_status sa_sparsepr_attn_fwd(const void *q, const void *k, const void *v,
                                const int32_t *kv_idx, const int32_t *kv_cnt,
