@@ -1,8 +1,8 @@
 """GPU parity of SparsePR's probe-fitted residual correction (page "Partition the Support,
 Reconstruct the Residual", abstract and summary section 3) against the oracle, through the C ABI.
 
-The GPU fits on bf16 sparse and exact probe outputs (fp64 solve) and writes bf16; the oracle
-works in fp64 throughout.  The comparison is the attention tolerance on every row of every head,
+The GPU fits on the bf16 sparse output and fp32 exact probe outputs (fp64 solve) and writes
+bf16; the oracle works in fp64 throughout.  The comparison is the attention tolerance on every row of every head,
 for probe counts well below and well above d + 1 (where the fit is well conditioned: with about
 d + 1 probes the square system amplifies the bf16 rounding of its inputs, so that case is
 checked through the properties that hold at any precision instead: the probe rows come out at
