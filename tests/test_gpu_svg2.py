@@ -94,11 +94,14 @@ def test_kmeans_matches_oracle_on_separated_clusters(orc, d, N, C, iters):
         assert np.array_equal(cz[h], np.bincount(assign[h], minlength=C))
 
 
-def test_kmeans_assignment_is_the_nearest_centroid(orc):
+@pytest.mark.parametrize("d,C", [(128, 64),
+                                 (64, 300),    # three 128-centroid tiles, merged per token
+                                 (128, 257)])  # a last tile of one centroid
+def test_kmeans_assignment_is_the_nearest_centroid(orc, d, C):
     # overlapping clusters: ties within rounding may go either way; every choice must be
     # nearest within 1e-5 relative, and with no update step the centroids stay as given
-    rng = np.random.default_rng(5)
-    BH, N, d, C = 2, 2000, 128, 64
+    rng = np.random.default_rng(5 + C)
+    BH, N = 2, 2000
     bits = f32_to_bf16_bits(rng.standard_normal((BH, N, d)).astype(np.float32))
     init = rng.standard_normal((BH, C, d)).astype(np.float32)
     cent = torch.from_numpy(init.reshape(1, BH, C, d)).to(DEV)
