@@ -8,9 +8,8 @@
 // and E the exact outputs of the probe rows:
 //   X = [O_s[P], 1]  (m x (d + 1)),   R = E - O_s[P]  (m x d)
 //   W = X^+ R, the minimum-norm least-squares map, and O = O_s + [O_s, 1] W for every row.
-// At the full numerical rank this is the page's fit of the residuals in their observed output
-// subspace: the minimum-norm least-squares map of the residuals is already a combination of the
-// rows of R.
+// At the full numerical rank this is the page's fit limited to the span of the residuals: the
+// minimum-norm least-squares map of the residuals is already a combination of the rows of R.
 //
 // Steps (one stream, no host synchronisation):
 //   1. O_s by the block-sparse attention kernel;

@@ -298,7 +298,7 @@ sa_status sa_block_sparse_attn_fwd_noalloc(const void *q, const void *k, const v
  * "Partition the Support, Reconstruct the Residual: Training-Free Sparse Attention for Video
  * Generation and World Models", abstract and summary section 3: a few probe queries are computed
  * exactly, and their residuals against the sparse output are fitted by an affine map of the
- * sparse output in the observed output subspace, which then corrects every row).
+ * sparse output, restricted to the span of those residuals, which then corrects every row).
  *   O_s = sa_block_sparse_attn_fwd(q, k, v, kv_idx, kv_cnt);  per head, with P = probes[b, h, :]
  *   X = [O_s[P], 1], R = exact(P) - O_s[P], W = X^+ R (minimum norm), O = O_s + [O_s, 1] W.
  * probes  : [B, H, m] int32 token ids in [0, N) chosen by the caller (ids outside are clamped);

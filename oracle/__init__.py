@@ -300,17 +300,17 @@ def dense_attention(q_bits, k_bits, v_bits, scale: float, rows=None):
 # ---------------------------------------------------------------------------------------------
 # Probe-fitted residual reconstruction (page "Partition the Support, Reconstruct the Residual:
 # Training-Free Sparse Attention for Video Generation and World Models", the abstract and the
-# summary's section 3).  The page gives this step in one sentence: a few exact query rows
-# calibrate, for each call, an affine correction computed from the sparse output, confined to
-# the output subspace the probe residuals span.  The steps below are the plainest reading of it;
-# their library steps are numpy's SVD and least squares.
+# summary's section 3).  The page describes this step in a single sentence: per call, a handful
+# of rows computed exactly fix an affine correction of the sparse output, limited to the
+# directions their residuals occupy.  The steps below are the plainest reading of it; their
+# library steps are numpy's SVD and least squares.
 # ---------------------------------------------------------------------------------------------
 def probe_fit_correction(o_sparse, probes, exact, rtol: float = 1e-9, rank=None):
     """One head of one call.  o_sparse [n, d]: the sparse attention output; probes [m]: probe
     query rows; exact [m, d]: their exact (dense) attention outputs.
 
       R  = exact - o_sparse[probes]                the probe residuals
-      Bs = orthonormal basis [d, r] of the observed output subspace: the right singular vectors
+      Bs = orthonormal basis [d, r] of the residual subspace: the right singular vectors
            of R whose singular value exceeds rtol times the largest (its numerical row space),
            or only the leading `rank` of them when rank is given
       A  = argmin || [o_sparse[probes], 1] A - R Bs ||   over A [(d + 1), r]; the minimum-norm
