@@ -98,3 +98,41 @@ def test_sparsepr_full_mask_is_dense(orc):
     for h in range(B * H):
         dense = orc.dense_attention(q[h][None], k[h][None], v[h][None], 1 / math.sqrt(d))
         compare_attention(got[h], dense.reshape(N, d))
+
+
+@pytest.mark.slow
+def test_sparsepr_full_shape_sampled_rows(orc):
+    # the bench's SparsePR configuration on two heads of the Wan2.1-14B-720p workload (N = 75600,
+    # d = 128, block 128, k = 30, p = 0.9, 256 seeded probes per head, keys split into runs): the
+    # oracle fits W in fp64 from the sparse (GPU selection) and dense outputs of the probe rows,
+    # computed row by row, and corrects a seeded sample of rows (first, last, random)
+    from block_sparse_attention_blocks_b200 import workloads as W
+    from dataclasses import replace
+    w = W.get("wan14b_720p")
+    heads = [0, 1]
+    qb, kb, vb = W.make_qkv(w, heads=heads)
+    wh = replace(w, B=1, H=len(heads))
+    BH, N, d, bs, nb = len(heads), w.N, w.d, w.bs, w.nb
+    q, k, v = _dev(qb), _dev(kb), _dev(vb)
+    _, _, mask, idx, cnt = bsa.pool_select_topk_topp(q, k, bs, w.topk, w.topp)
+    rng = np.random.default_rng(11)
+    m = 256
+    probes = np.stack([np.sort(rng.choice(N, m, replace=False)) for _ in range(BH)]).astype(np.int32)
+    o = bsa.sparsepr_attn_fwd(q, k, v, idx, cnt, torch.from_numpy(probes.reshape(1, BH, m)).to(DEV), bs)
+    torch.cuda.synchronize()
+    assert bsa.device_error() == 0
+    got = _host(o).reshape(BH, N, d)
+    gmask = mask.cpu().numpy().reshape(BH, nb, nb)
+    scale = 1 / math.sqrt(d)
+    for h in range(BH):
+        samples = np.unique(np.concatenate([[0, N - 1], rng.choice(N, 30, replace=False)]))
+        rows = np.concatenate([probes[h], samples])
+        blocks = sorted({int(t) // bs for t in rows})
+        ob = orc.masked_attention(qb[0, h][None], kb[0, h][None], vb[0, h][None],
+                                  gmask[h][None], bs, scale, [(0, i) for i in blocks])
+        pos = {i: s for s, i in enumerate(blocks)}
+        o_rows = np.stack([ob[pos[int(t) // bs], int(t) % bs] for t in rows])
+        exact = orc.dense_attention(qb[0, h][None], kb[0, h][None], vb[0, h][None], scale,
+                                    rows=[(0, int(t)) for t in probes[h]])
+        corrected, _, _ = orc.probe_fit_correction(o_rows, np.arange(m), exact)
+        compare_attention(got[h][samples], corrected[m:])
